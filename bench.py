@@ -1,0 +1,367 @@
+#!/usr/bin/env python
+"""Attention forward throughput on B200: TFLOPS and fraction of dense BF16 peak.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+A step is one attn_fwd call over the whole workload (every query row of every
+head), inputs resident in HBM. The default workload is the long video
+self-attention, BF16 Q,K,V [1, 20480, 56, 128], non-causal: 12.03 TFLOP per
+step. Its inputs (881 MB) exceed the 126 MB L2, so no flush is needed between
+steps. Timing: W untimed steps, then K steps between CUDA events on the
+launching stream, with a barrier and a device synchronize on both sides; the
+max over ranks is reported. With N > 1 (torchrun), every rank runs its own
+instance of the workload (independent problems: weak scaling, no data-path
+collective; NCCL carries only the timing reduction).
+
+Also reported on the same JSON line:
+  roofline      achieved TFLOP/s of the attention kernel (algorithmic FLOPs per
+                launch / mean CUDA-event launch time) against the measured
+                dense BF16 peak of this pool (MEASURED_PEAKS.json);
+  e2e           the same metric through attn_fwd_host: pinned host inputs
+                copied in, the forward, the output copied back, every step;
+  cpu_baseline  the FP64 oracle timed on this host's cores on a bounded sample
+                of the same workload (rank 0, N = 1);
+  clocks        SM clock samples taken by nvidia-smi during the timed region.
+
+--impl reference times the FP64 CPU oracle (the only reference this build has)
+on the same workload, metric and unit, each step a bounded sample of it.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd TFLOPS on 1 B200 and % of dense BF16 tensor-core peak"
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "attn_fwd_video_20480x56x128.md")
+KERNEL_SOURCES = [os.path.join(ROOT, "head_attention_streaming_b200", "csrc", f)
+                  for f in ("attn_fwd_sm100.cu", "sm100_ptx.cuh", "tmem_ldst.inc")]
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="video_20480x56x128")
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="minimum CPU time spent timing the oracle sample")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per launch from the committed ncu summary, if it matches this kernel."""
+    try:
+        text = open(PROFILE_SUMMARY).read()
+    except OSError:
+        return None, "no ncu summary"
+    m_bytes = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    m_hash = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", text)
+    if not m_bytes or not m_hash:
+        return None, "summary lacks traffic"
+    if m_hash.group(1) != kernel_source_hash():
+        return None, "kernel changed since the ncu capture"
+    return float(m_bytes.group(1)), "ncu"
+
+
+class ClockSampler:
+    """nvidia-smi SM clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.err = None
+        try:
+            import torch
+            ident = str(device_index)
+            try:
+                uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+                ident = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            except Exception:
+                pass
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", ident],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception as e:  # no nvidia-smi: report why
+            self.err = str(e)
+
+    def stop(self):
+        if self.proc is None:
+            return {"error": self.err or "nvidia-smi unavailable"}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r.split(",") for r in out.strip().splitlines() if r.count(",") >= 8]
+        sm, mx, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+                power.append(float(r[3]))
+            except ValueError:
+                continue
+            for name, val in zip(names, r[5:9]):
+                if val.strip().lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"error": "no samples"}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": max(power) if power else None}
+
+
+def oracle_sample_tflops(w, q, k, v, seconds: float):
+    """FP64 oracle on the workload's seeded sample rows, repeated for >= `seconds`."""
+    import numpy as np
+
+    import oracle
+    from head_attention_streaming_b200 import inputs
+    n_rows = w.sample_rows or min(256, w.Lq)
+    rows = inputs.sample_rows(w.Lq, n_rows, seed=w.seed * 1000)
+    hkv = 0
+    qh = q[:, :, 0:1].to(dtype=q.dtype).double().numpy()
+    kh = k[:, :, hkv:hkv + 1].double().numpy()
+    vh = v[:, :, hkv:hkv + 1].double().numpy()
+    if w.mask == 1:   # causal: FLOPs of the visible prefix of each sampled row
+        f_once = sum(4.0 * min(w.Lk, w.kv_offset + int(i) + 1) * w.d for i in rows) * w.B
+    else:
+        f_once = 4.0 * w.B * len(rows) * min(w.Lk, w.kv_offset + w.Lq if w.mask == 2 else w.Lk) * w.d
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.attention_fwd(qh, kh, vh, w.scale, w.mask, w.kv_offset, rows=rows)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    threads = os.cpu_count()
+    try:
+        from threadpoolctl import threadpool_info
+        info = [i for i in threadpool_info() if i.get("user_api") == "blas"]
+        if info:
+            threads = max(i.get("num_threads", 1) for i in info)
+    except Exception:
+        pass
+    sample = (f"{len(rows)} seeded query rows of head 0 x {reps} repetitions "
+              f"(B={w.B}, Lk={w.Lk}, d={w.d}), numpy float64")
+    return f_once * reps / el / 1e12, threads, sample, el
+
+
+def workload_config(w, n_gpus):
+    mask = {0: "none", 1: "causal", 2: "chunk"}[w.mask]
+    in_bytes = 2 * w.B * w.d * (w.Lq * w.Hq + 2 * w.Lk * w.Hkv)
+    return {"workload": w.name, "B": w.B, "Lq": w.Lq, "Lk": w.Lk, "Hq": w.Hq, "Hkv": w.Hkv,
+            "d": w.d, "mask": mask, "kv_offset": w.kv_offset, "scale": w.scale,
+            "flops_per_step": w.flops(),
+            "l2": (f"inputs {in_bytes / 1e6:.0f} MB vs 126 MB L2: "
+                   + ("larger than L2, no flush" if in_bytes > 126e6 else "L2 flushed between steps")),
+            "parallelism": f"replicas x{n_gpus}" if n_gpus > 1 else "single GPU"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from head_attention_streaming_b200 import inputs
+    w = inputs.WORKLOADS[args.workload]
+    q, k, v = inputs.workload_inputs(w)
+    per_step = max(0.05, min(1.0, 120.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample_tflops(w, q, k, v, per_step)
+    vals, secs = [], 0.0
+    for _ in range(args.steps):
+        tf, threads, sample, el = oracle_sample_tflops(w, q, k, v, per_step)
+        vals.append(tf)
+        secs += el
+    value = statistics.mean(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, 1),
+        "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": threads, "kind": "oracle",
+                         "sample": sample + f"; each step >= {per_step:.2f} s"},
+        "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    import head_attention_streaming_b200 as hasb
+    from head_attention_streaming_b200 import inputs
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    w = inputs.WORKLOADS[args.workload]
+    q_cpu, k_cpu, v_cpu = inputs.make_qkv(w.B, w.Lq, w.Lk, w.Hq, w.Hkv, w.d, w.torch_dtype,
+                                          seed=w.seed + 7919 * rank, qk_rmsnorm=w.qk_rmsnorm)
+    q, k, v = q_cpu.cuda(), k_cpu.cuda(), v_cpu.cuda()
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.Lq), dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        hasb.attn_fwd(q, k, v, scale=w.scale, causal=w.mask, kv_offset=w.kv_offset, out=o, lse=lse)
+
+    # ---- kernel-only timed region (inputs resident in HBM)
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    time.sleep(0.3)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for a, b in ev:
+        a.record(stream)
+        step()
+        b.record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    clock_info = clocks.stop()
+    fault = hasb.device_fault(clear=True)
+    ms_total = t_start.elapsed_time(t_end)
+    launch_ms = [a.elapsed_time(b) for a, b in ev]
+    ms_step = ms_total / args.steps
+    if world > 1:
+        t = torch.tensor([ms_step], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step = float(t.item())
+    value = world * w.flops() / (ms_step * 1e-3) / 1e12
+
+    # ---- end to end through the host-buffer C ABI entry point
+    e2e = None
+    if args.e2e_steps > 0:
+        qh, kh, vh = q_cpu.pin_memory(), k_cpu.pin_memory(), v_cpu.pin_memory()
+        oh = torch.empty_like(q_cpu).pin_memory()
+        lh = torch.empty((w.B, w.Hq, w.Lq), dtype=torch.float32).pin_memory()
+        qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+        def e2e_step():
+            hasb.attn_fwd_host(qh, kh, vh, oh, lh, qd, kd, vd, o, lse, scale=w.scale,
+                               causal=w.mask, kv_offset=w.kv_offset)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e_ms = e0.elapsed_time(e1) / args.e2e_steps
+        if world > 1:
+            t = torch.tensor([e_ms], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
+        d2h = oh.numel() * oh.element_size() + lh.numel() * lh.element_size()
+        e2e = {"value": world * w.flops() / (e_ms * 1e-3) / 1e12, "unit": "TFLOPS",
+               "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "path": "attn_fwd_host (pinned host -> device, forward, device -> host), one stream"}
+
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    launch_avg = statistics.mean(launch_ms)
+    achieved = w.flops() / (launch_avg * 1e-3) / 1e12
+    traffic, traffic_src = profiled_traffic()
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": traffic,
+                "peak_source": f"bf16_tflops (burst) of {peak_src}",
+                "frac_of_sustained": achieved / peak_sus, "traffic_source": traffic_src,
+                "kernel": "attn_fwd_sm100_kernel", "launch_ms_mean": launch_avg,
+                "launch_ms_min": min(launch_ms), "launch_ms_max": max(launch_ms)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tf, threads, sample, _ = oracle_sample_tflops(w, q_cpu, k_cpu, v_cpu, args.cpu_seconds)
+        cpu = {"value": tf, "unit": "TFLOPS", "cores": threads, "kind": "oracle", "sample": sample}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": w.dtype, "data": "synthetic: seeded N(0,1) inputs of the workload's shape",
+            "config": workload_config(w, world),
+            "pct_of_peak": 100.0 * value / world / peak,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": args.steps, "clocks": clock_info, "device_fault_bits": fault,
+        }
+        print(json.dumps(line))
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,17 @@
+"""Fused scaled-dot-product attention forward for NVIDIA B200 (sm_100a).
+
+The computation runs in ``libattn_sm100.so`` (C ABI in ``include/attn.h``);
+``binding`` marshals torch tensors into it. The library is loaded on first use,
+so importing ``head_attention_streaming_b200.inputs`` needs no GPU.
+"""
+
+from .binding import (ATTN_ERR_CUDA, ATTN_ERR_INVALID_ARG, ATTN_ERR_TIMEOUT, ATTN_ERR_UNSUPPORTED,
+                      ATTN_OK, MASK_CAUSAL, MASK_CHUNK, MASK_NONE, AttnError, attn_fwd,
+                      attn_fwd_host,
+                      device_fault, lib, library_path, selftest_mma, selftest_wait_timeout,
+                      set_wait_timeout_ns, status_string)
+
+__all__ = ["attn_fwd", "attn_fwd_host", "AttnError", "lib", "library_path", "status_string", "device_fault",
+           "set_wait_timeout_ns", "selftest_mma", "selftest_wait_timeout", "ATTN_OK",
+           "ATTN_ERR_INVALID_ARG", "ATTN_ERR_UNSUPPORTED", "ATTN_ERR_CUDA", "ATTN_ERR_TIMEOUT",
+           "MASK_NONE", "MASK_CAUSAL", "MASK_CHUNK"]

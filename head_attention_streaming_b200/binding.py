@@ -1,0 +1,186 @@
+"""ctypes binding of the C ABI in include/attn.h.
+
+Argument marshalling only: tensors are turned into device pointers and sizes,
+the status code is turned into an exception. Every step of the computation runs
+in the CUDA library; there is no fallback path. If the library has not been
+built, every call raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_SO_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libattn_sm100.so")
+_LIB = None
+
+ATTN_OK = 0
+ATTN_ERR_INVALID_ARG = 1
+ATTN_ERR_UNSUPPORTED = 2
+ATTN_ERR_CUDA = 3
+ATTN_ERR_TIMEOUT = 4
+
+MASK_NONE = 0
+MASK_CAUSAL = 1
+MASK_CHUNK = 2
+
+DTYPE_CODES = {torch.bfloat16: 0, torch.float16: 1}
+
+# name -> (restype, argtypes) of every exported function
+_SIGNATURES = {
+    "attn_fwd": (ctypes.c_int, [ctypes.c_void_p] * 5 + [ctypes.c_int] * 6 +
+                 [ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
+    "attn_fwd_host": (ctypes.c_int, [ctypes.c_void_p] * 10 + [ctypes.c_int] * 6 +
+                      [ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
+    "attn_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "attn_device_fault": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint), ctypes.c_int]),
+    "attn_set_wait_timeout_ns": (ctypes.c_int, [ctypes.c_ulonglong]),
+    "attn_selftest_mma": (ctypes.c_int, [ctypes.c_void_p] * 5 + [ctypes.c_int, ctypes.c_void_p]),
+    "attn_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_ulonglong, ctypes.c_void_p]),
+}
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: status {status} ({status_string(status)})")
+
+
+def library_path() -> str:
+    return _SO_PATH
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library (loaded on first use)."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(_SO_PATH):
+            raise RuntimeError(
+                f"CUDA library {_SO_PATH} is missing; build it with "
+                "`python -m head_attention_streaming_b200.build`")
+        L = ctypes.CDLL(_SO_PATH)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _LIB = L
+    return _LIB
+
+
+def status_string(status: int) -> str:
+    try:
+        return lib().attn_status_string(int(status)).decode()
+    except Exception:  # library missing: still format the error
+        return "unknown"
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream, device) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, scale: float | None = None,
+             causal: int = MASK_NONE, kv_offset: int = 0, out: torch.Tensor | None = None,
+             lse: torch.Tensor | None = None, return_lse: bool = True, stream=None):
+    """Fused attention forward through ``attn_fwd`` of the C ABI.
+
+    q: [B, Lq, Hq, d]; k, v: [B, Lk, Hkv, d]; CUDA, contiguous, bf16 or fp16.
+    causal: 0 none, 1 causal (key j <= kv_offset + i), 2 streaming chunk
+    (key j < kv_offset + Lq). Returns ``(out, lse)`` with out [B, Lq, Hq, d]
+    in q's dtype and lse [B, Hq, Lq] float32 (None if return_lse is False and
+    no lse buffer was given).
+    """
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_cuda or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError(f"{name} must be a contiguous 4-D CUDA tensor")
+    if q.dtype not in DTYPE_CODES or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must share one dtype, bf16 or fp16")
+    if k.shape != v.shape:
+        raise ValueError("k and v must have the same shape")
+    B, Lq, Hq, d = q.shape
+    Bk, Lk, Hkv, dk = k.shape
+    if Bk != B or dk != d:
+        raise ValueError("batch and head_dim of q and k/v must match")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    elif out.shape != q.shape or out.dtype != q.dtype or not out.is_contiguous() or not out.is_cuda:
+        raise ValueError("out must be a contiguous CUDA tensor shaped and typed like q")
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
+    elif lse is not None and (lse.shape != (B, Hq, Lq) or lse.dtype != torch.float32
+                              or not lse.is_contiguous() or not lse.is_cuda):
+        raise ValueError("lse must be a contiguous float32 CUDA tensor [B, Hq, Lq]")
+    st = lib().attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Lq, Lk, Hq, Hkv, d,
+                        float(scale), int(causal), int(kv_offset), DTYPE_CODES[q.dtype],
+                        _stream_handle(stream, q.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fwd")
+    return out, lse
+
+
+def attn_fwd_host(q_host, k_host, v_host, o_host, lse_host, q_dev, k_dev, v_dev, o_dev, lse_dev, *,
+                  scale: float | None = None, causal: int = MASK_NONE, kv_offset: int = 0,
+                  stream=None) -> None:
+    """Queue host->device copies of q, k, v, the forward, and device->host copies of
+    o (and lse) on ``stream`` through ``attn_fwd_host`` of the C ABI.
+
+    Host tensors should be pinned CPU tensors; device tensors are the caller's
+    staging buffers of the same shapes. Returns once queued.
+    """
+    B, Lq, Hq, d = q_host.shape
+    _, Lk, Hkv, _ = k_host.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    for t in (q_host, k_host, v_host, o_host):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("host operands must be contiguous CPU tensors")
+    for t in (q_dev, k_dev, v_dev, o_dev):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("device buffers must be contiguous CUDA tensors")
+    if q_host.dtype not in DTYPE_CODES:
+        raise ValueError("dtype must be bf16 or fp16")
+    st = lib().attn_fwd_host(_ptr(q_host), _ptr(k_host), _ptr(v_host), _ptr(o_host), _ptr(lse_host),
+                             _ptr(q_dev), _ptr(k_dev), _ptr(v_dev), _ptr(o_dev), _ptr(lse_dev),
+                             B, Lq, Lk, Hq, Hkv, d, float(scale), int(causal), int(kv_offset),
+                             DTYPE_CODES[q_host.dtype], _stream_handle(stream, q_dev.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fwd_host")
+
+
+def device_fault(clear: bool = True) -> int:
+    """Synchronize the device and return (and optionally clear) the fault bits."""
+    bits = ctypes.c_uint(0)
+    st = lib().attn_device_fault(ctypes.byref(bits), 1 if clear else 0)
+    if st not in (ATTN_OK, ATTN_ERR_TIMEOUT):
+        raise AttnError(st, "attn_device_fault")
+    return int(bits.value)
+
+
+def set_wait_timeout_ns(ns: int) -> None:
+    lib().attn_set_wait_timeout_ns(int(ns))
+
+
+def selftest_mma(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor):
+    """One 128x128 tile through the tensor-core path: returns (S, O) float32."""
+    s_out = torch.empty((128, 128), dtype=torch.float32, device=q.device)
+    o_out = torch.empty((128, 128), dtype=torch.float32, device=q.device)
+    st = lib().attn_selftest_mma(_ptr(q), _ptr(k), _ptr(v), _ptr(s_out), _ptr(o_out),
+                                 DTYPE_CODES[q.dtype], _stream_handle(None, q.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_selftest_mma")
+    return s_out, o_out
+
+
+def selftest_wait_timeout(timeout_ns: int, device=None) -> int:
+    """Status of a launch whose only wait can never complete (expect ATTN_ERR_TIMEOUT)."""
+    return int(lib().attn_selftest_wait_timeout(int(timeout_ns), _stream_handle(None, device)))

@@ -1,0 +1,925 @@
+// Fused attention forward for B200 (sm_100a): TMA-fed K/V ring, tcgen05 MMAs
+// accumulating in tensor memory, warp-specialised load / MMA / softmax roles,
+// exp2 online softmax with lazy O rescaling, mask-tile skipping, GQA indexing.
+//
+// What is computed: the per-head scaled dot-product attention of the
+// flashdreams.accelerated developer guide ("Multi Head Attention Definition",
+// the equation for A_h), O = softmax(scale * Q K^T + mask) V, for token-major
+// [B, L, H, d] tensors, plus the per-row log-sum-exp. The skill page
+// "optimizing-attention-flash" ("Quick start") names the IO-aware tiling this
+// kernel uses: scores never leave the chip; each KV tile updates a running row
+// max / row sum and the output accumulator (the exact online rewrite of the
+// softmax).
+//
+// CTA organisation (one persistent CTA per SM, 384 threads):
+//   warps 0-3   softmax for query tile 0 (rows r0 .. r0+127 of a work unit)
+//   warps 4-7   softmax for query tile 1 (rows r0+128 .. r0+255)
+//   warp  8     TMA producer: Q tiles, then K_0, V_0, K_1, V_1, ... into a ring
+//   warp  9     MMA issuer (one thread): S_t = Q_t K^T and O_t += P_t V
+//   warps 10-11 idle
+// A work unit is (batch, query head, 256-row pair of query tiles). Tensor
+// memory holds S_0, S_1 (128 fp32 columns each, P aliased as packed 16-bit in
+// the first 64 columns) and O_0, O_1 (d columns each).
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "attn.h"
+#include "sm100_ptx.cuh"
+
+namespace hasb {
+
+// Device fault word: bit set by a kernel whose bounded wait ran out.
+__device__ unsigned int g_fault_bits = 0;
+
+enum FaultBit : unsigned int {
+  kFaultLoadQEmpty = 1u << 0,
+  kFaultLoadKvEmpty = 1u << 1,
+  kFaultMmaQFull = 1u << 2,
+  kFaultMmaKvFull = 1u << 3,
+  kFaultMmaPFull = 1u << 4,
+  kFaultSoftmaxSFull = 1u << 5,
+  kFaultSoftmaxOFull = 1u << 6,
+  kFaultSelftest = 1u << 8,
+};
+
+constexpr int kThreads = 384;
+// Register split: 384 threads x 168 launch registers = 64512. The producer
+// warpgroup (warps 8-11) drops to 56, the two softmax warpgroups rise to 224:
+// 128 x 56 + 256 x 224 = 64512.
+constexpr int kRegsProducer = 56;
+constexpr int kRegsSoftmax = 224;
+constexpr int kTileRows = 128;         // query rows per softmax tile = keys per KV tile
+constexpr float kRescaleTau = 8.0f;    // lazy rescale threshold, log2 units (P <= 256)
+constexpr float kLn2 = 0.69314718055994531f;
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int D>
+struct Cfg {
+  static constexpr int kChunks = D / 64;              // 128-byte swizzle chunks per row
+  static constexpr int kChunkBytes = kTileRows * 128;  // one chunk of a 128-row tile
+  static constexpr int kTileBytes = kTileRows * D * 2;
+  static constexpr int kStages = (D == 128) ? 4 : 8;   // K/V ring depth (128 KB)
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffKV = 2 * kTileBytes;
+  static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
+  static constexpr int kSmemBytes = kOffBar + 512 + 1024;  // barriers + 1 KB alignment slack
+  // tensor-memory columns of S_t (P_t aliased) and O_t
+  static __device__ __forceinline__ uint32_t col_s(int t) { return t ? 128u : 0u; }
+  static __device__ __forceinline__ uint32_t col_o(int t) { return t ? 256u + D : 256u; }
+  static constexpr uint32_t kTmemCols = 512;
+};
+
+// barrier slots (8 bytes each) in the barrier area
+enum Bar : int {
+  kBarQFull = 0,    // [2] TMA -> MMA: Q tile t landed
+  kBarQEmpty = 2,   // [2] MMA -> TMA: last S_t of the unit done, Q tile t reusable
+  kBarSFull = 4,    // [2] MMA -> softmax t: S_t ready (also: previous PV_t done)
+  kBarPFull = 6,    // [2] softmax t -> MMA: P_t written (128 arrivals)
+  kBarOFull = 8,    // [2] MMA -> softmax t: O_t final for the unit
+  kBarDrain = 10,   //     MMA abort path: all issued MMAs done
+  kBarKvFull = 16,  // [kStages] TMA -> MMA
+  kBarKvEmpty = 24, // [kStages] MMA -> TMA
+};
+
+struct FwdParams {
+  void* o;
+  float* lse;
+  int B, Lq, Lk, Hq, Hkv, group, kv_offset;
+  int kv_limit;      // keys visible to every row (masks 0 and 2): Lk or kv_offset + Lq
+  int n_pairs;       // ceil(Lq / 256)
+  int n_units;       // B * Hq * n_pairs
+  float sl2;         // scale * log2(e)
+  unsigned long long timeout_ns;
+};
+
+struct Unit {
+  int b, hq, hkv, r0, n0, n1;  // n_t: KV tiles visited by query tile t
+};
+
+__device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+// Work unit u -> (b, hq, row pair). Query heads of one GQA group are adjacent
+// and the row pairs of one head are adjacent, so CTAs running together read
+// the same K/V head (L2 reuse). Causal units run longest first.
+template <bool CAUSAL>
+__device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
+  Unit x;
+  int pt = u % p.n_pairs;
+  int t = u / p.n_pairs;
+  int g = t % p.group;
+  t /= p.group;
+  x.hkv = t % p.Hkv;
+  x.b = t / p.Hkv;
+  x.hq = x.hkv * p.group + g;
+  if (CAUSAL) pt = p.n_pairs - 1 - pt;
+  x.r0 = pt * 2 * kTileRows;
+  if (CAUSAL) {
+    x.n0 = cdiv(min(p.Lk, p.kv_offset + x.r0 + kTileRows), kTileRows);
+    x.n1 = cdiv(min(p.Lk, p.kv_offset + x.r0 + 2 * kTileRows), kTileRows);
+  } else {
+    x.n0 = x.n1 = cdiv(p.kv_limit, kTileRows);
+  }
+  return x;
+}
+
+// Bounded barrier wait. Fast path: one probe. Slow path: poll until the phase
+// completes, another role has aborted, or the time limit passes (then record
+// `bit`, raise the CTA's abort flag and return false).
+__device__ __forceinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                            unsigned int bit, unsigned long long timeout_ns) {
+  const uint64_t t0 = global_timer_ns();
+  // iteration cap as a second bound, should the timer not advance
+  const unsigned long long max_iters = (timeout_ns >> 4) + (1ull << 20);
+  for (unsigned long long it = 0;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (((it & 63u) == 63u && global_timer_ns() - t0 > timeout_ns) || it > max_iters) {
+      atomicOr(&g_fault_bits, bit);
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          unsigned int bit, unsigned long long timeout_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, abort_flag, bit, timeout_ns);
+}
+
+// Abort path: wait a short, fixed time for a phase, ignoring the abort flag.
+__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 0; !mbar_try_wait(bar, parity); ++it) {
+    if (global_timer_ns() - t0 > 200000000ull || it > (1u << 24)) return;  // ~200 ms
+  }
+}
+
+// S[tmem] = Q K^T over head_dim D: D/16 MMAs of 128x128x16. Q and K tiles are
+// K-major with the 128-byte swizzle (TMA boxes of 64 elements x 128 rows).
+template <int D, bool BF16>
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_smem, uint32_t k_smem) {
+  constexpr uint32_t idesc = mma_idesc_f16(BF16, 128, 128, false, false);
+  const uint64_t a0 = smem_desc_sw128(q_smem, 16, 1024);
+  const uint64_t b0 = smem_desc_sw128(k_smem, 16, 1024);
+#pragma unroll 1
+  for (int kk = 0; kk < D / 16; ++kk) {
+    // 16 elements = 32 bytes along K inside a 128-byte chunk, then the next chunk;
+    // the descriptor address field counts 16-byte units
+    const uint64_t off = static_cast<uint64_t>(((kk >> 2) * Cfg<D>::kChunkBytes + (kk & 3) * 32) >> 4);
+    mma_f16_ss(d_tmem, a0 + off, b0 + off, idesc, kk > 0 ? 1u : 0u);
+  }
+}
+
+// O[tmem] (+)= P[tmem] V over 128 keys: 8 MMAs of 128xDx16. P is packed 16-bit
+// in tensor memory (two keys per column); V is MN-major (d contiguous): 8-key
+// groups 1024 bytes apart, 64-column d chunks one chunk apart.
+template <int D, bool BF16>
+__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_smem,
+                                         bool accumulate) {
+  constexpr uint32_t idesc = mma_idesc_f16(BF16, 128, D, false, true);
+  const uint64_t b0 = smem_desc_sw128(v_smem, Cfg<D>::kChunkBytes, 1024);
+#pragma unroll 1
+  for (int kk = 0; kk < 8; ++kk) {
+    // 16 keys = two 8-row groups = 2048 bytes; P advances 8 packed columns
+    mma_f16_ts(d_tmem, p_tmem + kk * 8, b0 + static_cast<uint64_t>(kk * (2048 >> 4)), idesc,
+               (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+template <int D, bool BF16, bool CAUSAL>
+__device__ __forceinline__ void load_role(const CUtensorMap* tm_q, const CUtensorMap* tm_k,
+                                          const CUtensorMap* tm_v, const FwdParams& p,
+                                          uint32_t sQ, uint32_t sKV, uint32_t bars,
+                                          volatile int* abort_flag) {
+  using C = Cfg<D>;
+  const uint64_t pol_q = l2_policy_evict_first();
+  const uint64_t pol_kv = l2_policy_evict_last();
+  int kv_it = 0, uit = 0;
+  bool aborted = false;
+  for (int u = blockIdx.x; u < p.n_units && !aborted; u += gridDim.x, ++uit) {
+    const Unit x = decode_unit<CAUSAL>(p, u);
+    for (int t = 0; t < 2; ++t) {
+      const uint32_t bq = bars + 8 * (kBarQEmpty + t);
+      if (!mbar_wait(bq, (uit & 1) ^ 1, abort_flag, kFaultLoadQEmpty, p.timeout_ns)) {
+        aborted = true;
+        break;
+      }
+      const uint32_t bf = bars + 8 * (kBarQFull + t);
+      mbar_arrive_expect_tx(bf, C::kTileBytes);
+#pragma unroll
+      for (int c = 0; c < C::kChunks; ++c)
+        tma_load_4d(sQ + t * C::kTileBytes + c * C::kChunkBytes, tm_q, bf, c * 64, x.hq,
+                    x.r0 + t * kTileRows, x.b, pol_q);
+    }
+    for (int j = 0; j < x.n1 && !aborted; ++j) {
+      for (int kv = 0; kv < 2; ++kv) {
+        const int slot = kv_it % C::kStages;
+        const uint32_t be = bars + 8 * (kBarKvEmpty + slot);
+        if (!mbar_wait(be, ((kv_it / C::kStages) & 1) ^ 1, abort_flag, kFaultLoadKvEmpty,
+                       p.timeout_ns)) {
+          aborted = true;
+          break;
+        }
+        const uint32_t bf = bars + 8 * (kBarKvFull + slot);
+        mbar_arrive_expect_tx(bf, C::kTileBytes);
+#pragma unroll
+        for (int c = 0; c < C::kChunks; ++c)
+          tma_load_4d(sKV + slot * C::kTileBytes + c * C::kChunkBytes, kv ? tm_v : tm_k, bf,
+                      c * 64, x.hkv, j * kTileRows, x.b, pol_kv);
+        ++kv_it;
+      }
+    }
+  }
+  if (aborted) {
+    // let the copies already issued land before the CTA exits
+    const int first = kv_it > C::kStages ? kv_it - C::kStages : 0;
+    for (int i = first; i < kv_it; ++i)
+      mbar_drain(bars + 8 * (kBarKvFull + i % C::kStages), (i / C::kStages) & 1);
+    if (uit > 0)
+      for (int t = 0; t < 2; ++t) mbar_drain(bars + 8 * (kBarQFull + t), (uit - 1) & 1);
+  }
+}
+
+template <int D, bool BF16, bool CAUSAL>
+__device__ __forceinline__ void mma_role(const FwdParams& p, uint32_t tmem, uint32_t sQ,
+                                         uint32_t sKV, uint32_t bars, volatile int* abort_flag) {
+  using C = Cfg<D>;
+  auto bar = [&](int i) { return bars + 8 * i; };
+  auto kv_addr = [&](int idx) { return sKV + (idx % C::kStages) * C::kTileBytes; };
+  auto kv_full = [&](int idx) {
+    return mbar_wait(bar(kBarKvFull + idx % C::kStages), (idx / C::kStages) & 1, abort_flag,
+                     kFaultMmaKvFull, p.timeout_ns);
+  };
+  int kv_it = 0, uit = 0;
+  int pcnt[2] = {0, 0};
+  bool ok = true;
+  for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++uit) {
+    const Unit x = decode_unit<CAUSAL>(p, u);
+    ok = mbar_wait(bar(kBarQFull + 0), uit & 1, abort_flag, kFaultMmaQFull, p.timeout_ns) &&
+         mbar_wait(bar(kBarQFull + 1), uit & 1, abort_flag, kFaultMmaQFull, p.timeout_ns) &&
+         kv_full(kv_it);
+    if (!ok) break;
+    tc_fence_after_sync();
+    // S_t(0) = Q_t K_0^T for both tiles
+    issue_qk<D, BF16>(tmem + C::col_s(0), sQ, kv_addr(kv_it));
+    mma_commit(bar(kBarSFull + 0));
+    issue_qk<D, BF16>(tmem + C::col_s(1), sQ + C::kTileBytes, kv_addr(kv_it));
+    mma_commit(bar(kBarSFull + 1));
+    mma_commit(bar(kBarKvEmpty + kv_it % C::kStages));
+    if (x.n0 == 1) mma_commit(bar(kBarQEmpty + 0));
+    if (x.n1 == 1) mma_commit(bar(kBarQEmpty + 1));
+
+    for (int j = 0; j < x.n1 && ok; ++j) {
+      const int vidx = kv_it + 2 * j + 1;  // V_j
+      const int knext = vidx + 1;          // K_{j+1}
+      bool k_ready = false;
+      if (!kv_full(vidx)) { ok = false; break; }
+      tc_fence_after_sync();
+      if (j < x.n0) {
+        if (!mbar_wait(bar(kBarPFull + 0), pcnt[0] & 1, abort_flag, kFaultMmaPFull, p.timeout_ns)) {
+          ok = false;
+          break;
+        }
+        ++pcnt[0];
+        tc_fence_after_sync();
+        issue_pv<D, BF16>(tmem + C::col_o(0), tmem + C::col_s(0), kv_addr(vidx), j > 0);
+        if (j == x.n0 - 1) {
+          mma_commit(bar(kBarOFull + 0));
+        } else {
+          if (!kv_full(knext)) { ok = false; break; }
+          k_ready = true;
+          tc_fence_after_sync();
+          issue_qk<D, BF16>(tmem + C::col_s(0), sQ, kv_addr(knext));
+          mma_commit(bar(kBarSFull + 0));
+          if (j + 1 == x.n0 - 1) mma_commit(bar(kBarQEmpty + 0));
+        }
+      }
+      if (!mbar_wait(bar(kBarPFull + 1), pcnt[1] & 1, abort_flag, kFaultMmaPFull, p.timeout_ns)) {
+        ok = false;
+        break;
+      }
+      ++pcnt[1];
+      tc_fence_after_sync();
+      issue_pv<D, BF16>(tmem + C::col_o(1), tmem + C::col_s(1), kv_addr(vidx), j > 0);
+      mma_commit(bar(kBarKvEmpty + vidx % C::kStages));
+      if (j == x.n1 - 1) {
+        mma_commit(bar(kBarOFull + 1));
+      } else {
+        if (!k_ready) {
+          if (!kv_full(knext)) { ok = false; break; }
+          tc_fence_after_sync();
+        }
+        issue_qk<D, BF16>(tmem + C::col_s(1), sQ + C::kTileBytes, kv_addr(knext));
+        mma_commit(bar(kBarSFull + 1));
+        mma_commit(bar(kBarKvEmpty + knext % C::kStages));
+        if (j + 1 == x.n1 - 1) mma_commit(bar(kBarQEmpty + 1));
+      }
+    }
+    kv_it += 2 * x.n1;
+  }
+  if (!ok) {
+    // every MMA issued so far must finish before tensor memory is freed
+    mma_commit(bar(kBarDrain));
+    mbar_drain(bar(kBarDrain), 0);
+  }
+}
+
+template <int D, bool BF16, bool CAUSAL>
+__device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, uint32_t tmem,
+                                             uint32_t bars, volatile int* abort_flag) {
+  using C = Cfg<D>;
+  const int warp = threadIdx.x / 32;
+  const int r_in = threadIdx.x % kTileRows;                      // row in tile = TMEM lane
+  const uint32_t lane_bits = static_cast<uint32_t>((warp % 4) * 32) << 16;
+  const uint32_t tS = tmem + lane_bits + C::col_s(t);
+  const uint32_t tO = tmem + lane_bits + C::col_o(t);
+  const uint32_t bar_s = bars + 8 * (kBarSFull + t);
+  const uint32_t bar_p = bars + 8 * (kBarPFull + t);
+  const uint32_t bar_o = bars + 8 * (kBarOFull + t);
+  const float sl2 = p.sl2;
+  int scnt = 0, ocnt = 0;
+
+  for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
+    const Unit x = decode_unit<CAUSAL>(p, u);
+    const int n = t ? x.n1 : x.n0;
+    const int row = x.r0 + t * kTileRows + r_in;
+    const int row_lim = CAUSAL ? min(p.Lk, p.kv_offset + row + 1) : p.kv_limit;
+    float ref = -INFINITY;  // scaled (log2) max the exponentials are taken against
+    float l = 0.f;          // running row sum of exp2(s * sl2 - ref)
+
+    for (int j = 0; j < n; ++j) {
+      bool ok = mbar_wait(bar_s, scnt & 1, abort_flag, kFaultSoftmaxSFull, p.timeout_ns);
+      if (!__all_sync(0xffffffffu, ok)) return;
+      ++scnt;
+      tc_fence_after_sync();
+
+      uint32_t r[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(tS + 32 * c, r + 32 * c);
+      tmem_wait_ld_x128(r);
+
+      const int lim = row_lim - j * kTileRows;  // keys c < lim of this tile are visible
+      const bool partial = lim < kTileRows;
+      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      if (partial) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          const float s = c < lim ? __uint_as_float(r[c]) : -INFINITY;
+          mx[c & 3] = fmaxf(mx[c & 3], s);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) mx[c & 3] = fmaxf(mx[c & 3], __uint_as_float(r[c]));
+      }
+      const float m_tile = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+      const float m_scaled = (m_tile == -INFINITY) ? -INFINITY : m_tile * sl2;
+
+      // lazy rescale: move the reference only when the max grew by > tau
+      const bool rescale = m_scaled > ref + kRescaleTau;
+      float alpha = 1.f;
+      if (rescale) {
+        alpha = ex2_approx(ref - m_scaled);
+        ref = m_scaled;
+        l *= alpha;
+      }
+      if (__any_sync(0xffffffffu, rescale && j > 0)) {
+        const float a = (rescale && j > 0) ? alpha : 1.f;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t ov[32];
+          tmem_ld_32x32b_x32(tO + 32 * c, ov);
+          tmem_wait_ld_x32(ov);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * a);
+          tmem_st_32x32b_x32(tO + 32 * c, ov);
+        }
+        tmem_wait_st();
+      }
+
+      // P = exp2(s * sl2 - ref), packed to 16 bits into the first 64 columns of S
+      const float neg_ref = -ref;
+      float sum[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t pk[64];
+#pragma unroll
+      for (int c = 0; c < 128; c += 2) {
+        float p0 = ex2_approx(fmaf(__uint_as_float(r[c]), sl2, neg_ref));
+        float p1 = ex2_approx(fmaf(__uint_as_float(r[c + 1]), sl2, neg_ref));
+        if (partial) {
+          p0 = c < lim ? p0 : 0.f;
+          p1 = c + 1 < lim ? p1 : 0.f;
+        }
+        sum[(c >> 1) & 3] += p0 + p1;
+        pk[c >> 1] = pack2<BF16>(p0, p1);
+      }
+      l += (sum[0] + sum[1]) + (sum[2] + sum[3]);
+      tmem_st_32x32b_x32(tS, pk);
+      tmem_st_32x32b_x32(tS + 32, pk + 32);
+      tmem_wait_st();
+      tc_fence_before_sync();
+      mbar_arrive(bar_p);
+    }
+
+    // epilogue: O / l to 16-bit, 16-byte stores; LSE
+    bool ok = mbar_wait(bar_o, ocnt & 1, abort_flag, kFaultSoftmaxOFull, p.timeout_ns);
+    if (!__all_sync(0xffffffffu, ok)) return;
+    ++ocnt;
+    tc_fence_after_sync();
+    const float inv_l = 1.f / l;
+    const bool in_range = row < p.Lq;
+    uint16_t* orow = static_cast<uint16_t*>(p.o) +
+                     ((static_cast<size_t>(x.b) * p.Lq + row) * p.Hq + x.hq) * D;
+#pragma unroll 1
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t ov[32];
+      tmem_ld_32x32b_x32(tO + 32 * c, ov);
+      tmem_wait_ld_x32(ov);
+      uint32_t pk[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e)
+        pk[e] = pack2<BF16>(__uint_as_float(ov[2 * e]) * inv_l, __uint_as_float(ov[2 * e + 1]) * inv_l);
+      if (in_range) {
+        uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+      }
+    }
+    if (p.lse != nullptr && in_range)
+      p.lse[(static_cast<size_t>(x.b) * p.Hq + x.hq) * p.Lq + row] = (ref + log2f(l)) * kLn2;
+  }
+}
+
+template <int D, bool BF16, bool CAUSAL>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
+                          const __grid_constant__ CUtensorMap tm_k,
+                          const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  using C = Cfg<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t sQ = sbase + C::kOffQ;
+  const uint32_t sKV = sbase + C::kOffKV;
+  const uint32_t bars = sbase + C::kOffBar;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffBar + 256);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffBar + 260);
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+
+  if (threadIdx.x == 0) {
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bars + 8 * (kBarQFull + t), 1);
+      mbar_init(bars + 8 * (kBarQEmpty + t), 1);
+      mbar_init(bars + 8 * (kBarSFull + t), 1);
+      mbar_init(bars + 8 * (kBarPFull + t), kTileRows);
+      mbar_init(bars + 8 * (kBarOFull + t), 1);
+    }
+    mbar_init(bars + 8 * kBarDrain, 1);
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(bars + 8 * (kBarKvFull + s), 1);
+      mbar_init(bars + 8 * (kBarKvEmpty + s), 1);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 8 && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp < 8) {
+    regs_increase<kRegsSoftmax>();
+    softmax_role<D, BF16, CAUSAL>(warp / 4, p, tmem, bars, abort_flag);
+  } else {
+    regs_decrease<kRegsProducer>();
+    if (warp == 8) {
+      if (lane == 0) load_role<D, BF16, CAUSAL>(&tm_q, &tm_k, &tm_v, p, sQ, sKV, bars, abort_flag);
+    } else if (warp == 9) {
+      if (lane == 0) mma_role<D, BF16, CAUSAL>(p, tmem, sQ, sKV, bars, abort_flag);
+    }
+  }
+  __syncwarp();
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------- diagnostics
+
+// One 128x128 tile: S = Q K^T, then O = round16(S/16) V, through the same
+// descriptors and MMA issue code as the forward kernel. 128 threads.
+template <bool BF16>
+__global__ void __launch_bounds__(128, 1)
+    selftest_mma_kernel(const __grid_constant__ CUtensorMap tm_q,
+                        const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, float* s_out, float* o_out,
+                        unsigned long long timeout_ns) {
+  constexpr int D = 128;
+  using C = Cfg<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sQ = smem_u32(smem);
+  const uint32_t sK = sQ + C::kTileBytes;
+  const uint32_t sV = sK + C::kTileBytes;
+  const uint32_t bars = sV + C::kTileBytes;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + 3 * C::kTileBytes + 64);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + 3 * C::kTileBytes + 68);
+  const int warp = threadIdx.x / 32;
+  if (threadIdx.x == 0) {
+    mbar_init(bars, 1);      // TMA
+    mbar_init(bars + 8, 1);  // MMA
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t lane_bits = static_cast<uint32_t>(warp * 32) << 16;
+  bool ok = true;
+
+  if (threadIdx.x == 0) {
+    const uint64_t pol = l2_policy_evict_first();
+    mbar_arrive_expect_tx(bars, 3 * C::kTileBytes);
+    for (int c = 0; c < 2; ++c) {
+      tma_load_4d(sQ + c * C::kChunkBytes, &tm_q, bars, c * 64, 0, 0, 0, pol);
+      tma_load_4d(sK + c * C::kChunkBytes, &tm_k, bars, c * 64, 0, 0, 0, pol);
+      tma_load_4d(sV + c * C::kChunkBytes, &tm_v, bars, c * 64, 0, 0, 0, pol);
+    }
+    ok = mbar_wait(bars, 0, abort_flag, kFaultSelftest, timeout_ns);
+    if (ok) {
+      tc_fence_after_sync();
+      issue_qk<D, BF16>(tmem + 0, sQ, sK);
+    }
+    mma_commit(bars + 8);
+  }
+  ok = mbar_wait(bars + 8, 0, abort_flag, kFaultSelftest, timeout_ns);
+  ok = __all_sync(0xffffffffu, ok);
+  tc_fence_after_sync();
+  const int row = threadIdx.x;
+  if (ok) {
+    uint32_t r[128];
+    for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(tmem + lane_bits + 32 * c, r + 32 * c);
+    tmem_wait_ld_x128(r);
+    uint32_t pk[64];
+    for (int c = 0; c < 128; ++c) s_out[row * 128 + c] = __uint_as_float(r[c]);
+    for (int c = 0; c < 64; ++c)
+      pk[c] = pack2<BF16>(__uint_as_float(r[2 * c]) * 0.0625f, __uint_as_float(r[2 * c + 1]) * 0.0625f);
+    tmem_st_32x32b_x32(tmem + lane_bits, pk);
+    tmem_st_32x32b_x32(tmem + lane_bits + 32, pk + 32);
+    tmem_wait_st();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    tc_fence_after_sync();
+    if (!*abort_flag) issue_pv<D, BF16>(tmem + 256, tmem + 0, sV, false);
+    mma_commit(bars + 8);
+  }
+  ok = !*abort_flag && mbar_wait(bars + 8, 1, abort_flag, kFaultSelftest, timeout_ns);
+  ok = __all_sync(0xffffffffu, ok);
+  tc_fence_after_sync();
+  if (ok) {
+    for (int c = 0; c < 4; ++c) {
+      uint32_t ov[32];
+      tmem_ld_32x32b_x32(tmem + lane_bits + 256 + 32 * c, ov);
+      tmem_wait_ld_x32(ov);
+      for (int e = 0; e < 32; ++e) o_out[row * 128 + 32 * c + e] = __uint_as_float(ov[e]);
+    }
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// One thread waits on a barrier nothing completes; the bounded wait must give up.
+__global__ void selftest_timeout_kernel(unsigned long long timeout_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(smem_u32(&bar), 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    (void)mbar_wait(smem_u32(&bar), 0, &abort_flag, kFaultSelftest, timeout_ns);
+  }
+}
+
+// ------------------------------------------------------------------- host
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+std::atomic<unsigned long long> g_timeout_ns{4000000000ull};
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<EncodeTiledFn>(f);
+  }();
+  return fn;
+}
+
+struct DeviceInfo {
+  bool ok = false;
+  bool sm100 = false;
+  int num_sms = 0;
+};
+
+constexpr int kMaxDevices = 64;
+
+DeviceInfo device_info(int dev) {
+  static DeviceInfo infos[kMaxDevices];
+  static std::once_flag flags[kMaxDevices];
+  if (dev < 0 || dev >= kMaxDevices) return DeviceInfo{};
+  std::call_once(flags[dev], [dev]() {
+    DeviceInfo di;
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess) {
+      di.ok = true;
+      di.sm100 = (major == 10 && minor == 0);
+      di.num_sms = sms;
+    }
+    infos[dev] = di;
+  });
+  return infos[dev];
+}
+
+// [B, L, H, d] 16-bit tensor as a 4-D TMA map (innermost first: d, H, L, B);
+// box = 64 elements of d x 1 head x 128 rows x 1 batch, 128-byte swizzle.
+bool encode_bl_hd(CUtensorMap* map, const void* ptr, int B, int L, int H, int d, bool bf16) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)L, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2, (cuuint64_t)L * H * d * 2};
+  const cuuint32_t box[4] = {64, 1, (cuuint32_t)kTileRows, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
+                  const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int D, bool BF16, bool CAUSAL>
+int launch_fwd(const FwdParams& p, const void* q, const void* k, const void* v, int grid,
+               cudaStream_t stream) {
+  using C = Cfg<D>;
+  CUtensorMap tq, tk, tv;
+  if (!encode_bl_hd(&tq, q, p.B, p.Lq, p.Hq, D, BF16) ||
+      !encode_bl_hd(&tk, k, p.B, p.Lk, p.Hkv, D, BF16) ||
+      !encode_bl_hd(&tv, v, p.B, p.Lk, p.Hkv, D, BF16))
+    return ATTN_ERR_CUDA;
+  auto kern = attn_fwd_sm100_kernel<D, BF16, CAUSAL>;
+  static std::once_flag attr_flags[kMaxDevices];
+  static int attr_status[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
+  std::call_once(attr_flags[dev], [&]() {
+    attr_status[dev] = ATTN_OK;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
+        cudaSuccess) {
+      attr_status[dev] = ATTN_ERR_CUDA;
+      return;
+    }
+    // The warpgroup register split must fit the block's launch budget, or the
+    // softmax warpgroups' setmaxnreg.inc would wait for registers forever.
+    cudaFuncAttributes fa{};
+    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess ||
+        fa.numRegs * kThreads < 128 * kRegsProducer + 256 * kRegsSoftmax)
+      attr_status[dev] = ATTN_ERR_CUDA;
+  });
+  if (attr_status[dev] != ATTN_OK) return attr_status[dev];
+  (void)cudaGetLastError();  // launch errors below are this launch's own
+  kern<<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+bool ranges_overlap(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+}  // namespace hasb
+
+using namespace hasb;
+
+extern "C" {
+
+const char* attn_status_string(int status) {
+  switch (status) {
+    case ATTN_OK: return "ok";
+    case ATTN_ERR_INVALID_ARG: return "invalid argument";
+    case ATTN_ERR_UNSUPPORTED: return "unsupported configuration (head_dim or device)";
+    case ATTN_ERR_CUDA: return "CUDA error";
+    case ATTN_ERR_TIMEOUT: return "device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int attn_set_wait_timeout_ns(unsigned long long ns) {
+  g_timeout_ns.store(ns < 1000000ull ? 1000000ull : ns);
+  return ATTN_OK;
+}
+
+}  // extern "C"
+
+namespace hasb {
+
+// The argument contract of attn_fwd; makes no CUDA call.
+int attn_fwd_validate(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                      int B, int Lq, int Lk, int Hq, int Hkv, int d, float scale, int causal,
+                      int kv_offset, int dtype) {
+  // ---- argument contract (no CUDA call before this block is passed)
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return ATTN_ERR_INVALID_ARG;
+  if (B < 1 || Lq < 1 || Lk < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (d < 16 || d > 256 || (d & (d - 1)) != 0) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || scale < 0.f) return ATTN_ERR_INVALID_ARG;
+  if (dtype != ATTN_DTYPE_BF16 && dtype != ATTN_DTYPE_FP16) return ATTN_ERR_INVALID_ARG;
+  if (causal != ATTN_MASK_NONE && causal != ATTN_MASK_CAUSAL && causal != ATTN_MASK_CHUNK)
+    return ATTN_ERR_INVALID_ARG;
+  if (causal == ATTN_MASK_NONE) {
+    if (kv_offset != 0) return ATTN_ERR_INVALID_ARG;
+  } else if (kv_offset < 0 || static_cast<long long>(kv_offset) + Lq > Lk) {
+    return ATTN_ERR_INVALID_ARG;
+  }
+  const auto aligned16 = [](const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; };
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ATTN_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return ATTN_ERR_INVALID_ARG;
+  const unsigned long long q_elems = 1ull * B * Lq * Hq * d;
+  const unsigned long long kv_elems = 1ull * B * Lk * Hkv * d;
+  if (q_elems * 2 >= (1ull << 40) || kv_elems * 2 >= (1ull << 40)) return ATTN_ERR_INVALID_ARG;
+  const long long n_pairs = (Lq + 2LL * kTileRows - 1) / (2LL * kTileRows);
+  const long long n_units = n_pairs * B * Hq;
+  if (n_units > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+  if (ranges_overlap(o, q_elems * 2, q, q_elems * 2) || ranges_overlap(o, q_elems * 2, k, kv_elems * 2) ||
+      ranges_overlap(o, q_elems * 2, v, kv_elems * 2))
+    return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  return ATTN_OK;
+}
+
+}  // namespace hasb
+
+extern "C" {
+
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Lq,
+             int Lk, int Hq, int Hkv, int d, float scale, int causal, int kv_offset, int dtype,
+             void* stream) {
+  // ---- argument contract (no CUDA call before it passes)
+  const int valid = attn_fwd_validate(q, k, v, o, lse, B, Lq, Lk, Hq, Hkv, d, scale, causal,
+                                      kv_offset, dtype);
+  if (valid != ATTN_OK) return valid;
+  const long long n_pairs = (Lq + 2LL * kTileRows - 1) / (2LL * kTileRows);
+  const long long n_units = n_pairs * B * Hq;
+
+  // ---- device
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+  const DeviceInfo di = device_info(dev);
+  if (!di.ok) return ATTN_ERR_CUDA;
+  if (!di.sm100) return ATTN_ERR_UNSUPPORTED;
+
+  FwdParams p;
+  p.o = o;
+  p.lse = lse;
+  p.B = B; p.Lq = Lq; p.Lk = Lk; p.Hq = Hq; p.Hkv = Hkv; p.group = Hq / Hkv;
+  p.kv_offset = kv_offset;
+  p.kv_limit = (causal == ATTN_MASK_CHUNK) ? kv_offset + Lq : Lk;
+  p.n_pairs = static_cast<int>(n_pairs);
+  p.n_units = static_cast<int>(n_units);
+  p.sl2 = scale * kLog2e;
+  p.timeout_ns = g_timeout_ns.load();
+  const int grid = static_cast<int>(n_units < di.num_sms ? n_units : di.num_sms);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool bf16 = dtype == ATTN_DTYPE_BF16;
+  const bool cz = causal == ATTN_MASK_CAUSAL;
+  if (d == 128) {
+    if (bf16) return cz ? launch_fwd<128, true, true>(p, q, k, v, grid, s) : launch_fwd<128, true, false>(p, q, k, v, grid, s);
+    return cz ? launch_fwd<128, false, true>(p, q, k, v, grid, s) : launch_fwd<128, false, false>(p, q, k, v, grid, s);
+  }
+  if (bf16) return cz ? launch_fwd<64, true, true>(p, q, k, v, grid, s) : launch_fwd<64, true, false>(p, q, k, v, grid, s);
+  return cz ? launch_fwd<64, false, true>(p, q, k, v, grid, s) : launch_fwd<64, false, false>(p, q, k, v, grid, s);
+}
+
+int attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, void* o_host,
+                  float* lse_host, void* q_dev, void* k_dev, void* v_dev, void* o_dev,
+                  float* lse_dev, int B, int Lq, int Lk, int Hq, int Hkv, int d, float scale,
+                  int causal, int kv_offset, int dtype, void* stream) {
+  if (!q_host || !k_host || !v_host || !o_host) return ATTN_ERR_INVALID_ARG;
+  if ((lse_host == nullptr) != (lse_dev == nullptr)) return ATTN_ERR_INVALID_ARG;
+  if (B < 1 || Lq < 1 || Lk < 1 || Hq < 1 || Hkv < 1 || d < 1) return ATTN_ERR_INVALID_ARG;
+  const size_t q_bytes = 2ull * B * Lq * Hq * d;
+  const size_t kv_bytes = 2ull * B * Lk * Hkv * d;
+  const size_t lse_bytes = 4ull * B * Hq * Lq;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // attn_fwd checks the device side; run its validation first by a dry call
+  // ordering: copies only once the arguments are known to be valid
+  const int pre = attn_fwd_validate(q_dev, k_dev, v_dev, o_dev, lse_dev, B, Lq, Lk, Hq, Hkv, d, scale,
+                                    causal, kv_offset, dtype);
+  if (pre != ATTN_OK) return pre;
+  if (cudaMemcpyAsync(q_dev, q_host, q_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(k_dev, k_host, kv_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(v_dev, v_host, kv_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  const int st = attn_fwd(q_dev, k_dev, v_dev, o_dev, lse_dev, B, Lq, Lk, Hq, Hkv, d, scale, causal,
+                          kv_offset, dtype, stream);
+  if (st != ATTN_OK) return st;
+  if (cudaMemcpyAsync(o_host, o_dev, q_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  if (lse_host != nullptr &&
+      cudaMemcpyAsync(lse_host, lse_dev, lse_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  return ATTN_OK;
+}
+
+int attn_device_fault(unsigned int* bits, int clear) {
+  if (bits == nullptr) return ATTN_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return ATTN_ERR_CUDA;
+  unsigned int b = 0;
+  if (cudaMemcpyFromSymbol(&b, g_fault_bits, sizeof(b)) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (clear) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(g_fault_bits, &zero, sizeof(zero)) != cudaSuccess) return ATTN_ERR_CUDA;
+  }
+  *bits = b;
+  return b ? ATTN_ERR_TIMEOUT : ATTN_OK;
+}
+
+int attn_selftest_mma(const void* q, const void* k, const void* v, float* s_out, float* o_out,
+                      int dtype, void* stream) {
+  if (!q || !k || !v || !s_out || !o_out) return ATTN_ERR_INVALID_ARG;
+  if (dtype != ATTN_DTYPE_BF16 && dtype != ATTN_DTYPE_FP16) return ATTN_ERR_INVALID_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+  const DeviceInfo di = device_info(dev);
+  if (!di.ok) return ATTN_ERR_CUDA;
+  if (!di.sm100) return ATTN_ERR_UNSUPPORTED;
+  const bool bf16 = dtype == ATTN_DTYPE_BF16;
+  CUtensorMap tq, tk, tv;
+  if (!encode_bl_hd(&tq, q, 1, 128, 1, 128, bf16) || !encode_bl_hd(&tk, k, 1, 128, 1, 128, bf16) ||
+      !encode_bl_hd(&tv, v, 1, 128, 1, 128, bf16))
+    return ATTN_ERR_CUDA;
+  const int smem = 3 * Cfg<128>::kTileBytes + 128 + 1024;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  auto kern = bf16 ? selftest_mma_kernel<true> : selftest_mma_kernel<false>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  kern<<<1, 128, smem, s>>>(tq, tk, tv, s_out, o_out, g_timeout_ns.load());
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return ATTN_ERR_CUDA;
+  unsigned int bits = 0;
+  return attn_device_fault(&bits, 1);
+}
+
+int attn_selftest_wait_timeout(unsigned long long timeout_ns, void* stream) {
+  if (timeout_ns < 1000000ull || timeout_ns > 10000000000ull) return ATTN_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned int bits = 0;
+  int st = attn_device_fault(&bits, 1);  // start from a clear word
+  if (st == ATTN_ERR_CUDA) return st;
+  selftest_timeout_kernel<<<1, 32, 0, s>>>(timeout_ns);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return ATTN_ERR_CUDA;
+  return attn_device_fault(&bits, 1);
+}
+
+}  // extern "C"

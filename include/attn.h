@@ -1,0 +1,143 @@
+/*
+ * head_attention_streaming_b200 — C ABI of the fused attention forward for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The library computes, per batch b, query head hq and query row i,
+ *
+ *     O[b,i,hq,:] = sum_j softmax_j( scale * Q[b,i,hq,:] . K[b,j,hkv,:] ) V[b,j,hkv,:]
+ *
+ * over the keys j visible to row i. This is the per-head scaled dot-product
+ * attention of the flashdreams.accelerated developer guide ("Optimized Multi
+ * Head Attention" -> "Multi Head Attention Definition", the equation for A_h),
+ * with the scale given explicitly (1/sqrt(d) there), for the token-major
+ * [batch, seq, heads, head_dim] layout that page and the FlashAttention-4
+ * runtime page ("FLASH4.md", H3 call layout) use.
+ *
+ * All functions are plain C. Pointers named "device" must point to CUDA device
+ * memory of the current device; the library allocates no device memory and
+ * owns no buffer. Every function returns an attn_status_t value (as int).
+ */
+#ifndef HEAD_ATTENTION_STREAMING_B200_ATTN_H_
+#define HEAD_ATTENTION_STREAMING_B200_ATTN_H_
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = 1,   /* an argument breaks the contract below; nothing was launched */
+  ATTN_ERR_UNSUPPORTED = 2,   /* valid by the pages' contract but not built (head_dim, device) */
+  ATTN_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed (launch, descriptor encode) */
+  ATTN_ERR_TIMEOUT = 4        /* a device-side wait ran past its limit (see attn_device_fault) */
+} attn_status_t;
+
+typedef enum { ATTN_DTYPE_BF16 = 0, ATTN_DTYPE_FP16 = 1 } attn_dtype_t;
+
+typedef enum {
+  ATTN_MASK_NONE = 0,    /* every key visible (cross-attention, full self-attention) */
+  ATTN_MASK_CAUSAL = 1,  /* key j visible to row i iff j <= kv_offset + i */
+  ATTN_MASK_CHUNK = 2    /* streaming chunk: key j visible iff j < kv_offset + Lq */
+} attn_mask_t;
+
+/*
+ * attn_fwd — fused attention forward, asynchronous on `stream`.
+ *
+ * Operation: scaled dot-product attention (developer guide, "Multi Head
+ * Attention Definition"); grouped K/V heads as in the skill page
+ * "optimizing-attention-flash", "Workflow 2" Step 3 (multi-query attention),
+ * with query head hq reading K/V head hq / (Hq / Hkv); the causal flag of the
+ * same page's flash-attn call; and the streaming self-attention step of the
+ * developer guide's "Generic Multi Head Attention Interface" and the user
+ * guide's "Cache lifecycle", where the current chunk's K/V are already in the
+ * rolling cache when the chunk is queried and the chunk attends to the whole
+ * visible cache.
+ *
+ * Arguments (all tensors contiguous, row-major, 16-byte aligned base):
+ *   q    device, [B, Lq, Hq, d]  of dtype            (read)
+ *   k    device, [B, Lk, Hkv, d] of dtype            (read)
+ *   v    device, [B, Lk, Hkv, d] of dtype            (read)
+ *   o    device, [B, Lq, Hq, d]  of dtype            (written; must not overlap q, k, v)
+ *   lse  device, [B, Hq, Lq] float32, natural log of sum_j exp(scale * s_ij)
+ *        over visible keys; may be NULL (then not written)
+ *   B, Lq, Lk, Hq, Hkv  >= 1, Hq % Hkv == 0
+ *   d    head_dim; the pages allow powers of two 16..256; this build runs 64 and 128
+ *   scale  finite, >= 0 (1/sqrt(d) in the pages)
+ *   causal attn_mask_t: 0 none, 1 causal, 2 streaming chunk
+ *   kv_offset  cache position of query row 0: 0 for mask 0; for masks 1 and 2,
+ *        0 <= kv_offset and kv_offset + Lq <= Lk (a causal call with
+ *        kv_offset = Lk - Lq aligns the diagonal bottom-right)
+ *   dtype  attn_dtype_t, the element type of q, k, v and o
+ *   stream cudaStream_t (NULL = legacy default stream)
+ *
+ * Errors: every argument is checked before any CUDA call; a violation returns
+ * ATTN_ERR_INVALID_ARG (or ATTN_ERR_UNSUPPORTED for a head_dim or device this
+ * build does not run) and launches nothing. There is no fallback to another
+ * kernel or to the CPU. A failed launch returns ATTN_ERR_CUDA. The call does
+ * not synchronize; a device-side timeout is reported by attn_device_fault.
+ */
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+             int B, int Lq, int Lk, int Hq, int Hkv, int d, float scale,
+             int causal, int kv_offset, int dtype, void* stream);
+
+/*
+ * attn_fwd_host — the same forward for operands in host memory: copies q, k, v
+ * from host to the caller's device buffers, runs attn_fwd, and copies o (and
+ * lse when both lse pointers are given) back to host memory, all queued on
+ * `stream` in that order (cudaMemcpyAsync; use pinned host memory for
+ * asynchronous copies). The call returns once the work is queued; synchronize
+ * `stream` before reading o_host. Shapes, dtype, mask and errors as attn_fwd;
+ * additionally every host pointer but lse_host must be non-NULL, and lse_host
+ * and lse_dev must be both NULL or both non-NULL. Device buffers are owned by
+ * the caller and sized as attn_fwd's q, k, v, o, lse.
+ */
+int attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, void* o_host,
+                  float* lse_host, void* q_dev, void* k_dev, void* v_dev, void* o_dev,
+                  float* lse_dev, int B, int Lq, int Lk, int Hq, int Hkv, int d, float scale,
+                  int causal, int kv_offset, int dtype, void* stream);
+
+/* Short English text of a status code (static storage). */
+const char* attn_status_string(int status);
+
+/*
+ * attn_device_fault — synchronizes the current device, then returns in *bits
+ * the device fault word that kernels of this library set when a bounded wait
+ * on a shared-memory barrier ran out (0: none). Each bit names the wait that
+ * gave up. With clear != 0 the word is reset to 0. Returns ATTN_ERR_TIMEOUT
+ * when *bits != 0, else ATTN_OK (or ATTN_ERR_CUDA).
+ */
+int attn_device_fault(unsigned int* bits, int clear);
+
+/*
+ * attn_set_wait_timeout_ns — limit, in nanoseconds, of every device-side
+ * barrier wait in kernels launched after this call (default 4e9). A wait that
+ * runs out sets its bit in the fault word, stops its CTA's pipeline, waits
+ * briefly for its own copies and MMAs in flight, frees its tensor memory and
+ * exits. Values below 1e6 are raised to 1e6.
+ */
+int attn_set_wait_timeout_ns(unsigned long long ns);
+
+/*
+ * Diagnostics, used by the tests to check the building blocks of attn_fwd on
+ * the device. Neither is needed to compute attention.
+ *
+ * attn_selftest_mma — one 128x128 tile through the same tensor-core path as
+ * attn_fwd: TMA loads of q, k, v ([128, 128] row-major, dtype), S = q k^T
+ * accumulated in tensor memory and copied to s_out ([128,128] float32), then
+ * P = round_dtype(S / 16) written back to tensor memory and O = P v copied to
+ * o_out ([128,128] float32). Synchronous.
+ *
+ * attn_selftest_wait_timeout — launches one CTA that waits on a barrier
+ * nothing completes, with the given limit in nanoseconds (1e6..1e10); returns
+ * ATTN_ERR_TIMEOUT when the wait gave up as designed (and clears the fault
+ * word), ATTN_OK if it did not. Synchronous.
+ */
+int attn_selftest_mma(const void* q, const void* k, const void* v, float* s_out, float* o_out,
+                      int dtype, void* stream);
+int attn_selftest_wait_timeout(unsigned long long timeout_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HEAD_ATTENTION_STREAMING_B200_ATTN_H_ */

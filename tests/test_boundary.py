@@ -1,0 +1,108 @@
+"""C-ABI boundary checks that need no GPU.
+
+The library must load on a machine without a device, export every function
+include/attn.h declares, and reject every invalid argument with the right
+status before making any CUDA call (so these calls are safe anywhere: nothing
+is launched). The pages' strict-backend convention (FlashAttention-4 runtime
+page, "FLASH4.md": a violated contract raises an error instead of changing
+kernels) is what the status codes implement.
+"""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import head_attention_streaming_b200 as hasb
+from head_attention_streaming_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "attn.h")
+
+A = 0x10000  # 16-byte aligned fake addresses: never dereferenced (calls fail validation first)
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:int|const char\*)\s+(attn_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_entry_points():
+    names = _declared_functions()
+    assert "attn_fwd" in names and "attn_status_string" in names
+    assert len(names) >= 6
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    L = hasb.lib()
+    for name in _declared_functions():
+        assert hasattr(L, name), name
+    assert set(_declared_functions()) == set(binding._SIGNATURES)
+
+
+def test_status_strings():
+    for st in range(5):
+        assert hasb.status_string(st) != "unknown status"
+    assert hasb.status_string(99) == "unknown status"
+
+
+def _call(**kw):
+    args = dict(q=A, k=A + 0x100000, v=A + 0x200000, o=A + 0x300000, lse=None, B=1, Lq=4, Lk=4,
+                Hq=2, Hkv=1, d=128, scale=0.125, causal=0, kv_offset=0, dtype=0)
+    args.update(kw)
+    L = hasb.lib()
+    return L.attn_fwd(args["q"], args["k"], args["v"], args["o"], args["lse"], args["B"], args["Lq"],
+                      args["Lk"], args["Hq"], args["Hkv"], args["d"], args["scale"], args["causal"],
+                      args["kv_offset"], args["dtype"], None)
+
+
+INVALID = [
+    dict(q=None), dict(k=None), dict(v=None), dict(o=None),
+    dict(B=0), dict(Lq=0), dict(Lk=0), dict(Hq=0), dict(Hkv=0), dict(Hq=3, Hkv=2),
+    dict(d=0), dict(d=96), dict(d=8), dict(d=512),
+    dict(scale=float("nan")), dict(scale=float("inf")), dict(scale=-0.5),
+    dict(dtype=2), dict(dtype=-1), dict(causal=3), dict(causal=-1),
+    dict(kv_offset=1),                              # mask none takes no offset
+    dict(causal=1, kv_offset=-1), dict(causal=1, Lq=4, Lk=4, kv_offset=1),
+    dict(causal=2, Lq=3, Lk=10, kv_offset=8),       # chunk end past the cache
+    dict(q=A + 8), dict(k=A + 0x100000 + 4), dict(o=A + 0x300000 + 2),
+    dict(lse=A + 0x400000 + 2),
+    dict(o=A),                                      # output overlaps q
+    dict(o=A + 0x100000 + 64),                      # output overlaps k
+    dict(B=1 << 16, Lq=1 << 16, Hq=1 << 10, Hkv=1 << 10),   # size overflow
+]
+
+
+@pytest.mark.parametrize("kw", INVALID, ids=[str(k) for k in INVALID])
+def test_invalid_arguments_are_rejected_before_any_launch(kw):
+    assert _call(**kw) == hasb.ATTN_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("d", [16, 32, 256])
+def test_head_dims_allowed_by_the_pages_but_not_built_are_unsupported(d):
+    assert _call(d=d) == hasb.ATTN_ERR_UNSUPPORTED
+
+
+def test_python_binding_rejects_cpu_tensors():
+    import torch
+    q = torch.zeros(1, 4, 2, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        hasb.attn_fwd(q, q, q)
+
+
+def test_device_fault_null_pointer():
+    assert hasb.lib().attn_device_fault(None, 0) == hasb.ATTN_ERR_INVALID_ARG
+
+
+def test_selftest_timeout_rejects_out_of_range_limits():
+    assert hasb.lib().attn_selftest_wait_timeout(10, None) == hasb.ATTN_ERR_INVALID_ARG
+    assert hasb.lib().attn_selftest_wait_timeout(10**11, None) == hasb.ATTN_ERR_INVALID_ARG
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(binding, "_LIB", None)
+    monkeypatch.setattr(binding, "_SO_PATH", str(tmp_path / "absent.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        binding.lib()
