@@ -56,6 +56,9 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="video_20480x56x128")
+    ap.add_argument("--shape", default=None,
+                    help="B,Lq,Lk,Hq,Hkv,d override of the workload's shape (profiling "
+                         "captures of a smaller case of the same kernel)")
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -197,12 +200,24 @@ def workload_config(w, n_gpus):
             "parallelism": f"replicas x{n_gpus}" if n_gpus > 1 else "single GPU"}
 
 
+def select_workload(args):
+    import dataclasses
+
+    from head_attention_streaming_b200 import inputs
+    w = inputs.WORKLOADS[args.workload]
+    if args.shape:
+        B, Lq, Lk, Hq, Hkv, d = (int(x) for x in args.shape.split(","))
+        w = dataclasses.replace(w, name=f"{w.name}@{B}x{Lq}x{Lk}x{Hq}x{Hkv}x{d}", B=B, Lq=Lq,
+                                Lk=Lk, Hq=Hq, Hkv=Hkv, d=d, scale=1.0 / math.sqrt(d))
+    return w
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
     from head_attention_streaming_b200 import inputs
-    w = inputs.WORKLOADS[args.workload]
+    w = select_workload(args)
     q, k, v = inputs.workload_inputs(w)
     per_step = max(0.05, min(1.0, 120.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
@@ -251,7 +266,7 @@ def main():
         if world > 1:
             dist.barrier()
 
-    w = inputs.WORKLOADS[args.workload]
+    w = select_workload(args)
     q_cpu, k_cpu, v_cpu = inputs.make_qkv(w.B, w.Lq, w.Lk, w.Hq, w.Hkv, w.d, w.torch_dtype,
                                           seed=w.seed + 7919 * rank, qk_rmsnorm=w.qk_rmsnorm)
     q, k, v = q_cpu.cuda(), k_cpu.cuda(), v_cpu.cuda()

@@ -51,10 +51,10 @@ enum FaultBit : unsigned int {
 
 constexpr int kThreads = 384;
 // Register split: 384 threads x 168 launch registers = 64512. The producer
-// warpgroup (warps 8-11) drops to 56, the two softmax warpgroups rise to 224:
-// 128 x 56 + 256 x 224 = 64512.
-constexpr int kRegsProducer = 56;
-constexpr int kRegsSoftmax = 224;
+// warpgroup (warps 8-11) drops to 88, the two softmax warpgroups rise to 208:
+// 128 x 88 + 256 x 208 = 64512.
+constexpr int kRegsProducer = 88;
+constexpr int kRegsSoftmax = 208;
 constexpr int kTileRows = 128;         // query rows per softmax tile = keys per KV tile
 constexpr float kRescaleTau = 8.0f;    // lazy rescale threshold, log2 units (P <= 256)
 constexpr float kLn2 = 0.69314718055994531f;
@@ -162,36 +162,33 @@ __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
   }
 }
 
-// S[tmem] = Q K^T over head_dim D: D/16 MMAs of 128x128x16. Q and K tiles are
-// K-major with the 128-byte swizzle (TMA boxes of 64 elements x 128 rows).
+// S[tmem] = Q K^T over head_dim D: D/16 MMAs of 128x128x16, fully unrolled (a
+// single thread issues every MMA; a rolled loop leaves the tensor core idle).
+// Q and K tiles are K-major with the 128-byte swizzle (TMA boxes of 64 elements
+// x 128 rows): 16 elements = 32 bytes along K inside a chunk, then the next
+// chunk. Descriptor address fields count 16-byte units.
 template <int D, bool BF16>
-__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_smem, uint32_t k_smem) {
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_lo, uint32_t k_lo) {
   constexpr uint32_t idesc = mma_idesc_f16(BF16, 128, 128, false, false);
-  const uint64_t a0 = smem_desc_sw128(q_smem, 16, 1024);
-  const uint64_t b0 = smem_desc_sw128(k_smem, 16, 1024);
-#pragma unroll 1
-  for (int kk = 0; kk < D / 16; ++kk) {
-    // 16 elements = 32 bytes along K inside a 128-byte chunk, then the next chunk;
-    // the descriptor address field counts 16-byte units
-    const uint64_t off = static_cast<uint64_t>(((kk >> 2) * Cfg<D>::kChunkBytes + (kk & 3) * 32) >> 4);
-    mma_f16_ss(d_tmem, a0 + off, b0 + off, idesc, kk > 0 ? 1u : 0u);
+  mma_f16_ss_lo<false>(d_tmem, q_lo, k_lo, idesc);
+#pragma unroll
+  for (int kk = 1; kk < D / 16; ++kk) {
+    const uint32_t off = static_cast<uint32_t>(((kk >> 2) * Cfg<D>::kChunkBytes + (kk & 3) * 32) >> 4);
+    mma_f16_ss_lo<true>(d_tmem, q_lo + off, k_lo + off, idesc);
   }
 }
 
 // O[tmem] (+)= P[tmem] V over 128 keys: 8 MMAs of 128xDx16. P is packed 16-bit
 // in tensor memory (two keys per column); V is MN-major (d contiguous): 8-key
-// groups 1024 bytes apart, 64-column d chunks one chunk apart.
+// groups 1024 bytes apart (SBO), 64-column d chunks one chunk apart (LBO), so
+// 16 keys advance the start address by 2048 bytes.
 template <int D, bool BF16>
-__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_smem,
-                                         bool accumulate) {
+__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_lo,
+                                         uint32_t accumulate) {
   constexpr uint32_t idesc = mma_idesc_f16(BF16, 128, D, false, true);
-  const uint64_t b0 = smem_desc_sw128(v_smem, Cfg<D>::kChunkBytes, 1024);
-#pragma unroll 1
-  for (int kk = 0; kk < 8; ++kk) {
-    // 16 keys = two 8-row groups = 2048 bytes; P advances 8 packed columns
-    mma_f16_ts(d_tmem, p_tmem + kk * 8, b0 + static_cast<uint64_t>(kk * (2048 >> 4)), idesc,
-               (accumulate || kk > 0) ? 1u : 0u);
-  }
+  mma_f16_ts_lo_flag(d_tmem, p_tmem, v_lo, idesc, accumulate);
+#pragma unroll
+  for (int kk = 1; kk < 8; ++kk) mma_f16_ts_lo<true>(d_tmem, p_tmem + kk * 8, v_lo + kk * (2048 >> 4), idesc);
 }
 
 template <int D, bool BF16, bool CAUSAL>
@@ -253,7 +250,12 @@ __device__ __forceinline__ void mma_role(const FwdParams& p, uint32_t tmem, uint
                                          uint32_t sKV, uint32_t bars, volatile int* abort_flag) {
   using C = Cfg<D>;
   auto bar = [&](int i) { return bars + 8 * i; };
-  auto kv_addr = [&](int idx) { return sKV + (idx % C::kStages) * C::kTileBytes; };
+  // low descriptor halves: K tiles / Q tiles K-major (LBO unused, 16), V tiles MN-major (LBO = chunk)
+  const uint32_t q_lo0 = smem_desc_lo(sQ, 16), q_lo1 = smem_desc_lo(sQ + C::kTileBytes, 16);
+  auto k_lo = [&](int idx) { return smem_desc_lo(sKV + (idx % C::kStages) * C::kTileBytes, 16); };
+  auto v_lo = [&](int idx) {
+    return smem_desc_lo(sKV + (idx % C::kStages) * C::kTileBytes, C::kChunkBytes);
+  };
   auto kv_full = [&](int idx) {
     return mbar_wait(bar(kBarKvFull + idx % C::kStages), (idx / C::kStages) & 1, abort_flag,
                      kFaultMmaKvFull, p.timeout_ns);
@@ -269,9 +271,9 @@ __device__ __forceinline__ void mma_role(const FwdParams& p, uint32_t tmem, uint
     if (!ok) break;
     tc_fence_after_sync();
     // S_t(0) = Q_t K_0^T for both tiles
-    issue_qk<D, BF16>(tmem + C::col_s(0), sQ, kv_addr(kv_it));
+    issue_qk<D, BF16>(tmem + C::col_s(0), q_lo0, k_lo(kv_it));
     mma_commit(bar(kBarSFull + 0));
-    issue_qk<D, BF16>(tmem + C::col_s(1), sQ + C::kTileBytes, kv_addr(kv_it));
+    issue_qk<D, BF16>(tmem + C::col_s(1), q_lo1, k_lo(kv_it));
     mma_commit(bar(kBarSFull + 1));
     mma_commit(bar(kBarKvEmpty + kv_it % C::kStages));
     if (x.n0 == 1) mma_commit(bar(kBarQEmpty + 0));
@@ -290,14 +292,14 @@ __device__ __forceinline__ void mma_role(const FwdParams& p, uint32_t tmem, uint
         }
         ++pcnt[0];
         tc_fence_after_sync();
-        issue_pv<D, BF16>(tmem + C::col_o(0), tmem + C::col_s(0), kv_addr(vidx), j > 0);
+        issue_pv<D, BF16>(tmem + C::col_o(0), tmem + C::col_s(0), v_lo(vidx), j > 0 ? 1u : 0u);
         if (j == x.n0 - 1) {
           mma_commit(bar(kBarOFull + 0));
         } else {
           if (!kv_full(knext)) { ok = false; break; }
           k_ready = true;
           tc_fence_after_sync();
-          issue_qk<D, BF16>(tmem + C::col_s(0), sQ, kv_addr(knext));
+          issue_qk<D, BF16>(tmem + C::col_s(0), q_lo0, k_lo(knext));
           mma_commit(bar(kBarSFull + 0));
           if (j + 1 == x.n0 - 1) mma_commit(bar(kBarQEmpty + 0));
         }
@@ -308,7 +310,7 @@ __device__ __forceinline__ void mma_role(const FwdParams& p, uint32_t tmem, uint
       }
       ++pcnt[1];
       tc_fence_after_sync();
-      issue_pv<D, BF16>(tmem + C::col_o(1), tmem + C::col_s(1), kv_addr(vidx), j > 0);
+      issue_pv<D, BF16>(tmem + C::col_o(1), tmem + C::col_s(1), v_lo(vidx), j > 0 ? 1u : 0u);
       mma_commit(bar(kBarKvEmpty + vidx % C::kStages));
       if (j == x.n1 - 1) {
         mma_commit(bar(kBarOFull + 1));
@@ -317,7 +319,7 @@ __device__ __forceinline__ void mma_role(const FwdParams& p, uint32_t tmem, uint
           if (!kv_full(knext)) { ok = false; break; }
           tc_fence_after_sync();
         }
-        issue_qk<D, BF16>(tmem + C::col_s(1), sQ + C::kTileBytes, kv_addr(knext));
+        issue_qk<D, BF16>(tmem + C::col_s(1), q_lo1, k_lo(knext));
         mma_commit(bar(kBarSFull + 1));
         mma_commit(bar(kBarKvEmpty + knext % C::kStages));
         if (j + 1 == x.n1 - 1) mma_commit(bar(kBarQEmpty + 1));
@@ -574,7 +576,7 @@ __global__ void __launch_bounds__(128, 1)
     ok = mbar_wait(bars, 0, abort_flag, kFaultSelftest, timeout_ns);
     if (ok) {
       tc_fence_after_sync();
-      issue_qk<D, BF16>(tmem + 0, sQ, sK);
+      issue_qk<D, BF16>(tmem + 0, smem_desc_lo(sQ, 16), smem_desc_lo(sK, 16));
     }
     mma_commit(bars + 8);
   }
@@ -598,7 +600,7 @@ __global__ void __launch_bounds__(128, 1)
   __syncthreads();
   if (threadIdx.x == 0) {
     tc_fence_after_sync();
-    if (!*abort_flag) issue_pv<D, BF16>(tmem + 256, tmem + 0, sV, false);
+    if (!*abort_flag) issue_pv<D, BF16>(tmem + 256, tmem + 0, smem_desc_lo(sV, C::kChunkBytes), 0u);
     mma_commit(bars + 8);
   }
   ok = !*abort_flag && mbar_wait(bars + 8, 1, abort_flag, kFaultSelftest, timeout_ns);

@@ -115,19 +115,10 @@ __device__ __forceinline__ void tmem_wait_st() {
 
 // ------------------------------------------------------------ tcgen05.mma
 
-// Shared-memory matrix descriptor for a tile stored with the 128-byte swizzle
-// (rows of 128 bytes, 8-row atoms of 1024 bytes), sm_100 descriptor version 1.
-//   lbo: leading-dimension byte offset, sbo: stride-dimension byte offset.
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-  uint64_t d = 0;
-  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
-  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
-  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
-  d |= static_cast<uint64_t>(1) << 46;  // descriptor version (sm_100)
-  d |= static_cast<uint64_t>(2) << 61;  // swizzle mode: 128 B
-  return d;
-}
-
+// Shared-memory matrix descriptor (64 bits) of a tile stored with the 128-byte
+// swizzle (rows of 128 bytes, 8-row atoms of 1024 bytes), sm_100 version 1:
+//   bits  0-13 start address >> 4     bits 16-29 leading-dimension byte offset >> 4
+//   bits 32-45 stride byte offset >> 4  bit 46 version = 1   bits 61-63 swizzle (2 = 128 B)
 // Instruction descriptor of tcgen05.mma.kind::f16 with an F32 accumulator.
 //   bf16: operand type (else fp16); a_mn / b_mn: operand stored MN-major.
 __host__ __device__ constexpr uint32_t mma_idesc_f16(bool bf16, int M, int N, bool a_mn, bool b_mn) {
@@ -140,25 +131,50 @@ __host__ __device__ constexpr uint32_t mma_idesc_f16(bool bf16, int M, int N, bo
          | (static_cast<uint32_t>(M >> 4) << 24);   // M / 16
 }
 
-// D[tmem] (+)= A[smem] * B[smem]^T, one CTA, issued by one thread.
-__device__ __forceinline__ void mma_f16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                           uint32_t idesc, uint32_t accumulate) {
+// The descriptor split into 32-bit halves. The high half (SBO = 1024,
+// version, 128-byte swizzle) is common to every operand tile here; the low half
+// carries the start address and LBO, so advancing along K is one 32-bit add.
+constexpr uint32_t kSmemDescHiSw128 = (1024u >> 4) | (1u << 14) | (2u << 29);
+__device__ __forceinline__ uint32_t smem_desc_lo(uint32_t saddr, uint32_t lbo) {
+  return ((saddr >> 4) & 0x3FFFu) | (((lbo >> 4) & 0x3FFFu) << 16);
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, descriptors given as low halves + common high half.
+template <bool ACC>
+__device__ __forceinline__ void mma_f16_ss_lo(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo,
+                                              uint32_t idesc) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "mov.b64 da, {%1, %3};\n\t"
+      "mov.b64 db, {%2, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %4, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_lo), "r"(b_lo), "n"(kSmemDescHiSw128), "r"(idesc), "n"(ACC ? 1 : 0)
       : "memory");
 }
 
-// D[tmem] (+)= A[tmem] * B[smem], A read from tensor memory.
-__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                           uint32_t idesc, uint32_t accumulate) {
+// D[tmem] (+)= A[tmem] * B[smem], B descriptor given as its low half.
+template <bool ACC>
+__device__ __forceinline__ void mma_f16_ts_lo(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo,
+                                              uint32_t idesc) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
+      "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
-      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      "mov.b64 db, {%2, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %5, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "r"(b_lo), "n"(kSmemDescHiSw128), "n"(ACC ? 1 : 0), "r"(idesc)
+      : "memory");
+}
+
+// Runtime accumulate flag (first PV of a unit overwrites O).
+__device__ __forceinline__ void mma_f16_ts_lo_flag(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo,
+                                                   uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "mov.b64 db, {%2, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %5, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "r"(b_lo), "n"(kSmemDescHiSw128), "r"(acc), "r"(idesc)
       : "memory");
 }
 
