@@ -370,18 +370,20 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
 
       const int lim = row_lim - j * kTileRows;  // keys c < lim of this tile are visible
       const bool partial = lim < kTileRows;
-      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
       if (partial) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          const float s = c < lim ? __uint_as_float(r[c]) : -INFINITY;
-          mx[c & 3] = fmaxf(mx[c & 3], s);
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < 128; ++c) mx[c & 3] = fmaxf(mx[c & 3], __uint_as_float(r[c]));
+        for (int c = 0; c < 128; ++c)
+          if (c >= lim) r[c] = __float_as_uint(-INFINITY);
       }
-      const float m_tile = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+      // row max: four independent chains of three-input max
+      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int c = 0; c < 128; c += 8) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          mx[q] = fmax3(mx[q], __uint_as_float(r[c + 2 * q]), __uint_as_float(r[c + 2 * q + 1]));
+      }
+      const float m_tile = fmax3(mx[0], mx[1], fmaxf(mx[2], mx[3]));
       const float m_scaled = (m_tile == -INFINITY) ? -INFINITY : m_tile * sl2;
 
       // lazy rescale: move the reference only when the max grew by > tau
@@ -394,34 +396,51 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
       }
       if (__any_sync(0xffffffffu, rescale && j > 0)) {
         const float a = (rescale && j > 0) ? alpha : 1.f;
+        const uint64_t a2 = f2_pack(a, a);
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           uint32_t ov[32];
           tmem_ld_32x32b_x32(tO + 32 * c, ov);
           tmem_wait_ld_x32(ov);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * a);
+          for (int e = 0; e < 32; e += 2) {
+            float lo, hi;
+            f2_unpack(f2_mul(f2_pack_bits(ov[e], ov[e + 1]), a2), lo, hi);
+            ov[e] = __float_as_uint(lo);
+            ov[e + 1] = __float_as_uint(hi);
+          }
           tmem_st_32x32b_x32(tO + 32 * c, ov);
         }
         tmem_wait_st();
       }
 
-      // P = exp2(s * sl2 - ref), packed to 16 bits into the first 64 columns of S
-      const float neg_ref = -ref;
-      float sum[4] = {0.f, 0.f, 0.f, 0.f};
+      // P = exp2(s * sl2 - ref), packed to 16 bits into the first 64 columns of
+      // S. On partial tiles the masked keys are zeroed after the exponential
+      // (their -inf scores times a zero scale, or -inf + inf when the row has
+      // no visible key yet, would give NaN).
+      const uint64_t sl2_2 = f2_pack(sl2, sl2);
+      const uint64_t nref2 = f2_pack(-ref, -ref);
+      uint64_t acc2[2] = {0ull, 0ull};
       uint32_t pk[64];
 #pragma unroll
-      for (int c = 0; c < 128; c += 2) {
-        float p0 = ex2_approx(fmaf(__uint_as_float(r[c]), sl2, neg_ref));
-        float p1 = ex2_approx(fmaf(__uint_as_float(r[c + 1]), sl2, neg_ref));
+      for (int c = 0; c < 64; ++c) {
+        float x0, x1;
+        f2_unpack(f2_fma(f2_pack_bits(r[2 * c], r[2 * c + 1]), sl2_2, nref2), x0, x1);
+        float p0 = ex2_approx(x0);
+        float p1 = ex2_approx(x1);
         if (partial) {
-          p0 = c < lim ? p0 : 0.f;
-          p1 = c + 1 < lim ? p1 : 0.f;
+          p0 = 2 * c < lim ? p0 : 0.f;
+          p1 = 2 * c + 1 < lim ? p1 : 0.f;
         }
-        sum[(c >> 1) & 3] += p0 + p1;
-        pk[c >> 1] = pack2<BF16>(p0, p1);
+        acc2[c & 1] = f2_add(acc2[c & 1], f2_pack(p0, p1));
+        pk[c] = pack2<BF16>(p0, p1);
       }
-      l += (sum[0] + sum[1]) + (sum[2] + sum[3]);
+      {
+        float a0, a1, b0, b1;
+        f2_unpack(acc2[0], a0, a1);
+        f2_unpack(acc2[1], b0, b1);
+        l += (a0 + a1) + (b0 + b1);
+      }
       tmem_st_32x32b_x32(tS, pk);
       tmem_st_32x32b_x32(tS + 32, pk + 32);
       tmem_wait_st();

@@ -183,6 +183,21 @@ def test_video_zero_scale_closed_form_every_row(video):
     assert (lse.double() - math.log(w.Lk)).abs().max() <= 1e-4
 
 
+@pytest.mark.parametrize("mask,off", [(1, 133), (2, 100), (1, 0)])
+def test_zero_scale_masked_closed_form(mask, off):
+    # scale 0 with a mask: row i is the mean of its visible V rows, LSE = ln(count);
+    # exercises partial tiles where masked scores meet a zero scale
+    Lq, Lk = 200, 333
+    q, k, v = inputs.make_qkv(1, Lq, Lk, 2, 1, 128, torch.bfloat16, seed=21)
+    o, lse = _gpu(q, k, v, 0.0, mask, off)
+    vd = v.double()
+    for i in range(Lq):
+        n = min(Lk, off + i + 1) if mask == 1 else off + Lq
+        ref = vd[0, :n, 0].mean(dim=0)
+        assert (o[0, i].double() - ref).abs().max() <= 8e-3, (i, n)
+        assert abs(float(lse[0, 0, i]) - math.log(n)) <= 1e-4
+
+
 # ---------------------------------------------------------------- invariants
 
 def test_deterministic_bitwise():
