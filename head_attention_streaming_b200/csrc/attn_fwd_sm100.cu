@@ -15,8 +15,9 @@
 //   warps 0-3   softmax for query tile 0 (rows r0 .. r0+127 of a work unit)
 //   warps 4-7   softmax for query tile 1 (rows r0+128 .. r0+255)
 //   warp  8     TMA producer: Q tiles, then K_0, V_0, K_1, V_1, ... into a ring
-//   warp  9     MMA issuer (one thread): S_t = Q_t K^T and O_t += P_t V
-//   warps 10-11 idle
+//   warps 9, 10 MMA issuers (one thread each), warp 9 + t for query tile t:
+//               S_t = Q_t K^T and O_t += P_t V
+//   warp  11    idle
 // A work unit is (batch, query head, 256-row pair of query tiles). Tensor
 // memory holds S_0, S_1 (128 fp32 columns each, P aliased as packed 16-bit in
 // the first 64 columns) and O_0, O_1 (d columns each).
@@ -46,6 +47,7 @@ enum FaultBit : unsigned int {
   kFaultMmaPFull = 1u << 4,
   kFaultSoftmaxSFull = 1u << 5,
   kFaultSoftmaxOFull = 1u << 6,
+  kFaultSoftmaxTurn = 1u << 7,
   kFaultSelftest = 1u << 8,
 };
 
@@ -81,11 +83,13 @@ enum Bar : int {
   kBarQFull = 0,    // [2] TMA -> MMA: Q tile t landed
   kBarQEmpty = 2,   // [2] MMA -> TMA: last S_t of the unit done, Q tile t reusable
   kBarSFull = 4,    // [2] MMA -> softmax t: S_t ready (also: previous PV_t done)
-  kBarPFull = 6,    // [2] softmax t -> MMA: P_t written (128 arrivals)
+  kBarPFull = 6,    // [2] softmax t -> MMA: all of P_t written (one arrival per warp)
   kBarOFull = 8,    // [2] MMA -> softmax t: O_t final for the unit
-  kBarDrain = 10,   //     MMA abort path: all issued MMAs done
+  kBarDrain = 10,   // [2] MMA issuer t, abort path: all its MMAs done
+  kBarPHalf = 12,   // [2] softmax t -> MMA: first half of P_t (keys 0-63) written
+  kBarTurn = 14,    // [2] softmax 1-t -> softmax t: t may run its exponentials now
   kBarKvFull = 16,  // [kStages] TMA -> MMA
-  kBarKvEmpty = 24, // [kStages] MMA -> TMA
+  kBarKvEmpty = 24, // [kStages] both MMA issuers -> TMA
 };
 
 struct FwdParams {
@@ -178,17 +182,30 @@ __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_lo, uint32_
   }
 }
 
-// O[tmem] (+)= P[tmem] V over 128 keys: 8 MMAs of 128xDx16. P is packed 16-bit
-// in tensor memory (two keys per column); V is MN-major (d contiguous): 8-key
-// groups 1024 bytes apart (SBO), 64-column d chunks one chunk apart (LBO), so
-// 16 keys advance the start address by 2048 bytes.
+// O[tmem] (+)= P[tmem] V over 128 keys: 8 MMAs of 128xDx16, issued as two halves
+// of 64 keys so the first half can start while the softmax still writes the
+// second. P is packed 16-bit in tensor memory (two keys per column); V is
+// MN-major (d contiguous): 8-key groups 1024 bytes apart (SBO), 64-column d
+// chunks one chunk apart (LBO), so 16 keys advance the start address by 2048 B.
+template <int D, bool BF16, int HALF>
+__device__ __forceinline__ void issue_pv_half(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_lo,
+                                              uint32_t accumulate) {
+  constexpr uint32_t idesc = mma_idesc_f16(BF16, 128, D, false, true);
+  if constexpr (HALF == 0) {
+    mma_f16_ts_lo_flag(d_tmem, p_tmem, v_lo, idesc, accumulate);
+  } else {
+    mma_f16_ts_lo<true>(d_tmem, p_tmem + 32, v_lo + 4 * (2048 >> 4), idesc);
+  }
+#pragma unroll
+  for (int kk = HALF * 4 + 1; kk < HALF * 4 + 4; ++kk)
+    mma_f16_ts_lo<true>(d_tmem, p_tmem + kk * 8, v_lo + kk * (2048 >> 4), idesc);
+}
+
 template <int D, bool BF16>
 __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_lo,
                                          uint32_t accumulate) {
-  constexpr uint32_t idesc = mma_idesc_f16(BF16, 128, D, false, true);
-  mma_f16_ts_lo_flag(d_tmem, p_tmem, v_lo, idesc, accumulate);
-#pragma unroll
-  for (int kk = 1; kk < 8; ++kk) mma_f16_ts_lo<true>(d_tmem, p_tmem + kk * 8, v_lo + kk * (2048 >> 4), idesc);
+  issue_pv_half<D, BF16, 0>(d_tmem, p_tmem, v_lo, accumulate);
+  issue_pv_half<D, BF16, 1>(d_tmem, p_tmem, v_lo, 1u);
 }
 
 template <int D, bool BF16, bool CAUSAL>
@@ -245,92 +262,89 @@ __device__ __forceinline__ void load_role(const CUtensorMap* tm_q, const CUtenso
   }
 }
 
+// One MMA issuer per query tile t (warps 9 and 10). A single issuing thread
+// serialises both tiles: every tcgen05.mma holds its thread about as long as the
+// tensor core takes to run it, so one thread cannot wait for one tile's P while
+// issuing the other's GEMMs. With one thread per tile, the tensor core runs
+// whichever tile has work. Both threads read the same K/V ring slots; each slot
+// use is released by both (kv_empty takes two arrivals).
 template <int D, bool BF16, bool CAUSAL>
-__device__ __forceinline__ void mma_role(const FwdParams& p, uint32_t tmem, uint32_t sQ,
+__device__ __forceinline__ void mma_role(const int t, const FwdParams& p, uint32_t tmem, uint32_t sQ,
                                          uint32_t sKV, uint32_t bars, volatile int* abort_flag) {
   using C = Cfg<D>;
   auto bar = [&](int i) { return bars + 8 * i; };
-  // low descriptor halves: K tiles / Q tiles K-major (LBO unused, 16), V tiles MN-major (LBO = chunk)
-  const uint32_t q_lo0 = smem_desc_lo(sQ, 16), q_lo1 = smem_desc_lo(sQ + C::kTileBytes, 16);
+  // low descriptor halves: Q and K tiles K-major (LBO unused, 16), V tiles MN-major (LBO = chunk)
+  const uint32_t q_lo = smem_desc_lo(sQ + t * C::kTileBytes, 16);
   auto k_lo = [&](int idx) { return smem_desc_lo(sKV + (idx % C::kStages) * C::kTileBytes, 16); };
   auto v_lo = [&](int idx) {
     return smem_desc_lo(sKV + (idx % C::kStages) * C::kTileBytes, C::kChunkBytes);
   };
+  // K/V tiles are written by TMA (async proxy) and read by the MMA (async proxy):
+  // the barrier's transaction count orders them, no tcgen05 fence is needed
   auto kv_full = [&](int idx) {
     return mbar_wait(bar(kBarKvFull + idx % C::kStages), (idx / C::kStages) & 1, abort_flag,
                      kFaultMmaKvFull, p.timeout_ns);
   };
-  int kv_it = 0, uit = 0;
-  int pcnt[2] = {0, 0};
+  const uint32_t s_t = tmem + C::col_s(t), o_t = tmem + C::col_o(t);
+  int kv_it = 0, uit = 0, pcnt = 0;
   bool ok = true;
   for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++uit) {
     const Unit x = decode_unit<CAUSAL>(p, u);
-    ok = mbar_wait(bar(kBarQFull + 0), uit & 1, abort_flag, kFaultMmaQFull, p.timeout_ns) &&
-         mbar_wait(bar(kBarQFull + 1), uit & 1, abort_flag, kFaultMmaQFull, p.timeout_ns) &&
+    const int n = t ? x.n1 : x.n0;  // KV tiles this query tile uses (n0 <= n1)
+    ok = mbar_wait(bar(kBarQFull + t), uit & 1, abort_flag, kFaultMmaQFull, p.timeout_ns) &&
          kv_full(kv_it);
     if (!ok) break;
-    tc_fence_after_sync();
-    // S_t(0) = Q_t K_0^T for both tiles
-    issue_qk<D, BF16>(tmem + C::col_s(0), q_lo0, k_lo(kv_it));
-    mma_commit(bar(kBarSFull + 0));
-    issue_qk<D, BF16>(tmem + C::col_s(1), q_lo1, k_lo(kv_it));
-    mma_commit(bar(kBarSFull + 1));
+    // S_t(0) = Q_t K_0^T
+    issue_qk<D, BF16>(s_t, q_lo, k_lo(kv_it));
+    mma_commit(bar(kBarSFull + t));
     mma_commit(bar(kBarKvEmpty + kv_it % C::kStages));
-    if (x.n0 == 1) mma_commit(bar(kBarQEmpty + 0));
-    if (x.n1 == 1) mma_commit(bar(kBarQEmpty + 1));
-
-    for (int j = 0; j < x.n1 && ok; ++j) {
+    if (n == 1) mma_commit(bar(kBarQEmpty + t));
+    for (int j = 0; j < n; ++j) {
       const int vidx = kv_it + 2 * j + 1;  // V_j
       const int knext = vidx + 1;          // K_{j+1}
-      bool k_ready = false;
-      if (!kv_full(vidx)) { ok = false; break; }
-      tc_fence_after_sync();
-      if (j < x.n0) {
-        if (!mbar_wait(bar(kBarPFull + 0), pcnt[0] & 1, abort_flag, kFaultMmaPFull, p.timeout_ns)) {
-          ok = false;
-          break;
-        }
-        ++pcnt[0];
-        tc_fence_after_sync();
-        issue_pv<D, BF16>(tmem + C::col_o(0), tmem + C::col_s(0), v_lo(vidx), j > 0 ? 1u : 0u);
-        if (j == x.n0 - 1) {
-          mma_commit(bar(kBarOFull + 0));
-        } else {
-          if (!kv_full(knext)) { ok = false; break; }
-          k_ready = true;
-          tc_fence_after_sync();
-          issue_qk<D, BF16>(tmem + C::col_s(0), q_lo0, k_lo(knext));
-          mma_commit(bar(kBarSFull + 0));
-          if (j + 1 == x.n0 - 1) mma_commit(bar(kBarQEmpty + 0));
-        }
-      }
-      if (!mbar_wait(bar(kBarPFull + 1), pcnt[1] & 1, abort_flag, kFaultMmaPFull, p.timeout_ns)) {
+      // O_t += P_t V_j: the first 64 keys as soon as their half of P is in
+      // tensor memory, the rest once all of P is
+      if (!kv_full(vidx) ||
+          !mbar_wait(bar(kBarPHalf + t), pcnt & 1, abort_flag, kFaultMmaPFull, p.timeout_ns)) {
         ok = false;
         break;
       }
-      ++pcnt[1];
       tc_fence_after_sync();
-      issue_pv<D, BF16>(tmem + C::col_o(1), tmem + C::col_s(1), v_lo(vidx), j > 0 ? 1u : 0u);
+      issue_pv_half<D, BF16, 0>(o_t, s_t, v_lo(vidx), j > 0 ? 1u : 0u);
+      if (!mbar_wait(bar(kBarPFull + t), pcnt & 1, abort_flag, kFaultMmaPFull, p.timeout_ns)) {
+        ok = false;
+        break;
+      }
+      ++pcnt;
+      tc_fence_after_sync();
+      issue_pv_half<D, BF16, 1>(o_t, s_t, v_lo(vidx), 1u);
       mma_commit(bar(kBarKvEmpty + vidx % C::kStages));
-      if (j == x.n1 - 1) {
-        mma_commit(bar(kBarOFull + 1));
+      if (j == n - 1) {
+        mma_commit(bar(kBarOFull + t));
       } else {
-        if (!k_ready) {
-          if (!kv_full(knext)) { ok = false; break; }
-          tc_fence_after_sync();
-        }
-        issue_qk<D, BF16>(tmem + C::col_s(1), q_lo1, k_lo(knext));
-        mma_commit(bar(kBarSFull + 1));
+        if (!kv_full(knext)) { ok = false; break; }
+        issue_qk<D, BF16>(s_t, q_lo, k_lo(knext));
+        mma_commit(bar(kBarSFull + t));
         mma_commit(bar(kBarKvEmpty + knext % C::kStages));
-        if (j + 1 == x.n1 - 1) mma_commit(bar(kBarQEmpty + 1));
+        if (j + 1 == n - 1) mma_commit(bar(kBarQEmpty + t));
+      }
+    }
+    // causal: tiles this query tile never sees (n <= j < n1) still pass through
+    // the ring; release this thread's share once each has landed (waiting for
+    // the landing keeps the arrival in the slot's current phase)
+    for (int j = n; j < x.n1 && ok; ++j) {
+      for (int kv = 0; kv < 2 && ok; ++kv) {
+        const int idx = kv_it + 2 * j + kv;
+        if (!kv_full(idx)) { ok = false; break; }
+        mbar_arrive(bar(kBarKvEmpty + idx % C::kStages));
       }
     }
     kv_it += 2 * x.n1;
   }
   if (!ok) {
-    // every MMA issued so far must finish before tensor memory is freed
-    mma_commit(bar(kBarDrain));
-    mbar_drain(bar(kBarDrain), 0);
+    // every MMA this thread issued must finish before tensor memory is freed
+    mma_commit(bar(kBarDrain + t));
+    mbar_drain(bar(kBarDrain + t), 0);
   }
 }
 
@@ -345,6 +359,11 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
   const uint32_t tO = tmem + lane_bits + C::col_o(t);
   const uint32_t bar_s = bars + 8 * (kBarSFull + t);
   const uint32_t bar_p = bars + 8 * (kBarPFull + t);
+  const uint32_t bar_ph = bars + 8 * (kBarPHalf + t);
+  const uint32_t bar_turn_mine = bars + 8 * (kBarTurn + t);
+  const uint32_t bar_turn_other = bars + 8 * (kBarTurn + (1 - t));
+  int tcnt = 0;
+  const int lane = threadIdx.x % 32;
   const uint32_t bar_o = bars + 8 * (kBarOFull + t);
   const float sl2 = p.sl2;
   int scnt = 0, ocnt = 0;
@@ -375,65 +394,102 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
         for (int c = 0; c < 128; ++c)
           if (c >= lim) r[c] = __float_as_uint(-INFINITY);
       }
-      // row max: four independent chains of three-input max
-      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      // row max: a three-input max tree (depth 5) over the 128 scores
+      float m_tile;
+      {
+        float a[43];
 #pragma unroll
-      for (int c = 0; c < 128; c += 8) {
+        for (int i = 0; i < 42; ++i)
+          a[i] = fmax3(__uint_as_float(r[3 * i]), __uint_as_float(r[3 * i + 1]), __uint_as_float(r[3 * i + 2]));
+        a[42] = fmaxf(__uint_as_float(r[126]), __uint_as_float(r[127]));
+        float b[15];
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          mx[q] = fmax3(mx[q], __uint_as_float(r[c + 2 * q]), __uint_as_float(r[c + 2 * q + 1]));
+        for (int i = 0; i < 14; ++i) b[i] = fmax3(a[3 * i], a[3 * i + 1], a[3 * i + 2]);
+        b[14] = a[42];
+        float c5[5];
+#pragma unroll
+        for (int i = 0; i < 5; ++i) c5[i] = fmax3(b[3 * i], b[3 * i + 1], b[3 * i + 2]);
+        m_tile = fmaxf(fmax3(c5[0], c5[1], c5[2]), fmaxf(c5[3], c5[4]));
       }
-      const float m_tile = fmax3(mx[0], mx[1], fmaxf(mx[2], mx[3]));
       const float m_scaled = (m_tile == -INFINITY) ? -INFINITY : m_tile * sl2;
 
-      // lazy rescale: move the reference only when the max grew by > tau
+      // lazy rescale: move the reference only when the max grew by > tau; after
+      // the first tiles of a row this almost never fires, so the warp takes the
+      // branch only when one of its rows needs it
       const bool rescale = m_scaled > ref + kRescaleTau;
-      float alpha = 1.f;
-      if (rescale) {
-        alpha = ex2_approx(ref - m_scaled);
-        ref = m_scaled;
-        l *= alpha;
-      }
-      if (__any_sync(0xffffffffu, rescale && j > 0)) {
-        const float a = (rescale && j > 0) ? alpha : 1.f;
-        const uint64_t a2 = f2_pack(a, a);
-#pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t ov[32];
-          tmem_ld_32x32b_x32(tO + 32 * c, ov);
-          tmem_wait_ld_x32(ov);
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            float lo, hi;
-            f2_unpack(f2_mul(f2_pack_bits(ov[e], ov[e + 1]), a2), lo, hi);
-            ov[e] = __float_as_uint(lo);
-            ov[e + 1] = __float_as_uint(hi);
-          }
-          tmem_st_32x32b_x32(tO + 32 * c, ov);
+      if (__any_sync(0xffffffffu, rescale)) {
+        float alpha = 1.f;
+        if (rescale) {
+          alpha = ex2_approx(ref - m_scaled);
+          ref = m_scaled;
+          l *= alpha;
         }
-        tmem_wait_st();
+        if (j > 0) {
+          const uint64_t a2 = f2_pack(alpha, alpha);
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t ov[32];
+            tmem_ld_32x32b_x32(tO + 32 * c, ov);
+            tmem_wait_ld_x32(ov);
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              float lo, hi;
+              f2_unpack(f2_mul(f2_pack_bits(ov[e], ov[e + 1]), a2), lo, hi);
+              ov[e] = __float_as_uint(lo);
+              ov[e + 1] = __float_as_uint(hi);
+            }
+            tmem_st_32x32b_x32(tO + 32 * c, ov);
+          }
+          tmem_wait_st();
+        }
+      }
+
+      // Ping-pong: the two softmax warpgroups take turns for their exponentials
+      // (tile 0 of KV tile j, then tile 1 of j, then tile 0 of j + 1, ...), so
+      // the MUFU serves one of them at a time and each tile's GEMMs run on the
+      // tensor core while the other tile computes. Waits and arrivals pair up:
+      // turn[1] gets one arrival per KV tile tile 0 processes (n0 per unit),
+      // turn[0] one per tile 1 processes below n0 - 1.
+      if (t == 0 ? j >= 1 : j < x.n0) {
+        bool ok_turn = mbar_wait(bar_turn_mine, tcnt & 1, abort_flag, kFaultSoftmaxTurn, p.timeout_ns);
+        if (!__all_sync(0xffffffffu, ok_turn)) return;
+        ++tcnt;
       }
 
       // P = exp2(s * sl2 - ref), packed to 16 bits into the first 64 columns of
-      // S. On partial tiles the masked keys are zeroed after the exponential
-      // (their -inf scores times a zero scale, or -inf + inf when the row has
-      // no visible key yet, would give NaN).
+      // S, in two halves of 64 keys, each handed to the MMA thread as soon as it
+      // is in tensor memory (one arrival per warp). On partial tiles the masked
+      // keys are zeroed after the exponential (their -inf scores times a zero
+      // scale, or -inf + inf when the row has no visible key yet, would give NaN).
       const uint64_t sl2_2 = f2_pack(sl2, sl2);
       const uint64_t nref2 = f2_pack(-ref, -ref);
       uint64_t acc2[2] = {0ull, 0ull};
-      uint32_t pk[64];
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        float x0, x1;
-        f2_unpack(f2_fma(f2_pack_bits(r[2 * c], r[2 * c + 1]), sl2_2, nref2), x0, x1);
-        float p0 = ex2_approx(x0);
-        float p1 = ex2_approx(x1);
-        if (partial) {
-          p0 = 2 * c < lim ? p0 : 0.f;
-          p1 = 2 * c + 1 < lim ? p1 : 0.f;
+      for (int h = 0; h < 2; ++h) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int cc = 0; cc < 32; ++cc) {
+          const int c = 32 * h + cc;
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack_bits(r[2 * c], r[2 * c + 1]), sl2_2, nref2), x0, x1);
+          float p0 = ex2_approx(x0);
+          float p1 = ex2_approx(x1);
+          if (partial) {
+            p0 = 2 * c < lim ? p0 : 0.f;
+            p1 = 2 * c + 1 < lim ? p1 : 0.f;
+          }
+          acc2[cc & 1] = f2_add(acc2[cc & 1], f2_pack(p0, p1));
+          pk[cc] = pack2<BF16>(p0, p1);
         }
-        acc2[c & 1] = f2_add(acc2[c & 1], f2_pack(p0, p1));
-        pk[c] = pack2<BF16>(p0, p1);
+        if (h == 1 && (t == 0 || j + 1 < x.n0)) {  // exponentials done: hand over the turn
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_turn_other);
+        }
+        tmem_st_32x32b_x32(tS + 32 * h, pk);
+        tmem_wait_st();
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(h == 0 ? bar_ph : bar_p);
       }
       {
         float a0, a1, b0, b1;
@@ -441,11 +497,6 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
         f2_unpack(acc2[1], b0, b1);
         l += (a0 + a1) + (b0 + b1);
       }
-      tmem_st_32x32b_x32(tS, pk);
-      tmem_st_32x32b_x32(tS + 32, pk + 32);
-      tmem_wait_st();
-      tc_fence_before_sync();
-      mbar_arrive(bar_p);
     }
 
     // epilogue: O / l to 16-bit, 16-byte stores; LSE
@@ -500,13 +551,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bars + 8 * (kBarQFull + t), 1);
       mbar_init(bars + 8 * (kBarQEmpty + t), 1);
       mbar_init(bars + 8 * (kBarSFull + t), 1);
-      mbar_init(bars + 8 * (kBarPFull + t), kTileRows);
+      mbar_init(bars + 8 * (kBarPFull + t), kTileRows / 32);
+      mbar_init(bars + 8 * (kBarPHalf + t), kTileRows / 32);
+      mbar_init(bars + 8 * (kBarTurn + t), kTileRows / 32);
       mbar_init(bars + 8 * (kBarOFull + t), 1);
     }
     mbar_init(bars + 8 * kBarDrain, 1);
+    mbar_init(bars + 8 * (kBarDrain + 1), 1);
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(bars + 8 * (kBarKvFull + s), 1);
-      mbar_init(bars + 8 * (kBarKvEmpty + s), 1);
+      mbar_init(bars + 8 * (kBarKvEmpty + s), 2);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -532,8 +586,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     regs_decrease<kRegsProducer>();
     if (warp == 8) {
       if (lane == 0) load_role<D, BF16, CAUSAL>(&tm_q, &tm_k, &tm_v, p, sQ, sKV, bars, abort_flag);
-    } else if (warp == 9) {
-      if (lane == 0) mma_role<D, BF16, CAUSAL>(p, tmem, sQ, sKV, bars, abort_flag);
+    } else if (warp == 9 || warp == 10) {
+      if (lane == 0) mma_role<D, BF16, CAUSAL>(warp - 9, p, tmem, sQ, sKV, bars, abort_flag);
     }
   }
   __syncwarp();
