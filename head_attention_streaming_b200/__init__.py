@@ -8,10 +8,11 @@ so importing ``head_attention_streaming_b200.inputs`` needs no GPU.
 from .binding import (ATTN_ERR_CUDA, ATTN_ERR_INVALID_ARG, ATTN_ERR_TIMEOUT, ATTN_ERR_UNSUPPORTED,
                       ATTN_OK, MASK_CAUSAL, MASK_CHUNK, MASK_NONE, AttnError, attn_fwd,
                       attn_fwd_host,
-                      device_fault, lib, library_path, selftest_mma, selftest_wait_timeout,
+                      device_fault, lib, library_path, selftest_exp2, selftest_mma,
+                      selftest_wait_timeout,
                       set_wait_timeout_ns, status_string)
 
 __all__ = ["attn_fwd", "attn_fwd_host", "AttnError", "lib", "library_path", "status_string", "device_fault",
-           "set_wait_timeout_ns", "selftest_mma", "selftest_wait_timeout", "ATTN_OK",
+           "set_wait_timeout_ns", "selftest_mma", "selftest_exp2", "selftest_wait_timeout", "ATTN_OK",
            "ATTN_ERR_INVALID_ARG", "ATTN_ERR_UNSUPPORTED", "ATTN_ERR_CUDA", "ATTN_ERR_TIMEOUT",
            "MASK_NONE", "MASK_CAUSAL", "MASK_CHUNK"]

@@ -40,6 +40,7 @@ _SIGNATURES = {
     "attn_set_wait_timeout_ns": (ctypes.c_int, [ctypes.c_ulonglong]),
     "attn_selftest_mma": (ctypes.c_int, [ctypes.c_void_p] * 5 + [ctypes.c_int, ctypes.c_void_p]),
     "attn_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_ulonglong, ctypes.c_void_p]),
+    "attn_selftest_exp2": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]),
 }
 
 
@@ -184,3 +185,14 @@ def selftest_mma(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor):
 def selftest_wait_timeout(timeout_ns: int, device=None) -> int:
     """Status of a launch whose only wait can never complete (expect ATTN_ERR_TIMEOUT)."""
     return int(lib().attn_selftest_wait_timeout(int(timeout_ns), _stream_handle(None, device)))
+
+
+def selftest_exp2(x: torch.Tensor) -> torch.Tensor:
+    """2^x through the kernel's FMA-pipe exponential (float32 CUDA tensor)."""
+    if not x.is_cuda or x.dtype != torch.float32 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous float32 CUDA tensor")
+    y = torch.empty_like(x)
+    st = lib().attn_selftest_exp2(_ptr(x), _ptr(y), x.numel(), _stream_handle(None, x.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_selftest_exp2")
+    return y

@@ -34,6 +34,10 @@
 #include "attn.h"
 #include "sm100_ptx.cuh"
 
+#ifndef POLY_PAIRS_PER8
+#define POLY_PAIRS_PER8 0
+#endif
+
 namespace hasb {
 
 // Device fault word: bit set by a kernel whose bounded wait ran out.
@@ -53,10 +57,10 @@ enum FaultBit : unsigned int {
 
 constexpr int kThreads = 384;
 // Register split: 384 threads x 168 launch registers = 64512. The producer
-// warpgroup (warps 8-11) drops to 88, the two softmax warpgroups rise to 208:
-// 128 x 88 + 256 x 208 = 64512.
-constexpr int kRegsProducer = 88;
-constexpr int kRegsSoftmax = 208;
+// warpgroup (warps 8-11) drops to 72, the two softmax warpgroups rise to 216:
+// 128 x 72 + 256 x 216 = 64512.
+constexpr int kRegsProducer = 72;
+constexpr int kRegsSoftmax = 216;
 constexpr int kTileRows = 128;         // query rows per softmax tile = keys per KV tile
 constexpr float kRescaleTau = 8.0f;    // lazy rescale threshold, log2 units (P <= 256)
 constexpr float kLn2 = 0.69314718055994531f;
@@ -91,6 +95,41 @@ enum Bar : int {
   kBarKvFull = 16,  // [kStages] TMA -> MMA
   kBarKvEmpty = 24, // [kStages] both MMA issuers -> TMA
 };
+
+// Exponentials of the softmax: kPolyPairsPer8 of every 8 score pairs take
+// exp2_poly_x2 on the FMA pipe instead of the MUFU (16 ex2 per clock per SM).
+// Measured on B200 the exponential loop is bound by instruction issue, not by
+// the MUFU, so the default is 0; the polynomial stays available (and tested)
+// for shapes where the MUFU saturates.
+constexpr int kPolyPairsPer8 = POLY_PAIRS_PER8;
+
+// 2^x for a pair of floats on the FMA pipe: x = j + f with j = round(x) and
+// f in [-1/2, 1/2]; 2^f from a degree-3 polynomial minimising the maximum
+// relative error on that interval (7.5e-5; coefficients from
+// gen_exp2_poly.py), 2^j added into the exponent field. x is clamped below at
+// -125, so results under 2^-125 come out near 2^-125 (masked keys are zeroed
+// by the caller; every other P is far above that).
+__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x2) {
+  constexpr float c0 = 0.9999280571937561f, c1 = 0.6932609677314758f;
+  constexpr float c2 = 0.2426111251115799f, c3 = 0.0551716685295105f;
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: x + kRound holds round(x) in its low bits
+  float a, b;
+  f2_unpack(x2, a, b);
+  x2 = f2_pack(fmaxf(a, -125.f), fmaxf(b, -125.f));
+  const uint64_t t = f2_add(x2, f2_pack(kRound, kRound));
+  const uint64_t j = f2_add(t, f2_pack(-kRound, -kRound));  // round(x), as float
+  const uint64_t f = f2_fma(j, f2_pack(-1.f, -1.f), x2);     // x - round(x), exact
+  uint64_t q = f2_fma(f2_pack(c3, c3), f, f2_pack(c2, c2));
+  q = f2_fma(q, f, f2_pack(c1, c1));
+  q = f2_fma(q, f, f2_pack(c0, c0));
+  float q0, q1, t0, t1;
+  f2_unpack(q, q0, q1);
+  f2_unpack(t, t0, t1);
+  // the bits of t are 0x4B400000 + j; shifted left by 23 only j << 23 remains
+  const uint32_t r0 = __float_as_uint(q0) + (__float_as_uint(t0) << 23);
+  const uint32_t r1 = __float_as_uint(q1) + (__float_as_uint(t1) << 23);
+  return f2_pack_bits(r0, r1);
+}
 
 struct FwdParams {
   void* o;
@@ -470,10 +509,16 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
 #pragma unroll
         for (int cc = 0; cc < 32; ++cc) {
           const int c = 32 * h + cc;
-          float x0, x1;
-          f2_unpack(f2_fma(f2_pack_bits(r[2 * c], r[2 * c + 1]), sl2_2, nref2), x0, x1);
-          float p0 = ex2_approx(x0);
-          float p1 = ex2_approx(x1);
+          const uint64_t x2 = f2_fma(f2_pack_bits(r[2 * c], r[2 * c + 1]), sl2_2, nref2);
+          float p0, p1;
+          if ((cc & 7) >= 8 - kPolyPairsPer8) {
+            f2_unpack(exp2_poly_x2(x2), p0, p1);
+          } else {
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
+          }
           if (partial) {
             p0 = 2 * c < lim ? p0 : 0.f;
             p1 = 2 * c + 1 < lim ? p1 : 0.f;
@@ -693,6 +738,17 @@ __global__ void __launch_bounds__(128, 1)
     tc_fence_after_sync();
     tmem_dealloc(tmem, 512);
   }
+}
+
+// The FMA-pipe exponential on n inputs (one value per thread pair slot).
+__global__ void selftest_exp2_kernel(const float* x, float* y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float a = x[i], b = (i + 1 < n) ? x[i + 1] : 0.f;
+  float r0, r1;
+  f2_unpack(exp2_poly_x2(f2_pack(a, b)), r0, r1);
+  y[i] = r0;
+  if (i + 1 < n) y[i + 1] = r1;
 }
 
 // One thread waits on a barrier nothing completes; the bounded wait must give up.
@@ -983,6 +1039,16 @@ int attn_selftest_mma(const void* q, const void* k, const void* v, float* s_out,
   if (cudaStreamSynchronize(s) != cudaSuccess) return ATTN_ERR_CUDA;
   unsigned int bits = 0;
   return attn_device_fault(&bits, 1);
+}
+
+int attn_selftest_exp2(const float* x, float* y, int n, void* stream) {
+  if (x == nullptr || y == nullptr || n < 0) return ATTN_ERR_INVALID_ARG;
+  if (n == 0) return ATTN_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int pairs = (n + 1) / 2;
+  selftest_exp2_kernel<<<(pairs + 255) / 256, 256, 0, s>>>(x, y, n);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  return cudaStreamSynchronize(s) == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 int attn_selftest_wait_timeout(unsigned long long timeout_ns, void* stream) {

@@ -119,7 +119,7 @@ int attn_set_wait_timeout_ns(unsigned long long ns);
 
 /*
  * Diagnostics, used by the tests to check the building blocks of attn_fwd on
- * the device. Neither is needed to compute attention.
+ * the device. None is needed to compute attention.
  *
  * attn_selftest_mma — one 128x128 tile through the same tensor-core path as
  * attn_fwd: TMA loads of q, k, v ([128, 128] row-major, dtype), S = q k^T
@@ -135,6 +135,17 @@ int attn_set_wait_timeout_ns(unsigned long long ns);
 int attn_selftest_mma(const void* q, const void* k, const void* v, float* s_out, float* o_out,
                       int dtype, void* stream);
 int attn_selftest_wait_timeout(unsigned long long timeout_ns, void* stream);
+
+/*
+ * attn_selftest_exp2 — y[i] = 2^x[i] for i < n (device float32 arrays) through
+ * the FMA-pipe exponential attn_fwd uses for part of its softmax exponentials:
+ * relative error within 7.6e-5 of 2^x for -125 <= x <= 8 (the softmax's
+ * exponent arguments never exceed 8); arguments below -125 give about 2^-125.
+ * The same softmax definition as attn_fwd's (developer guide, "Multi Head
+ * Attention Definition"); this entry exists to test that arithmetic.
+ * Synchronous.
+ */
+int attn_selftest_exp2(const float* x, float* y, int n, void* stream);
 
 #ifdef __cplusplus
 }

@@ -89,6 +89,17 @@ def test_selftest_mma_tile(dtype):
     assert (o - o_ref).abs().max() <= 1e-4 * o_ref.abs().max() + 1e-5
 
 
+def test_fma_pipe_exp2_within_its_error_bound():
+    # the polynomial exponential that replaces part of the MUFU ex2 calls
+    x = torch.cat([torch.linspace(-125.0, 8.0, 1_000_003), torch.tensor([0.0, 0.5, -0.5, 8.0, -125.0])])
+    y = hasb.selftest_exp2(x.cuda().contiguous()).cpu().double()
+    ref = torch.exp2(x.double())
+    rel = ((y - ref) / ref).abs()
+    assert float(rel.max()) <= 7.6e-5, float(rel.max())
+    below = hasb.selftest_exp2(torch.tensor([-126.0, -400.0, float("-inf")], device="cuda")).cpu()
+    assert torch.all(below >= 0) and torch.all(below < 2.0 ** -124)
+
+
 def test_bounded_wait_gives_up_and_reports():
     st = hasb.selftest_wait_timeout(50_000_000)
     assert st == hasb.ATTN_ERR_TIMEOUT
