@@ -387,6 +387,53 @@ __device__ __forceinline__ void mma_role(const int t, const FwdParams& p, uint32
   }
 }
 
+// P = exp2(s * sl2 - ref) for one row's 128 scores, packed to 16 bits into
+// the first 64 columns of S in two halves of 64 keys, each handed to the MMA
+// issuer (one arrival per warp) as soon as it is in tensor memory; the turn
+// goes to the other softmax warpgroup once the exponentials are done. Plain
+// scalar FMA/FADD keep the work on the FMA pipe (packed pairs cost register
+// moves on the ALU pipe here). MASKED: keys c >= lim are zeroed after the
+// exponential (their -inf scores times a zero scale, or -inf + inf when the
+// row has no visible key yet, would give NaN).
+template <bool BF16, bool MASKED>
+__device__ __forceinline__ void exp_tile(const uint32_t (&r)[128], float sl2, float nref, int lim,
+                                         float (&sum)[4], uint32_t tS, uint32_t bar_half,
+                                         uint32_t bar_full, uint32_t bar_turn_other, bool hand_over,
+                                         int lane) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t pk[32];
+#pragma unroll
+    for (int cc = 0; cc < 32; ++cc) {
+      const int c = 64 * h + 2 * cc;
+      float p0, p1;
+      if ((cc & 7) >= 8 - kPolyPairsPer8) {
+        f2_unpack(exp2_poly_x2(f2_pack(fmaf(__uint_as_float(r[c]), sl2, nref),
+                                       fmaf(__uint_as_float(r[c + 1]), sl2, nref))), p0, p1);
+      } else {
+        p0 = ex2_approx(fmaf(__uint_as_float(r[c]), sl2, nref));
+        p1 = ex2_approx(fmaf(__uint_as_float(r[c + 1]), sl2, nref));
+      }
+      if (MASKED) {
+        p0 = c < lim ? p0 : 0.f;
+        p1 = c + 1 < lim ? p1 : 0.f;
+      }
+      sum[(2 * cc) & 3] += p0;
+      sum[(2 * cc + 1) & 3] += p1;
+      pk[cc] = pack2<BF16>(p0, p1);
+    }
+    if (h == 1 && hand_over) {  // exponentials done: hand over the turn
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_turn_other);
+    }
+    tmem_st_32x32b_x32(tS + 32 * h, pk);
+    tmem_wait_st();
+    tc_fence_before_sync();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(h == 0 ? bar_half : bar_full);
+  }
+}
+
 template <int D, bool BF16, bool CAUSAL>
 __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, uint32_t tmem,
                                              uint32_t bars, volatile int* abort_flag) {
@@ -495,53 +542,20 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
         ++tcnt;
       }
 
-      // P = exp2(s * sl2 - ref), packed to 16 bits into the first 64 columns of
-      // S, in two halves of 64 keys, each handed to the MMA thread as soon as it
-      // is in tensor memory (one arrival per warp). On partial tiles the masked
-      // keys are zeroed after the exponential (their -inf scores times a zero
-      // scale, or -inf + inf when the row has no visible key yet, would give NaN).
-      const uint64_t sl2_2 = f2_pack(sl2, sl2);
-      const uint64_t nref2 = f2_pack(-ref, -ref);
-      uint64_t acc2[2] = {0ull, 0ull};
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int cc = 0; cc < 32; ++cc) {
-          const int c = 32 * h + cc;
-          const uint64_t x2 = f2_fma(f2_pack_bits(r[2 * c], r[2 * c + 1]), sl2_2, nref2);
-          float p0, p1;
-          if ((cc & 7) >= 8 - kPolyPairsPer8) {
-            f2_unpack(exp2_poly_x2(x2), p0, p1);
-          } else {
-            float x0, x1;
-            f2_unpack(x2, x0, x1);
-            p0 = ex2_approx(x0);
-            p1 = ex2_approx(x1);
-          }
-          if (partial) {
-            p0 = 2 * c < lim ? p0 : 0.f;
-            p1 = 2 * c + 1 < lim ? p1 : 0.f;
-          }
-          acc2[cc & 1] = f2_add(acc2[cc & 1], f2_pack(p0, p1));
-          pk[cc] = pack2<BF16>(p0, p1);
-        }
-        if (h == 1 && (t == 0 || j + 1 < x.n0)) {  // exponentials done: hand over the turn
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar_turn_other);
-        }
-        tmem_st_32x32b_x32(tS + 32 * h, pk);
-        tmem_wait_st();
-        tc_fence_before_sync();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(h == 0 ? bar_ph : bar_p);
+      const float nref = -ref;
+      const bool hand_over = (t == 0 || j + 1 < x.n0);
+      float sum[4] = {0.f, 0.f, 0.f, 0.f};
+      // the masked variant is a separate instantiation so full tiles carry no
+      // per-score compare/select. exp_tile holds warp-collective instructions
+      // (tcgen05.st, __syncwarp), so the choice must be the same for the whole
+      // warp: rows of one warp can differ (causal), and a lane whose keys are
+      // all visible is unaffected by the masked variant.
+      if (__any_sync(0xffffffffu, partial)) {
+        exp_tile<BF16, true>(r, sl2, nref, lim, sum, tS, bar_ph, bar_p, bar_turn_other, hand_over, lane);
+      } else {
+        exp_tile<BF16, false>(r, sl2, nref, lim, sum, tS, bar_ph, bar_p, bar_turn_other, hand_over, lane);
       }
-      {
-        float a0, a1, b0, b1;
-        f2_unpack(acc2[0], a0, a1);
-        f2_unpack(acc2[1], b0, b1);
-        l += (a0 + a1) + (b0 + b1);
-      }
+      l += (sum[0] + sum[1]) + (sum[2] + sum[3]);
     }
 
     // epilogue: O / l to 16-bit, 16-byte stores; LSE
