@@ -17,7 +17,7 @@
 //   warp  8     TMA producer: Q tiles, then K_0, V_0, K_1, V_1, ... into a ring
 //   warps 9, 10 MMA issuers (one thread each), warp 9 + t for query tile t:
 //               S_t = Q_t K^T and O_t += P_t V
-//   warp  11    idle
+//   warp  11    O store: staged O tiles to global memory by TMA
 // A work unit is (batch, query head, 256-row pair of query tiles). Tensor
 // memory holds S_0, S_1 (128 fp32 columns each, P aliased as packed 16-bit in
 // the first 64 columns) and O_0, O_1 (d columns each).
@@ -52,6 +52,7 @@ enum FaultBit : unsigned int {
   kFaultSoftmaxSFull = 1u << 5,
   kFaultSoftmaxOFull = 1u << 6,
   kFaultSoftmaxTurn = 1u << 7,
+  kFaultStore = 1u << 9,
   kFaultSelftest = 1u << 8,
 };
 
@@ -74,7 +75,8 @@ struct Cfg {
   static constexpr int kStages = (D == 128) ? 4 : 8;   // K/V ring depth (128 KB)
   static constexpr int kOffQ = 0;
   static constexpr int kOffKV = 2 * kTileBytes;
-  static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
+  static constexpr int kOffStg = kOffKV + kStages * kTileBytes;  // O staging for the TMA store
+  static constexpr int kOffBar = kOffStg + kTileBytes;
   static constexpr int kSmemBytes = kOffBar + 512 + 1024;  // barriers + 1 KB alignment slack
   // tensor-memory columns of S_t (P_t aliased) and O_t
   static __device__ __forceinline__ uint32_t col_s(int t) { return t ? 128u : 0u; }
@@ -94,6 +96,8 @@ enum Bar : int {
   kBarTurn = 14,    // [2] softmax 1-t -> softmax t: t may run its exponentials now
   kBarKvFull = 16,  // [kStages] TMA -> MMA
   kBarKvEmpty = 24, // [kStages] both MMA issuers -> TMA
+  kBarStgFull = 32, //     softmax t -> store warp: O tile t staged (one arrival per warp)
+  kBarStgFree = 34, // [2] store warp -> softmax t: staging buffer is t's to fill
 };
 
 // Exponentials of the softmax: kPolyPairsPer8 of every 8 score pairs take
@@ -434,9 +438,36 @@ __device__ __forceinline__ void exp_tile(const uint32_t (&r)[128], float sl2, fl
   }
 }
 
+// Warp 11 (one thread): writes each finished O tile from the shared staging
+// buffer to global memory with a TMA store (rows past Lq are clipped by the
+// tensor map), then hands the buffer to the other query tile. Order per unit:
+// tile 0, then tile 1, the same order the softmax warpgroups fill it in.
+template <int D, bool BF16, bool CAUSAL>
+__device__ __forceinline__ void store_role(const CUtensorMap* tm_o, const FwdParams& p, uint32_t sStg,
+                                           uint32_t bars, volatile int* abort_flag) {
+  using C = Cfg<D>;
+  int scnt = 0;
+  bool ok = true;
+  for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+    const Unit x = decode_unit<CAUSAL>(p, u);
+    for (int t = 0; t < 2 && ok; ++t) {
+      ok = mbar_wait(bars + 8 * kBarStgFull, scnt & 1, abort_flag, kFaultStore, p.timeout_ns);
+      if (!ok) break;
+      ++scnt;
+#pragma unroll
+      for (int c = 0; c < C::kChunks; ++c)
+        tma_store_4d(tm_o, sStg + c * C::kChunkBytes, c * 64, x.hq, x.r0 + t * kTileRows, x.b);
+      bulk_commit_group();
+      bulk_wait_group_read0();
+      mbar_arrive(bars + 8 * (kBarStgFree + (1 - t)));
+    }
+  }
+  bulk_wait_group0();  // every store complete before the CTA exits
+}
+
 template <int D, bool BF16, bool CAUSAL>
 __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, uint32_t tmem,
-                                             uint32_t bars, volatile int* abort_flag) {
+                                             uint32_t bars, uint32_t sstg, volatile int* abort_flag) {
   using C = Cfg<D>;
   const int warp = threadIdx.x / 32;
   const int r_in = threadIdx.x % kTileRows;                      // row in tile = TMEM lane
@@ -448,6 +479,9 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
   const uint32_t bar_ph = bars + 8 * (kBarPHalf + t);
   const uint32_t bar_turn_mine = bars + 8 * (kBarTurn + t);
   const uint32_t bar_turn_other = bars + 8 * (kBarTurn + (1 - t));
+  const uint32_t bar_stg_full = bars + 8 * kBarStgFull;
+  const uint32_t bar_stg_free = bars + 8 * (kBarStgFree + t);
+  const uint32_t stg = sstg;
   int tcnt = 0;
   const int lane = threadIdx.x % 32;
   const uint32_t bar_o = bars + 8 * (kBarOFull + t);
@@ -558,15 +592,18 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
       l += (sum[0] + sum[1]) + (sum[2] + sum[3]);
     }
 
-    // epilogue: O / l to 16-bit, 16-byte stores; LSE
-    bool ok = mbar_wait(bar_o, ocnt & 1, abort_flag, kFaultSoftmaxOFull, p.timeout_ns);
+    // epilogue: O / l to 16 bits into the shared staging tile (128-byte
+    // swizzle, the layout of the TMA box), handed to the store warp; LSE.
+    // The staging buffer alternates between the two query tiles: tile t fills
+    // it once the store warp has read out the other tile's previous O.
+    bool ok = mbar_wait(bar_o, ocnt & 1, abort_flag, kFaultSoftmaxOFull, p.timeout_ns) &&
+              mbar_wait(bar_stg_free, (ocnt & 1) ^ (t == 0 ? 1 : 0), abort_flag, kFaultStore,
+                        p.timeout_ns);
     if (!__all_sync(0xffffffffu, ok)) return;
     ++ocnt;
     tc_fence_after_sync();
     const float inv_l = 1.f / l;
     const bool in_range = row < p.Lq;
-    uint16_t* orow = static_cast<uint16_t*>(p.o) +
-                     ((static_cast<size_t>(x.b) * p.Lq + row) * p.Hq + x.hq) * D;
 #pragma unroll 1
     for (int c = 0; c < D / 32; ++c) {
       uint32_t ov[32];
@@ -576,12 +613,20 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
 #pragma unroll
       for (int e = 0; e < 16; ++e)
         pk[e] = pack2<BF16>(__uint_as_float(ov[2 * e]) * inv_l, __uint_as_float(ov[2 * e + 1]) * inv_l);
-      if (in_range) {
-        uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+      // 32 columns = 4 units of 16 bytes in the 64-column box (c / 2); unit u of
+      // row r sits at r * 128 + ((u ^ (r % 8)) * 16)
+      const uint32_t box = stg + (c >> 1) * C::kChunkBytes + r_in * 128;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t unit = static_cast<uint32_t>(((c & 1) * 4 + e) ^ (r_in & 7));
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(box + unit * 16),
+                     "r"(pk[4 * e]), "r"(pk[4 * e + 1]), "r"(pk[4 * e + 2]), "r"(pk[4 * e + 3])
+                     : "memory");
       }
     }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar_stg_full);
     if (p.lse != nullptr && in_range)
       p.lse[(static_cast<size_t>(x.b) * p.Hq + x.hq) * p.Lq + row] = (ref + log2f(l)) * kLn2;
   }
@@ -591,7 +636,8 @@ template <int D, bool BF16, bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
-                          const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+                          const __grid_constant__ CUtensorMap tm_v,
+                          const __grid_constant__ CUtensorMap tm_o, const FwdParams p) {
   using C = Cfg<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -599,9 +645,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sbase = smem_u32(smem);
   const uint32_t sQ = sbase + C::kOffQ;
   const uint32_t sKV = sbase + C::kOffKV;
+  const uint32_t sStg = sbase + C::kOffStg;
   const uint32_t bars = sbase + C::kOffBar;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffBar + 256);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffBar + 260);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffBar + 448);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffBar + 452);
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
 
@@ -616,6 +663,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bars + 8 * (kBarOFull + t), 1);
     }
     mbar_init(bars + 8 * kBarDrain, 1);
+    mbar_init(bars + 8 * kBarStgFull, kTileRows / 32);
+    mbar_init(bars + 8 * (kBarStgFree + 0), 1);
+    mbar_init(bars + 8 * (kBarStgFree + 1), 1);
     mbar_init(bars + 8 * (kBarDrain + 1), 1);
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(bars + 8 * (kBarKvFull + s), 1);
@@ -628,6 +678,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_o);
   }
   if (warp == 9) {
     tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
@@ -640,13 +691,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < 8) {
     regs_increase<kRegsSoftmax>();
-    softmax_role<D, BF16, CAUSAL>(warp / 4, p, tmem, bars, abort_flag);
+    softmax_role<D, BF16, CAUSAL>(warp / 4, p, tmem, bars, sStg, abort_flag);
   } else {
     regs_decrease<kRegsProducer>();
     if (warp == 8) {
       if (lane == 0) load_role<D, BF16, CAUSAL>(&tm_q, &tm_k, &tm_v, p, sQ, sKV, bars, abort_flag);
     } else if (warp == 9 || warp == 10) {
       if (lane == 0) mma_role<D, BF16, CAUSAL>(warp - 9, p, tmem, sQ, sKV, bars, abort_flag);
+    } else {
+      if (lane == 0) store_role<D, BF16, CAUSAL>(&tm_o, p, sStg, bars, abort_flag);
     }
   }
   __syncwarp();
@@ -848,10 +901,11 @@ template <int D, bool BF16, bool CAUSAL>
 int launch_fwd(const FwdParams& p, const void* q, const void* k, const void* v, int grid,
                cudaStream_t stream) {
   using C = Cfg<D>;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   if (!encode_bl_hd(&tq, q, p.B, p.Lq, p.Hq, D, BF16) ||
       !encode_bl_hd(&tk, k, p.B, p.Lk, p.Hkv, D, BF16) ||
-      !encode_bl_hd(&tv, v, p.B, p.Lk, p.Hkv, D, BF16))
+      !encode_bl_hd(&tv, v, p.B, p.Lk, p.Hkv, D, BF16) ||
+      !encode_bl_hd(&to, p.o, p.B, p.Lq, p.Hq, D, BF16))
     return ATTN_ERR_CUDA;
   auto kern = attn_fwd_sm100_kernel<D, BF16, CAUSAL>;
   static std::once_flag attr_flags[kMaxDevices];
@@ -874,7 +928,7 @@ int launch_fwd(const FwdParams& p, const void* q, const void* k, const void* v, 
   });
   if (attr_status[dev] != ATTN_OK) return attr_status[dev];
   (void)cudaGetLastError();  // launch errors below are this launch's own
-  kern<<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
+  kern<<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, to, p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
