@@ -688,6 +688,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
+  // Programmatic dependent launch: everything above (barriers, tensor memory,
+  // descriptor prefetch) may overlap the previous kernel on this stream; no
+  // global memory is touched before that kernel has completed and its writes
+  // are visible. The next kernel may then start its own set-up on SMs this
+  // grid leaves idle.
+  griddep_wait();
+  griddep_launch_dependents();
 
   if (warp < 8) {
     regs_increase<kRegsSoftmax>();
@@ -928,7 +935,17 @@ int launch_fwd(const FwdParams& p, const void* q, const void* k, const void* v, 
   });
   if (attr_status[dev] != ATTN_OK) return attr_status[dev];
   (void)cudaGetLastError();  // launch errors below are this launch's own
-  kern<<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, to, p);
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, to, p) != cudaSuccess) return ATTN_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

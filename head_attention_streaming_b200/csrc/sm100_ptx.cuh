@@ -107,6 +107,20 @@ __device__ __forceinline__ uint64_t l2_policy_evict_last() {
   return p;
 }
 
+// --------------------------------------------------- dependent launches
+
+// Blocks until the grids this one depends on (programmatic stream
+// serialization) have completed and their memory operations are visible.
+// Returns at once when there is no such grid.
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+// Lets the next grid on the stream start launching (its CTAs still wait for
+// free SMs and for their own griddepcontrol.wait).
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // -------------------------------------------------------------------- TMEM
 
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
