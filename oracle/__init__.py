@@ -1,4 +1,5 @@
-"""FP64 CPU oracle for the attention forward (test infrastructure only).
+"""FP64 CPU oracle for the attention forward and its Q/K prologue (test
+infrastructure only).
 
 Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
 and reference legs may import this package; the product path never does.
@@ -6,6 +7,9 @@ and reference legs may import this package; the product path never does.
 
 from .attention import (MASK_CAUSAL, MASK_CHUNK, MASK_NONE, attention_fwd, flops,
                         kv_head, visible_limit)
+from .prologue import (NORM_HEAD, NORM_INNER, NORM_NONE, ROPE_INTERLEAVED, ROPE_NONE,
+                          ROPE_SPLIT, qk_prologue, rms_norm, rope)
 
 __all__ = ["MASK_NONE", "MASK_CAUSAL", "MASK_CHUNK", "attention_fwd", "flops",
-           "kv_head", "visible_limit"]
+           "kv_head", "visible_limit", "NORM_NONE", "NORM_HEAD", "NORM_INNER", "ROPE_NONE",
+           "ROPE_INTERLEAVED", "ROPE_SPLIT", "qk_prologue", "rms_norm", "rope"]
