@@ -25,6 +25,12 @@ Also reported on the same JSON line:
 
 --impl reference times the FP64 CPU oracle (the only reference this build has)
 on the same workload, metric and unit, each step a bounded sample of it.
+
+--op prologue times the Q/K prologue instead (attn_qk_prologue: head-scope
+RMSNorm, eps 1e-6, then split-half RoPE, on Q and the new K chunk of the
+1785-token DiT workload, BF16 [1, 1785, 40, 128] each): an HBM-bound pass,
+reported in GB/s of algorithmic traffic (Q and K read once and written once,
+plus the weights and angle tables) against the measured HBM copy bandwidth.
 """
 
 from __future__ import annotations
@@ -46,6 +52,7 @@ sys.path.insert(0, ROOT)
 METRIC = "attention fwd TFLOPS on 1 B200 and % of dense BF16 tensor-core peak"
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "attn_fwd_video_20480x56x128.md")
+PROLOGUE_SUMMARY = os.path.join(ROOT, "profiles", "qk_prologue_dit_1785x40x128.md")
 KERNEL_SOURCES = [os.path.join(ROOT, "head_attention_streaming_b200", "csrc", f)
                   for f in ("attn_fwd_sm100.cu", "sm100_ptx.cuh", "tmem_ldst.inc")]
 
@@ -64,6 +71,7 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="minimum CPU time spent timing the oracle sample")
+    ap.add_argument("--op", default="attention", choices=["attention", "prologue"])
     return ap.parse_args()
 
 
@@ -77,25 +85,25 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(sources=None) -> str:
     h = hashlib.sha256()
-    for p in KERNEL_SOURCES:
+    for p in (sources or KERNEL_SOURCES):
         with open(p, "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic():
+def profiled_traffic(summary=None, sources=None):
     """DRAM bytes per launch from the committed ncu summary, if it matches this kernel."""
     try:
-        text = open(PROFILE_SUMMARY).read()
+        text = open(summary or PROFILE_SUMMARY).read()
     except OSError:
         return None, "no ncu summary"
     m_bytes = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
     m_hash = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", text)
     if not m_bytes or not m_hash:
         return None, "summary lacks traffic"
-    if m_hash.group(1) != kernel_source_hash():
+    if m_hash.group(1) != kernel_source_hash(sources):
         return None, "kernel changed since the ncu capture"
     return float(m_bytes.group(1)), "ncu"
 
@@ -257,8 +265,158 @@ def run_reference(args):
     return 0
 
 
+PROLOGUE_SOURCES = [os.path.join(ROOT, "head_attention_streaming_b200", "csrc", "qk_prologue.cu")]
+
+
+def run_prologue(args):
+    """Time attn_qk_prologue on Q and K of the 1785-token DiT workload (rank 0 of
+    each replica; weak scaling like the attention bench)."""
+    import torch
+    import torch.distributed as dist
+
+    import head_attention_streaming_b200 as hasb
+    from head_attention_streaming_b200 import inputs
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    B, L, H, d, pos0, eps = 1, 1785, 40, 128, 5355, 1e-6
+    g = torch.Generator().manual_seed(31 + 7919 * rank)
+    q_cpu = torch.randn(B, L, H, d, generator=g).to(torch.bfloat16)
+    k_cpu = torch.randn(B, L, H, d, generator=g).to(torch.bfloat16)
+    gq_cpu = 1.0 + 0.1 * torch.randn(d, generator=g)
+    gk_cpu = 1.0 + 0.1 * torch.randn(d, generator=g)
+    ang_cpu = inputs.rope_angle_table(L, d, hasb.ROPE_SPLIT, pos0)
+    q, k = q_cpu.cuda(), k_cpu.cuda()
+    gq, gk, ang = gq_cpu.cuda(), gk_cpu.cuda(), ang_cpu.cuda()
+    oq, ok = torch.empty_like(q), torch.empty_like(k)
+    stream = torch.cuda.current_stream()
+    tensor_bytes = 2 * q.numel() * 2                     # Q and K, 16-bit
+    algo_bytes = 2 * tensor_bytes + 2 * d * 4 + 2 * ang.numel() * 4  # read + write, weights, angles
+
+    def step():
+        hasb.qk_prologue(q, k, norm_scope=hasb.NORM_HEAD, eps=eps, gamma_q=gq, gamma_k=gk,
+                         rope_style=hasb.ROPE_SPLIT, angles_q=ang, angles_k=ang, out_q=oq, out_k=ok)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    time.sleep(0.3)
+    flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    for a, b in ev:
+        flush_buf.add_(1)  # inputs (37 MB) fit in L2: evict them between steps
+        a.record(stream)
+        step()
+        b.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    clock_info = clocks.stop()
+    launch_ms = [a.elapsed_time(b) for a, b in ev]
+    ms_step = statistics.mean(launch_ms)
+    if world > 1:
+        t = torch.tensor([ms_step], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step = float(t.item())
+    value = world * algo_bytes / (ms_step * 1e-3) / 1e9
+
+    # end to end: pinned host Q, K in, prologue, Q, K out, every step
+    qh, kh = q_cpu.pin_memory(), k_cpu.pin_memory()
+    oqh, okh = torch.empty_like(qh).pin_memory(), torch.empty_like(kh).pin_memory()
+    e2e_steps = max(1, args.e2e_steps)
+
+    def e2e_step():
+        q.copy_(qh, non_blocking=True)
+        k.copy_(kh, non_blocking=True)
+        step()
+        oqh.copy_(oq, non_blocking=True)
+        okh.copy_(ok, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e_ms = e0.elapsed_time(e1) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e_ms = float(t.item())
+    e2e = {"value": world * algo_bytes / (e_ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": e_ms,
+           "h2d_bytes_per_step": tensor_bytes, "d2h_bytes_per_step": tensor_bytes,
+           "path": "pinned host Q, K -> device, attn_qk_prologue, Q, K -> host, one stream"}
+
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    achieved = algo_bytes / (statistics.mean(launch_ms) * 1e-3) / 1e9
+    traffic, traffic_src = profiled_traffic(PROLOGUE_SUMMARY, PROLOGUE_SOURCES)
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "traffic": traffic, "traffic_source": traffic_src,
+                "peak_source": f"hbm_gbs of {peak_src}", "kernel": "qk_prologue_kernel",
+                "algorithmic_bytes_per_launch": algo_bytes, "launch_ms_mean": statistics.mean(launch_ms),
+                "launch_ms_min": min(launch_ms), "launch_ms_max": max(launch_ms)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import numpy as np
+        import oracle
+        ntok = 64  # tokens per oracle call; repeated for about --cpu-seconds
+        xs = q_cpu[:, :ntok].double().numpy()
+        angs = ang_cpu[:ntok].double().numpy()
+        gqn = gq_cpu.double().numpy()
+        reps, t0 = 0, time.perf_counter()
+        while True:
+            oracle.qk_prologue(xs, gqn, eps, oracle.NORM_HEAD, angs, oracle.ROPE_SPLIT)
+            reps += 1
+            el = time.perf_counter() - t0
+            if el >= args.cpu_seconds / 4 or reps >= 2000:
+                break
+        cpu_bytes = reps * ntok * H * d * 2 * 2
+        cpu = {"value": cpu_bytes / el / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+               "sample": f"{ntok} tokens x {H} heads of Q x {reps} repetitions, numpy float64, "
+                         "bytes counted as the 16-bit read + write the kernel does"}
+
+    if rank == 0:
+        line = {
+            "metric": "Q/K prologue (head RMSNorm + split RoPE) GB/s on 1 B200 and fraction of HBM copy bandwidth",
+            "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic: seeded N(0,1) Q and K, gamma = 1 + 0.1 N(0,1), angles of positions 5355..7139",
+            "config": {"workload": "dit_prologue_1785x40x128", "B": B, "L": L, "Hq": H, "Hkv": H, "d": d,
+                       "norm": "head", "eps": eps, "rope": "split", "pos0": pos0,
+                       "l2": "inputs 37 MB vs 126 MB L2: L2 flushed between steps",
+                       "parallelism": "single GPU" if world == 1 else f"{world} independent replicas"},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps,
+            "clocks": clock_info, "device_fault_bits": hasb.device_fault(clear=True),
+        }
+        print(json.dumps(line))
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     args = parse_args()
+    if args.op == "prologue":
+        return run_prologue(args)
     if args.impl == "reference":
         return run_reference(args)
 

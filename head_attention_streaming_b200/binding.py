@@ -27,6 +27,14 @@ MASK_NONE = 0
 MASK_CAUSAL = 1
 MASK_CHUNK = 2
 
+NORM_NONE = 0
+NORM_HEAD = 1
+NORM_INNER = 2
+
+ROPE_NONE = 0
+ROPE_INTERLEAVED = 1
+ROPE_SPLIT = 2
+
 DTYPE_CODES = {torch.bfloat16: 0, torch.float16: 1}
 
 # name -> (restype, argtypes) of every exported function
@@ -35,6 +43,8 @@ _SIGNATURES = {
                  [ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
     "attn_fwd_host": (ctypes.c_int, [ctypes.c_void_p] * 10 + [ctypes.c_int] * 6 +
                       [ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
+    "attn_qk_prologue": (ctypes.c_int, [ctypes.c_void_p] * 8 + [ctypes.c_int] * 7 +
+                         [ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
     "attn_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "attn_device_fault": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint), ctypes.c_int]),
     "attn_set_wait_timeout_ns": (ctypes.c_int, [ctypes.c_ulonglong]),
@@ -127,6 +137,61 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, scale: float 
     if st != ATTN_OK:
         raise AttnError(st, "attn_fwd")
     return out, lse
+
+
+def _check_f32(name, t, numel, device):
+    if t is None:
+        return
+    if (not t.is_cuda or t.dtype != torch.float32 or not t.is_contiguous() or t.numel() != numel
+            or t.device != device):
+        raise ValueError(f"{name} must be a contiguous float32 CUDA tensor of {numel} elements")
+
+
+def qk_prologue(q: torch.Tensor, k: torch.Tensor | None = None, *, norm_scope: int = NORM_NONE,
+                eps: float = 1e-6, gamma_q: torch.Tensor | None = None,
+                gamma_k: torch.Tensor | None = None, rope_style: int = ROPE_NONE,
+                angles_q: torch.Tensor | None = None, angles_k: torch.Tensor | None = None,
+                out_q: torch.Tensor | None = None, out_k: torch.Tensor | None = None,
+                stream=None):
+    """Q/K RMSNorm then RoPE through ``attn_qk_prologue`` of the C ABI.
+
+    q: [B, Lq, Hq, d], k: [B, Lk, Hkv, d] or None (CUDA, contiguous, bf16/fp16).
+    gamma_*: float32 [d] (head scope) or [H*d] (inner scope), None = ones.
+    angles_*: float32 [L, d] (the expanded rope_freqs table), required iff
+    rope_style != ROPE_NONE. ``out_q`` / ``out_k`` may be the inputs (in place);
+    by default new tensors. Returns ``(q_out, k_out)``.
+    """
+    tensors = [("q", q)] + ([("k", k)] if k is not None else [])
+    for name, t in tensors:
+        if not t.is_cuda or not t.is_contiguous() or t.dim() != 4 or t.dtype not in DTYPE_CODES:
+            raise ValueError(f"{name} must be a contiguous 4-D bf16/fp16 CUDA tensor")
+    B, Lq, Hq, d = q.shape
+    Lk, Hkv = 0, 0
+    if k is not None:
+        if k.dtype != q.dtype or k.shape[0] != B or k.shape[3] != d:
+            raise ValueError("k must share q's dtype, batch and head_dim")
+        Lk, Hkv = k.shape[1], k.shape[2]
+    wq = d if norm_scope == NORM_HEAD else Hq * d
+    wk = d if norm_scope == NORM_HEAD else Hkv * d
+    _check_f32("gamma_q", gamma_q, wq, q.device)
+    _check_f32("gamma_k", gamma_k, wk, q.device)
+    _check_f32("angles_q", angles_q, Lq * d, q.device)
+    _check_f32("angles_k", angles_k, Lk * d, q.device)
+    if out_q is None:
+        out_q = torch.empty_like(q)
+    if k is not None and out_k is None:
+        out_k = torch.empty_like(k)
+    for name, o, ref in (("out_q", out_q, q), ("out_k", out_k, k)):
+        if ref is not None and (o.shape != ref.shape or o.dtype != ref.dtype or not o.is_cuda
+                                or not o.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous CUDA tensor shaped and typed like its input")
+    st = lib().attn_qk_prologue(_ptr(q), _ptr(out_q), _ptr(k), _ptr(out_k if k is not None else None),
+                                _ptr(gamma_q), _ptr(gamma_k), _ptr(angles_q), _ptr(angles_k),
+                                B, Lq, Lk, Hq, Hkv, d, int(norm_scope), float(eps), int(rope_style),
+                                DTYPE_CODES[q.dtype], _stream_handle(stream, q.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_qk_prologue")
+    return out_q, (out_k if k is not None else None)
 
 
 def attn_fwd_host(q_host, k_host, v_host, o_host, lse_host, q_dev, k_dev, v_dev, o_dev, lse_dev, *,

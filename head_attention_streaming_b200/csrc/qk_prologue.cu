@@ -1,0 +1,312 @@
+// Q/K prologue for B200 (sm_100a): RMS normalisation, then rotary position
+// embedding, of Q and of the new K chunk, in one launch.
+//
+// What is computed: the flashdreams.accelerated developer guide, "Multi Head
+// Attention Definition": RMSNorm_gamma(z) = gamma * z / sqrt(mean(z^2) + eps)
+// over each head (head scope, m = d) or over all heads of a token (inner
+// scope, m = H d); then RoPE rotates feature pair r of the token at sequence
+// index p by the angle rope_freqs[p, a_r], pairs (2r, 2r + 1) (interleaved) or
+// (r, r + d/2) (split-half). Normalisation comes first, as on that page. V is
+// neither normalised nor rotated.
+//
+// The work is an elementwise pass bound by HBM bandwidth: each element is read
+// once and written once. One 128-thread block per token. The token's H d
+// features are cut into 16-feature items, d / 16 per head; thread t handles
+// items t, t + 128, ... An item is two 16-byte vectors of one head: features
+// [o, o + 8) and [o + d/2, o + d/2 + 8) for split-half RoPE (so both features
+// of every pair sit in one thread), [o, o + 16) otherwise. The d / 16 items of
+// a head sit on adjacent lanes of one warp, so the head's sum of squares is a
+// butterfly over those lanes. The rotation angles depend on the token's
+// position and the feature only, not on the head: the block computes the d / 2
+// cosines and sines once per token into shared memory and every head reuses
+// them. Arithmetic in fp32; one rounding to the 16-bit type at the end.
+
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "attn.h"
+
+namespace hasb_pro {
+
+constexpr int kWarps = 4;
+constexpr int kThreads = 32 * kWarps;
+
+struct ProTensor {
+  const void* x;
+  void* y;
+  const float* gamma;   // [m] or nullptr (all ones)
+  const float* angles;  // [L, d] or nullptr (no RoPE)
+  int L, H;
+};
+
+struct ProParams {
+  ProTensor t[2];
+  int tokens0;  // B * L of tensor 0; blocks past it belong to tensor 1
+  int d;
+  float eps;  // normalisation scope and RoPE style are template arguments of the kernel
+};
+
+template <bool BF16>
+__device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    if (BF16) {
+      f[2 * i] = __uint_as_float(w[i] << 16);
+      f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    } else {
+      const __half2 h = *reinterpret_cast<const __half2*>(&w[i]);
+      const float2 t = __half22float2(h);
+      f[2 * i] = t.x;
+      f[2 * i + 1] = t.y;
+    }
+  }
+}
+
+template <bool BF16>
+__device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint32_t r;
+    if (BF16)
+      asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(f[2 * i + 1]), "f"(f[2 * i]));
+    else
+      asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(f[2 * i + 1]), "f"(f[2 * i]));
+    w[i] = r;
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Feature index of element e (0..15) of item-offset o within its head.
+__device__ __forceinline__ int item_feature(int o, int e, int d, bool split) {
+  return split ? (e < 8 ? o + e : o + d / 2 + e - 8) : o + e;
+}
+
+template <bool BF16, int SCOPE, int STYLE>
+__global__ void __launch_bounds__(kThreads) qk_prologue_kernel(const ProParams p) {
+  __shared__ float red[kWarps];
+  __shared__ float cs_s[128], sn_s[128];  // cos / sin of the token's d/2 pair angles
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const int which = blockIdx.x < p.tokens0 ? 0 : 1;
+  const ProTensor T = which ? p.t[1] : p.t[0];
+  const int token = which ? blockIdx.x - p.tokens0 : blockIdx.x;  // b * L + l
+  const int pos = token % T.L;                                     // sequence index l
+  const int d = p.d;
+  constexpr bool split = STYLE == ATTN_ROPE_SPLIT;
+  const int per_head = d / 16;                  // items per head
+  const int sh = __ffs(per_head) - 1;           // log2(per_head)
+  const int items = T.H * per_head;             // items of the token
+  const size_t base = static_cast<size_t>(token) * T.H * d;
+  const uint16_t* x = static_cast<const uint16_t*>(T.x) + base;
+  uint16_t* y = static_cast<uint16_t*>(T.y) + base;
+  // intra-head item index is the same for every item this thread handles
+  // (128 is a multiple of d / 16)
+  const int io = threadIdx.x % per_head;
+  const int o = split ? 8 * io : 16 * io;       // first feature of the item in its head
+
+  if constexpr (STYLE != ATTN_ROPE_NONE) {
+    // pair r: first feature a_r = 2r (interleaved) or r (split-half)
+    if (threadIdx.x < d / 2) {
+      const int a = split ? threadIdx.x : 2 * threadIdx.x;
+      sincosf(T.angles[static_cast<size_t>(pos) * d + a], &sn_s[threadIdx.x], &cs_s[threadIdx.x]);
+    }
+  }
+  float ghead[16];
+  if (SCOPE == ATTN_NORM_HEAD) {
+#pragma unroll
+    for (int e = 0; e < 16; ++e)
+      ghead[e] = T.gamma != nullptr ? T.gamma[item_feature(o, e, d, split)] : 1.f;
+  }
+
+  auto load_item = [&](int it, float (&f)[16]) {
+    const int h = it >> sh;
+    const uint16_t* src = x + h * d + o;
+    unpack8<BF16>(*reinterpret_cast<const uint4*>(src), *reinterpret_cast<float(*)[8]>(&f[0]));
+    unpack8<BF16>(*reinterpret_cast<const uint4*>(src + (split ? d / 2 : 8)),
+                  *reinterpret_cast<float(*)[8]>(&f[8]));
+  };
+
+  // inner scope: one sum of squares over the whole token first
+  float inv_token = 1.f;
+  if (SCOPE == ATTN_NORM_INNER) {
+    float ss = 0.f;
+    for (int it = threadIdx.x; it < items; it += kThreads) {
+      float f[16];
+      load_item(it, f);
+#pragma unroll
+      for (int e = 0; e < 16; ++e) ss = fmaf(f[e], f[e], ss);
+    }
+#pragma unroll
+    for (int s = 16; s > 0; s >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, s);
+    if (lane == 0) red[warp] = ss;
+  }
+  __syncthreads();  // cos / sin table and partial sums visible
+  if (SCOPE == ATTN_NORM_INNER) {
+    const float tot = (red[0] + red[1]) + (red[2] + red[3]);
+    inv_token = rsqrtf(tot / static_cast<float>(T.H * d) + p.eps);
+  }
+  float c8[8], s8[8];
+  if (STYLE != ATTN_ROPE_NONE) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      // split: element e and e + 8 form pair o/1 + e; interleaved: elements
+      // 2m, 2m + 1 form pair o/2 + m
+      const int r = split ? o + e : o / 2 + e;
+      c8[e] = cs_s[r];
+      s8[e] = sn_s[r];
+    }
+  }
+
+  const int rounds = (items + kThreads - 1) / kThreads;
+  for (int k = 0; k < rounds; ++k) {
+    const int it = threadIdx.x + k * kThreads;
+    const bool live = it < items;
+    float2 f[8];  // f[m] = (element 2m, element 2m + 1) of the item
+    if (live) {
+      load_item(it, *reinterpret_cast<float(*)[16]>(f));
+    } else {
+#pragma unroll
+      for (int m = 0; m < 8; ++m) f[m] = make_float2(0.f, 0.f);
+    }
+    if (SCOPE == ATTN_NORM_HEAD) {
+      float2 ss2 = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int m = 0; m < 8; ++m) ss2 = __ffma2_rn(f[m], f[m], ss2);
+      float ss = ss2.x + ss2.y;
+      for (int q = 1; q < per_head; q <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, q);
+      const float inv = rsqrtf(ss / static_cast<float>(d) + p.eps);
+      const float2 inv2 = make_float2(inv, inv);
+#pragma unroll
+      for (int m = 0; m < 8; ++m)
+        f[m] = __fmul2_rn(make_float2(ghead[2 * m], ghead[2 * m + 1]), __fmul2_rn(f[m], inv2));
+    } else if (SCOPE == ATTN_NORM_INNER) {
+      const float* g = (T.gamma != nullptr && live) ? T.gamma + (it >> sh) * d : nullptr;
+      const float2 inv2 = make_float2(inv_token, inv_token);
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        const float2 gg = g != nullptr ? make_float2(g[item_feature(o, 2 * m, d, split)],
+                                                     g[item_feature(o, 2 * m + 1, d, split)])
+                                       : make_float2(1.f, 1.f);
+        f[m] = __fmul2_rn(gg, __fmul2_rn(f[m], inv2));
+      }
+    }
+    if constexpr (split) {
+      // element e (< 8) pairs with element e + 8: f[m] holds elements 2m, 2m+1
+      // of the first vector, f[m + 4] the same two of the second
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const float2 a = f[m], b = f[m + 4];
+        const float2 c = make_float2(c8[2 * m], c8[2 * m + 1]);
+        const float2 sn = make_float2(s8[2 * m], s8[2 * m + 1]);
+        f[m] = __ffma2_rn(a, c, __fmul2_rn(make_float2(-b.x, -b.y), sn));
+        f[m + 4] = __ffma2_rn(a, sn, __fmul2_rn(b, c));
+      }
+    } else if (STYLE == ATTN_ROPE_INTERLEAVED) {
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        const float a = f[m].x, b = f[m].y;
+        f[m] = make_float2(a * c8[m] - b * s8[m], a * s8[m] + b * c8[m]);
+      }
+    }
+    if (live) {
+      uint16_t* dst = y + (it >> sh) * d + o;
+      *reinterpret_cast<uint4*>(dst) = pack8<BF16>(*reinterpret_cast<const float(*)[8]>(&f[0]));
+      *reinterpret_cast<uint4*>(dst + (split ? d / 2 : 8)) =
+          pack8<BF16>(*reinterpret_cast<const float(*)[8]>(&f[4]));
+    }
+  }
+}
+
+}  // namespace hasb_pro
+
+using namespace hasb_pro;
+
+namespace {
+
+template <bool BF16, int SCOPE>
+void launch_style(const ProParams& p, int style, unsigned grid, cudaStream_t s) {
+  if (style == ATTN_ROPE_NONE)
+    qk_prologue_kernel<BF16, SCOPE, ATTN_ROPE_NONE><<<grid, kThreads, 0, s>>>(p);
+  else if (style == ATTN_ROPE_INTERLEAVED)
+    qk_prologue_kernel<BF16, SCOPE, ATTN_ROPE_INTERLEAVED><<<grid, kThreads, 0, s>>>(p);
+  else
+    qk_prologue_kernel<BF16, SCOPE, ATTN_ROPE_SPLIT><<<grid, kThreads, 0, s>>>(p);
+}
+
+template <bool BF16>
+void launch_scope(const ProParams& p, int scope, int style, unsigned grid, cudaStream_t s) {
+  if (scope == ATTN_NORM_NONE)
+    launch_style<BF16, ATTN_NORM_NONE>(p, style, grid, s);
+  else if (scope == ATTN_NORM_HEAD)
+    launch_style<BF16, ATTN_NORM_HEAD>(p, style, grid, s);
+  else
+    launch_style<BF16, ATTN_NORM_INNER>(p, style, grid, s);
+}
+
+void launch_prologue(const ProParams& p, bool bf16, int scope, int style, unsigned grid,
+                     cudaStream_t s) {
+  if (bf16)
+    launch_scope<true>(p, scope, style, grid, s);
+  else
+    launch_scope<false>(p, scope, style, grid, s);
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool overlap(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+}  // namespace
+
+extern "C" int attn_qk_prologue(const void* q, void* q_out, const void* k, void* k_out,
+                                const float* gamma_q, const float* gamma_k, const float* angles_q,
+                                const float* angles_k, int B, int Lq, int Lk, int Hq, int Hkv, int d,
+                                int norm_scope, float eps, int rope_style, int dtype, void* stream) {
+  // ---- arguments (all checked before any CUDA call)
+  if (q == nullptr || q_out == nullptr) return ATTN_ERR_INVALID_ARG;
+  if ((k == nullptr) != (k_out == nullptr)) return ATTN_ERR_INVALID_ARG;
+  if (dtype != ATTN_DTYPE_BF16 && dtype != ATTN_DTYPE_FP16) return ATTN_ERR_INVALID_ARG;
+  if (norm_scope < ATTN_NORM_NONE || norm_scope > ATTN_NORM_INNER) return ATTN_ERR_INVALID_ARG;
+  if (rope_style < ATTN_ROPE_NONE || rope_style > ATTN_ROPE_SPLIT) return ATTN_ERR_INVALID_ARG;
+  if (!(eps >= 0.f) || !std::isfinite(eps)) return ATTN_ERR_INVALID_ARG;
+  if (B < 1 || Lq < 1 || Hq < 1) return ATTN_ERR_INVALID_ARG;
+  if (k != nullptr && (Lk < 1 || Hkv < 1)) return ATTN_ERR_INVALID_ARG;
+  if (d < 16 || d > 256 || (d & (d - 1)) != 0) return ATTN_ERR_UNSUPPORTED;
+  if ((rope_style != ATTN_ROPE_NONE) != (angles_q != nullptr)) return ATTN_ERR_INVALID_ARG;
+  if (k != nullptr && (rope_style != ATTN_ROPE_NONE) != (angles_k != nullptr)) return ATTN_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(q_out, 16) || (k && (!aligned(k, 16) || !aligned(k_out, 16))))
+    return ATTN_ERR_INVALID_ARG;
+  for (const float* f : {gamma_q, gamma_k, angles_q, angles_k})
+    if (f != nullptr && !aligned(f, 4)) return ATTN_ERR_INVALID_ARG;
+  const long long nq = 1LL * B * Lq * Hq * d, nk = k ? 1LL * B * Lk * Hkv * d : 0;
+  const long long tokens = 1LL * B * Lq + (k ? 1LL * B * Lk : 0);
+  if (tokens > 0x7fffffffLL || 1LL * Hq * d > (1 << 20) || 1LL * Hkv * d > (1 << 20))
+    return ATTN_ERR_INVALID_ARG;
+  // outputs may be their own input (in place) but may not overlap anything else
+  if (q_out != q && overlap(q_out, nq * 2, q, nq * 2)) return ATTN_ERR_INVALID_ARG;
+  if (k != nullptr) {
+    if (k_out != k && overlap(k_out, nk * 2, k, nk * 2)) return ATTN_ERR_INVALID_ARG;
+    if (overlap(q_out, nq * 2, k, nk * 2) || overlap(k_out, nk * 2, q, nq * 2) ||
+        overlap(q_out, nq * 2, k_out, nk * 2))
+      return ATTN_ERR_INVALID_ARG;
+  }
+
+  ProParams p{};
+  p.t[0] = ProTensor{q, q_out, norm_scope ? gamma_q : nullptr, angles_q, Lq, Hq};
+  p.t[1] = ProTensor{k, k_out, norm_scope ? gamma_k : nullptr, angles_k, Lk, Hkv};
+  p.tokens0 = B * Lq;
+  p.d = d;
+  p.eps = eps;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  (void)cudaGetLastError();
+  launch_prologue(p, dtype == ATTN_DTYPE_BF16, norm_scope, rope_style, static_cast<unsigned>(tokens), s);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}

@@ -115,3 +115,27 @@ def sample_rows(Lq: int, n: int, seed: int):
     g = torch.Generator(device="cpu")
     g.manual_seed(int(seed) + 1000)
     return torch.randperm(Lq, generator=g)[:n].sort().values
+
+
+def rope_angle_table(L: int, d: int, style: int, pos0: int = 0, base: float = 10000.0) -> torch.Tensor:
+    """The caller-side ``rope_freqs`` input: float32 [L, d] rotation angles for
+    sequence positions ``pos0 .. pos0 + L - 1``, built as the developer guide
+    ("Multi Head Attention Definition") describes the model doing it: pair r
+    of a head gets ``theta = p * base**(-2 r / d)``, and the table is
+    "expanded" to one angle per feature, the pair's angle stored at both of its
+    features ((2r, 2r + 1) for style 1, interleaved; (r, r + d/2) for style 2,
+    split-half). The prologue reads it; it computes no angles itself.
+    """
+    r = torch.arange(d // 2, dtype=torch.float64)
+    omega = base ** (-2.0 * r / d)
+    theta = (pos0 + torch.arange(L, dtype=torch.float64))[:, None] * omega[None, :]
+    table = torch.empty(L, d, dtype=torch.float64)
+    if style == 1:
+        table[:, 0::2] = theta
+        table[:, 1::2] = theta
+    elif style == 2:
+        table[:, : d // 2] = theta
+        table[:, d // 2:] = theta
+    else:
+        raise ValueError("style must be 1 (interleaved) or 2 (split-half)")
+    return table.to(torch.float32)

@@ -96,6 +96,61 @@ int attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, vo
                   float* lse_dev, int B, int Lq, int Lk, int Hq, int Hkv, int d, float scale,
                   int causal, int kv_offset, int dtype, void* stream);
 
+typedef enum {
+  ATTN_NORM_NONE = 0,   /* Q and K unchanged */
+  ATTN_NORM_HEAD = 1,   /* RMSNorm over each head's d features (m = d) */
+  ATTN_NORM_INNER = 2   /* RMSNorm over all H*d features of a token (m = H d) */
+} attn_norm_scope_t;
+
+typedef enum {
+  ATTN_ROPE_NONE = 0,        /* no rotation */
+  ATTN_ROPE_INTERLEAVED = 1, /* pair r = features (2r, 2r + 1) */
+  ATTN_ROPE_SPLIT = 2        /* pair r = features (r, r + d/2) */
+} attn_rope_style_t;
+
+/*
+ * attn_qk_prologue — Q/K RMS normalisation followed by rotary position
+ * embedding, for Q and (optionally) the new K chunk in one launch,
+ * asynchronous on `stream`.
+ *
+ * Operation (developer guide, "Multi Head Attention Definition"): for every
+ * token, RMSNorm_gamma(z) = gamma * z / sqrt(mean(z^2) + eps) over each head
+ * (ATTN_NORM_HEAD) or over the whole token (ATTN_NORM_INNER); then feature
+ * pair r of the token at sequence index p is rotated by the angle
+ * angles[p * d + a_r], where a_r is the pair's first feature (2r interleaved,
+ * r split-half): (z_a, z_b) -> (z_a cos - z_b sin, z_a sin + z_b cos). The
+ * page normalises before RoPE; so does this call. Arithmetic in float32 from
+ * the 16-bit inputs, one round-to-nearest to dtype at the end. V is not
+ * touched.
+ *
+ * Arguments (tensors contiguous, row-major; 16-bit tensors 16-byte aligned,
+ * float arrays 4-byte aligned):
+ *   q      device, [B, Lq, Hq, d] of dtype                   (read)
+ *   q_out  device, [B, Lq, Hq, d] of dtype (written; may equal q for in place,
+ *          must not otherwise overlap any other operand)
+ *   k, k_out  as q / q_out with [B, Lk, Hkv, d]; both NULL to process Q only
+ *   gamma_q, gamma_k  device float32 weights of length d (head scope) or
+ *          Hq*d / Hkv*d (inner scope); NULL means all ones; ignored for
+ *          ATTN_NORM_NONE
+ *   angles_q, angles_k  device float32 [Lq, d] / [Lk, d]: the expanded angle
+ *          table rope_freqs[L, 1, 1, d] of the pages, one angle per feature
+ *          (row p is sequence index p of every batch); NULL iff
+ *          rope_style == ATTN_ROPE_NONE
+ *   d      a power of two, 16..256
+ *   norm_scope  attn_norm_scope_t; eps finite, >= 0 (1e-6 in the pages)
+ *   rope_style  attn_rope_style_t
+ *   dtype  attn_dtype_t of q, q_out, k, k_out
+ *
+ * Errors: every argument is checked before any CUDA call; a violation returns
+ * ATTN_ERR_INVALID_ARG (ATTN_ERR_UNSUPPORTED for another head_dim) and
+ * launches nothing. A failed launch returns ATTN_ERR_CUDA. No allocation, no
+ * synchronisation.
+ */
+int attn_qk_prologue(const void* q, void* q_out, const void* k, void* k_out,
+                     const float* gamma_q, const float* gamma_k, const float* angles_q,
+                     const float* angles_k, int B, int Lq, int Lk, int Hq, int Hkv, int d,
+                     int norm_scope, float eps, int rope_style, int dtype, void* stream);
+
 /* Short English text of a status code (static storage). */
 const char* attn_status_string(int status);
 

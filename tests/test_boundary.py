@@ -106,3 +106,47 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(binding, "_SO_PATH", str(tmp_path / "absent.so"))
     with pytest.raises(RuntimeError, match="missing"):
         binding.lib()
+
+
+# ----------------------------------------------------------- Q/K prologue
+
+def _pro(**kw):
+    args = dict(q=A, q_out=A + 0x100000, k=A + 0x200000, k_out=A + 0x300000, gq=None, gk=None,
+                aq=A + 0x400000, ak=A + 0x500000, B=1, Lq=4, Lk=4, Hq=2, Hkv=1, d=64,
+                scope=1, eps=1e-6, style=2, dtype=0)
+    args.update(kw)
+    return hasb.lib().attn_qk_prologue(args["q"], args["q_out"], args["k"], args["k_out"], args["gq"],
+                                       args["gk"], args["aq"], args["ak"], args["B"], args["Lq"],
+                                       args["Lk"], args["Hq"], args["Hkv"], args["d"], args["scope"],
+                                       args["eps"], args["style"], args["dtype"], None)
+
+
+PRO_INVALID = [
+    dict(q=None), dict(q_out=None), dict(k_out=None), dict(k=None),   # k and k_out both or neither
+    dict(B=0), dict(Lq=0), dict(Lk=0), dict(Hq=0), dict(Hkv=0),
+    dict(scope=3), dict(scope=-1), dict(style=3), dict(style=-1),
+    dict(eps=-1e-6), dict(eps=float("nan")), dict(eps=float("inf")), dict(dtype=2),
+    dict(aq=None), dict(ak=None),                 # RoPE requested without angles
+    dict(style=0),                                # angles given without RoPE
+    dict(q=A + 8), dict(k_out=A + 0x300000 + 4), dict(gq=A + 0x600000 + 2), dict(aq=A + 0x400000 + 1),
+    dict(q_out=A + 64),                           # partial overlap of q_out and q
+    dict(k_out=A + 0x100000),                     # k_out overlaps q_out
+    dict(q_out=A + 0x200000),                     # q_out overlaps k
+]
+
+
+@pytest.mark.parametrize("kw", PRO_INVALID, ids=[str(k) for k in PRO_INVALID])
+def test_prologue_invalid_arguments_are_rejected_before_any_launch(kw):
+    assert _pro(**kw) == hasb.ATTN_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("d", [8, 24, 96, 512])
+def test_prologue_head_dims_outside_16_to_256_powers_of_two_are_unsupported(d):
+    assert _pro(d=d) == hasb.ATTN_ERR_UNSUPPORTED
+
+
+def test_prologue_python_binding_rejects_cpu_tensors():
+    import torch
+    q = torch.zeros(1, 4, 2, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        hasb.qk_prologue(q)
