@@ -45,6 +45,10 @@ _SIGNATURES = {
                       [ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
     "attn_qk_prologue": (ctypes.c_int, [ctypes.c_void_p] * 8 + [ctypes.c_int] * 7 +
                          [ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
+    "attn_stream_update": (ctypes.c_int, [ctypes.c_void_p] * 10 + [ctypes.c_int] * 7 +
+                           [ctypes.c_int, ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
+    "attn_fwd_cache": (ctypes.c_int, [ctypes.c_void_p] * 5 + [ctypes.c_int] * 7 +
+                       [ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
     "attn_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "attn_device_fault": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint), ctypes.c_int]),
     "attn_set_wait_timeout_ns": (ctypes.c_int, [ctypes.c_ulonglong]),
@@ -192,6 +196,76 @@ def qk_prologue(q: torch.Tensor, k: torch.Tensor | None = None, *, norm_scope: i
     if st != ATTN_OK:
         raise AttnError(st, "attn_qk_prologue")
     return out_q, (out_k if k is not None else None)
+
+
+def stream_update(k: torch.Tensor, v: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                  slot: int, *, q: torch.Tensor | None = None, q_out: torch.Tensor | None = None,
+                  norm_scope: int = NORM_NONE, eps: float = 1e-6, gamma_q=None, gamma_k=None,
+                  rope_style: int = ROPE_NONE, angles_q=None, angles_k=None, stream=None):
+    """Write the chunk's K (normalised and rotated) and V into cache slots
+    ``slot .. slot + L - 1`` and, when ``q`` is given, the query prologue,
+    through ``attn_stream_update`` of the C ABI. Returns ``q_out`` (or None).
+
+    k, v: [B, L, Hkv, d]; k_cache, v_cache: [B, S, Hkv, d]; q: [B, L, Hq, d].
+    """
+    for name, t in (("k", k), ("v", v), ("k_cache", k_cache), ("v_cache", v_cache)) + \
+            ((("q", q),) if q is not None else ()):
+        if not t.is_cuda or not t.is_contiguous() or t.dim() != 4 or t.dtype not in DTYPE_CODES:
+            raise ValueError(f"{name} must be a contiguous 4-D bf16/fp16 CUDA tensor")
+    B, L, Hkv, d = k.shape
+    if v.shape != k.shape or k_cache.shape != v_cache.shape or k_cache.shape[0] != B or \
+            k_cache.shape[2:] != (Hkv, d) or len({t.dtype for t in (k, v, k_cache, v_cache)}) != 1:
+        raise ValueError("k, v and the caches must agree in batch, heads, head_dim and dtype")
+    S = k_cache.shape[1]
+    Hq = 0
+    if q is not None:
+        if q.dtype != k.dtype or q.shape[0] != B or q.shape[1] != L or q.shape[3] != d:
+            raise ValueError("q must be [B, L, Hq, d] in k's dtype")
+        Hq = q.shape[2]
+        if q_out is None:
+            q_out = torch.empty_like(q)
+    wq = d if norm_scope == NORM_HEAD else Hq * d
+    wk = d if norm_scope == NORM_HEAD else Hkv * d
+    _check_f32("gamma_q", gamma_q, wq, k.device)
+    _check_f32("gamma_k", gamma_k, wk, k.device)
+    _check_f32("angles_q", angles_q, L * d, k.device)
+    _check_f32("angles_k", angles_k, L * d, k.device)
+    st = lib().attn_stream_update(_ptr(q), _ptr(q_out), _ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache),
+                                  _ptr(gamma_q), _ptr(gamma_k), _ptr(angles_q), _ptr(angles_k), B, L, S,
+                                  int(slot), Hq, Hkv, d, int(norm_scope), float(eps), int(rope_style),
+                                  DTYPE_CODES[k.dtype], _stream_handle(stream, k.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_stream_update")
+    return q_out
+
+
+def attn_fwd_cache(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, Lk: int, *,
+                   scale: float | None = None, causal: int = MASK_NONE, kv_offset: int = 0,
+                   out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+                   return_lse: bool = True, stream=None):
+    """``attn_fwd`` over the first ``Lk`` tokens of [B, S, Hkv, d] caches
+    (``attn_fwd_cache`` of the C ABI). Returns ``(out, lse)``."""
+    for name, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
+        if not t.is_cuda or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError(f"{name} must be a contiguous 4-D CUDA tensor")
+    if q.dtype not in DTYPE_CODES or k_cache.dtype != q.dtype or v_cache.dtype != q.dtype:
+        raise ValueError("q and the caches must share one dtype, bf16 or fp16")
+    if k_cache.shape != v_cache.shape:
+        raise ValueError("k_cache and v_cache must have the same shape")
+    B, Lq, Hq, d = q.shape
+    S, Hkv = k_cache.shape[1], k_cache.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
+    st = lib().attn_fwd_cache(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(lse), B, Lq, int(Lk),
+                              S, Hq, Hkv, d, float(scale), int(causal), int(kv_offset),
+                              DTYPE_CODES[q.dtype], _stream_handle(stream, q.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fwd_cache")
+    return out, lse
 
 
 def attn_fwd_host(q_host, k_host, v_host, o_host, lse_host, q_dev, k_dev, v_dev, o_dev, lse_dev, *,

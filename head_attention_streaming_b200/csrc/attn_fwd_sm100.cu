@@ -890,11 +890,15 @@ DeviceInfo device_info(int dev) {
 
 // [B, L, H, d] 16-bit tensor as a 4-D TMA map (innermost first: d, H, L, B);
 // box = 64 elements of d x 1 head x 128 rows x 1 batch, 128-byte swizzle.
-bool encode_bl_hd(CUtensorMap* map, const void* ptr, int B, int L, int H, int d, bool bf16) {
+// Consecutive batches are `batch_rows` rows apart (L for a contiguous tensor,
+// the capacity S when the rows are the valid prefix of a [B, S, H, d] cache).
+bool encode_bl_hd(CUtensorMap* map, const void* ptr, int B, int L, int H, int d, bool bf16,
+                  int batch_rows = -1) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
+  const cuuint64_t rows = batch_rows < 0 ? (cuuint64_t)L : (cuuint64_t)batch_rows;
   const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)L, (cuuint64_t)B};
-  const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2, (cuuint64_t)L * H * d * 2};
+  const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2, rows * H * d * 2};
   const cuuint32_t box[4] = {64, 1, (cuuint32_t)kTileRows, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
@@ -905,13 +909,13 @@ bool encode_bl_hd(CUtensorMap* map, const void* ptr, int B, int L, int H, int d,
 }
 
 template <int D, bool BF16, bool CAUSAL>
-int launch_fwd(const FwdParams& p, const void* q, const void* k, const void* v, int grid,
+int launch_fwd(const FwdParams& p, const void* q, const void* k, const void* v, int kv_rows, int grid,
                cudaStream_t stream) {
   using C = Cfg<D>;
   CUtensorMap tq, tk, tv, to;
   if (!encode_bl_hd(&tq, q, p.B, p.Lq, p.Hq, D, BF16) ||
-      !encode_bl_hd(&tk, k, p.B, p.Lk, p.Hkv, D, BF16) ||
-      !encode_bl_hd(&tv, v, p.B, p.Lk, p.Hkv, D, BF16) ||
+      !encode_bl_hd(&tk, k, p.B, p.Lk, p.Hkv, D, BF16, kv_rows) ||
+      !encode_bl_hd(&tv, v, p.B, p.Lk, p.Hkv, D, BF16, kv_rows) ||
       !encode_bl_hd(&to, p.o, p.B, p.Lq, p.Hq, D, BF16))
     return ATTN_ERR_CUDA;
   auto kern = attn_fwd_sm100_kernel<D, BF16, CAUSAL>;
@@ -983,7 +987,7 @@ namespace hasb {
 // The argument contract of attn_fwd; makes no CUDA call.
 int attn_fwd_validate(const void* q, const void* k, const void* v, const void* o, const float* lse,
                       int B, int Lq, int Lk, int Hq, int Hkv, int d, float scale, int causal,
-                      int kv_offset, int dtype) {
+                      int kv_offset, int dtype, int kv_rows) {
   // ---- argument contract (no CUDA call before this block is passed)
   if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return ATTN_ERR_INVALID_ARG;
   if (B < 1 || Lq < 1 || Lk < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
@@ -1001,7 +1005,8 @@ int attn_fwd_validate(const void* q, const void* k, const void* v, const void* o
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ATTN_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return ATTN_ERR_INVALID_ARG;
   const unsigned long long q_elems = 1ull * B * Lq * Hq * d;
-  const unsigned long long kv_elems = 1ull * B * Lk * Hkv * d;
+  if (kv_rows < Lk) return ATTN_ERR_INVALID_ARG;
+  const unsigned long long kv_elems = 1ull * B * kv_rows * Hkv * d;
   if (q_elems * 2 >= (1ull << 40) || kv_elems * 2 >= (1ull << 40)) return ATTN_ERR_INVALID_ARG;
   const long long n_pairs = (Lq + 2LL * kTileRows - 1) / (2LL * kTileRows);
   const long long n_units = n_pairs * B * Hq;
@@ -1013,16 +1018,13 @@ int attn_fwd_validate(const void* q, const void* k, const void* v, const void* o
   return ATTN_OK;
 }
 
-}  // namespace hasb
-
-extern "C" {
-
-int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Lq,
-             int Lk, int Hq, int Hkv, int d, float scale, int causal, int kv_offset, int dtype,
-             void* stream) {
+// attn_fwd over K/V whose consecutive batches are kv_rows rows apart.
+int attn_fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Lq,
+                  int Lk, int kv_rows, int Hq, int Hkv, int d, float scale, int causal, int kv_offset,
+                  int dtype, void* stream) {
   // ---- argument contract (no CUDA call before it passes)
   const int valid = attn_fwd_validate(q, k, v, o, lse, B, Lq, Lk, Hq, Hkv, d, scale, causal,
-                                      kv_offset, dtype);
+                                      kv_offset, dtype, kv_rows);
   if (valid != ATTN_OK) return valid;
   const long long n_pairs = (Lq + 2LL * kTileRows - 1) / (2LL * kTileRows);
   const long long n_units = n_pairs * B * Hq;
@@ -1049,11 +1051,30 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   const bool bf16 = dtype == ATTN_DTYPE_BF16;
   const bool cz = causal == ATTN_MASK_CAUSAL;
   if (d == 128) {
-    if (bf16) return cz ? launch_fwd<128, true, true>(p, q, k, v, grid, s) : launch_fwd<128, true, false>(p, q, k, v, grid, s);
-    return cz ? launch_fwd<128, false, true>(p, q, k, v, grid, s) : launch_fwd<128, false, false>(p, q, k, v, grid, s);
+    if (bf16) return cz ? launch_fwd<128, true, true>(p, q, k, v, kv_rows, grid, s) : launch_fwd<128, true, false>(p, q, k, v, kv_rows, grid, s);
+    return cz ? launch_fwd<128, false, true>(p, q, k, v, kv_rows, grid, s) : launch_fwd<128, false, false>(p, q, k, v, kv_rows, grid, s);
   }
-  if (bf16) return cz ? launch_fwd<64, true, true>(p, q, k, v, grid, s) : launch_fwd<64, true, false>(p, q, k, v, grid, s);
-  return cz ? launch_fwd<64, false, true>(p, q, k, v, grid, s) : launch_fwd<64, false, false>(p, q, k, v, grid, s);
+  if (bf16) return cz ? launch_fwd<64, true, true>(p, q, k, v, kv_rows, grid, s) : launch_fwd<64, true, false>(p, q, k, v, kv_rows, grid, s);
+  return cz ? launch_fwd<64, false, true>(p, q, k, v, kv_rows, grid, s) : launch_fwd<64, false, false>(p, q, k, v, kv_rows, grid, s);
+}
+
+}  // namespace hasb
+
+extern "C" {
+
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Lq,
+             int Lk, int Hq, int Hkv, int d, float scale, int causal, int kv_offset, int dtype,
+             void* stream) {
+  return attn_fwd_impl(q, k, v, o, lse, B, Lq, Lk, Lk, Hq, Hkv, d, scale, causal, kv_offset, dtype,
+                       stream);
+}
+
+int attn_fwd_cache(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
+                   int B, int Lq, int Lk, int S, int Hq, int Hkv, int d, float scale, int causal,
+                   int kv_offset, int dtype, void* stream) {
+  if (S < 1) return ATTN_ERR_INVALID_ARG;
+  return attn_fwd_impl(q, k_cache, v_cache, o, lse, B, Lq, Lk, S, Hq, Hkv, d, scale, causal,
+                       kv_offset, dtype, stream);
 }
 
 int attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, void* o_host,
@@ -1070,7 +1091,7 @@ int attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, vo
   // attn_fwd checks the device side; run its validation first by a dry call
   // ordering: copies only once the arguments are known to be valid
   const int pre = attn_fwd_validate(q_dev, k_dev, v_dev, o_dev, lse_dev, B, Lq, Lk, Hq, Hkv, d, scale,
-                                    causal, kv_offset, dtype);
+                                    causal, kv_offset, dtype, Lk);
   if (pre != ATTN_OK) return pre;
   if (cudaMemcpyAsync(q_dev, q_host, q_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
       cudaMemcpyAsync(k_dev, k_host, kv_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||

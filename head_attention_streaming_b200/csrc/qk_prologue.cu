@@ -35,17 +35,22 @@ namespace hasb_pro {
 constexpr int kWarps = 4;
 constexpr int kThreads = 32 * kWarps;
 
+// One input tensor [B, L, H, d] and where its tokens go: token (b, l) is
+// written to token b * ystride + yoff + l of the output (ystride = L, yoff = 0
+// for a plain [B, L, H, d] output; a cache slot range otherwise).
 struct ProTensor {
   const void* x;
   void* y;
   const float* gamma;   // [m] or nullptr (all ones)
   const float* angles;  // [L, d] or nullptr (no RoPE)
   int L, H;
+  int ystride, yoff;
+  int raw;              // copy only: neither normalised nor rotated (V)
 };
 
 struct ProParams {
-  ProTensor t[2];
-  int tokens0;  // B * L of tensor 0; blocks past it belong to tensor 1
+  ProTensor t[3];
+  int tok_end[3];  // cumulative token counts: block i serves the first tensor with i < tok_end
   int d;
   float eps;  // normalisation scope and RoPE style are template arguments of the kernel
 };
@@ -93,18 +98,21 @@ __global__ void __launch_bounds__(kThreads) qk_prologue_kernel(const ProParams p
   __shared__ float cs_s[128], sn_s[128];  // cos / sin of the token's d/2 pair angles
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  const int which = blockIdx.x < p.tokens0 ? 0 : 1;
-  const ProTensor T = which ? p.t[1] : p.t[0];
-  const int token = which ? blockIdx.x - p.tokens0 : blockIdx.x;  // b * L + l
-  const int pos = token % T.L;                                     // sequence index l
+  const int bid = blockIdx.x;
+  const int which = bid < p.tok_end[0] ? 0 : (bid < p.tok_end[1] ? 1 : 2);
+  const ProTensor T = which == 0 ? p.t[0] : (which == 1 ? p.t[1] : p.t[2]);
+  const int token = bid - (which == 0 ? 0 : p.tok_end[which - 1]);  // b * L + l
+  const int pos = token % T.L;                                      // sequence index l
+  const int bat = token / T.L;
+  const bool raw = T.raw != 0;
   const int d = p.d;
   constexpr bool split = STYLE == ATTN_ROPE_SPLIT;
   const int per_head = d / 16;                  // items per head
   const int sh = __ffs(per_head) - 1;           // log2(per_head)
   const int items = T.H * per_head;             // items of the token
-  const size_t base = static_cast<size_t>(token) * T.H * d;
-  const uint16_t* x = static_cast<const uint16_t*>(T.x) + base;
-  uint16_t* y = static_cast<uint16_t*>(T.y) + base;
+  const uint16_t* x = static_cast<const uint16_t*>(T.x) + static_cast<size_t>(token) * T.H * d;
+  uint16_t* y = static_cast<uint16_t*>(T.y) +
+                (static_cast<size_t>(bat) * T.ystride + T.yoff + pos) * T.H * d;
   // intra-head item index is the same for every item this thread handles
   // (128 is a multiple of d / 16)
   const int io = threadIdx.x % per_head;
@@ -112,13 +120,13 @@ __global__ void __launch_bounds__(kThreads) qk_prologue_kernel(const ProParams p
 
   if constexpr (STYLE != ATTN_ROPE_NONE) {
     // pair r: first feature a_r = 2r (interleaved) or r (split-half)
-    if (threadIdx.x < d / 2) {
+    if (!raw && threadIdx.x < d / 2) {
       const int a = split ? threadIdx.x : 2 * threadIdx.x;
       sincosf(T.angles[static_cast<size_t>(pos) * d + a], &sn_s[threadIdx.x], &cs_s[threadIdx.x]);
     }
   }
   float ghead[16];
-  if (SCOPE == ATTN_NORM_HEAD) {
+  if (SCOPE == ATTN_NORM_HEAD && !raw) {
 #pragma unroll
     for (int e = 0; e < 16; ++e)
       ghead[e] = T.gamma != nullptr ? T.gamma[item_feature(o, e, d, split)] : 1.f;
@@ -134,7 +142,7 @@ __global__ void __launch_bounds__(kThreads) qk_prologue_kernel(const ProParams p
 
   // inner scope: one sum of squares over the whole token first
   float inv_token = 1.f;
-  if (SCOPE == ATTN_NORM_INNER) {
+  if (SCOPE == ATTN_NORM_INNER && !raw) {
     float ss = 0.f;
     for (int it = threadIdx.x; it < items; it += kThreads) {
       float f[16];
@@ -147,12 +155,12 @@ __global__ void __launch_bounds__(kThreads) qk_prologue_kernel(const ProParams p
     if (lane == 0) red[warp] = ss;
   }
   __syncthreads();  // cos / sin table and partial sums visible
-  if (SCOPE == ATTN_NORM_INNER) {
+  if (SCOPE == ATTN_NORM_INNER && !raw) {
     const float tot = (red[0] + red[1]) + (red[2] + red[3]);
     inv_token = rsqrtf(tot / static_cast<float>(T.H * d) + p.eps);
   }
   float c8[8], s8[8];
-  if (STYLE != ATTN_ROPE_NONE) {
+  if (STYLE != ATTN_ROPE_NONE && !raw) {
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       // split: element e and e + 8 form pair o/1 + e; interleaved: elements
@@ -174,7 +182,9 @@ __global__ void __launch_bounds__(kThreads) qk_prologue_kernel(const ProParams p
 #pragma unroll
       for (int m = 0; m < 8; ++m) f[m] = make_float2(0.f, 0.f);
     }
-    if (SCOPE == ATTN_NORM_HEAD) {
+    if (raw) {
+      // copy only
+    } else if (SCOPE == ATTN_NORM_HEAD) {
       float2 ss2 = make_float2(0.f, 0.f);
 #pragma unroll
       for (int m = 0; m < 8; ++m) ss2 = __ffma2_rn(f[m], f[m], ss2);
@@ -196,7 +206,8 @@ __global__ void __launch_bounds__(kThreads) qk_prologue_kernel(const ProParams p
         f[m] = __fmul2_rn(gg, __fmul2_rn(f[m], inv2));
       }
     }
-    if constexpr (split) {
+    if (raw) {
+    } else if constexpr (split) {
       // element e (< 8) pairs with element e + 8: f[m] holds elements 2m, 2m+1
       // of the first vector, f[m + 4] the same two of the second
 #pragma unroll
@@ -300,13 +311,71 @@ extern "C" int attn_qk_prologue(const void* q, void* q_out, const void* k, void*
   }
 
   ProParams p{};
-  p.t[0] = ProTensor{q, q_out, norm_scope ? gamma_q : nullptr, angles_q, Lq, Hq};
-  p.t[1] = ProTensor{k, k_out, norm_scope ? gamma_k : nullptr, angles_k, Lk, Hkv};
-  p.tokens0 = B * Lq;
+  p.t[0] = ProTensor{q, q_out, norm_scope ? gamma_q : nullptr, angles_q, Lq, Hq, Lq, 0, 0};
+  p.t[1] = ProTensor{k, k_out, norm_scope ? gamma_k : nullptr, angles_k, Lk, Hkv, Lk, 0, 0};
+  p.tok_end[0] = B * Lq;
+  p.tok_end[1] = p.tok_end[2] = static_cast<int>(tokens);
   p.d = d;
   p.eps = eps;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   (void)cudaGetLastError();
   launch_prologue(p, dtype == ATTN_DTYPE_BF16, norm_scope, rope_style, static_cast<unsigned>(tokens), s);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+extern "C" int attn_stream_update(const void* q, void* q_out, const void* k, const void* v,
+                                  void* k_cache, void* v_cache, const float* gamma_q,
+                                  const float* gamma_k, const float* angles_q, const float* angles_k,
+                                  int B, int L, int S, int slot, int Hq, int Hkv, int d,
+                                  int norm_scope, float eps, int rope_style, int dtype, void* stream) {
+  // ---- arguments (all checked before any CUDA call)
+  if (k == nullptr || v == nullptr || k_cache == nullptr || v_cache == nullptr)
+    return ATTN_ERR_INVALID_ARG;
+  if ((q == nullptr) != (q_out == nullptr)) return ATTN_ERR_INVALID_ARG;
+  if (dtype != ATTN_DTYPE_BF16 && dtype != ATTN_DTYPE_FP16) return ATTN_ERR_INVALID_ARG;
+  if (norm_scope < ATTN_NORM_NONE || norm_scope > ATTN_NORM_INNER) return ATTN_ERR_INVALID_ARG;
+  if (rope_style < ATTN_ROPE_NONE || rope_style > ATTN_ROPE_SPLIT) return ATTN_ERR_INVALID_ARG;
+  if (!(eps >= 0.f) || !std::isfinite(eps)) return ATTN_ERR_INVALID_ARG;
+  if (B < 1 || L < 1 || Hkv < 1 || (q != nullptr && Hq < 1)) return ATTN_ERR_INVALID_ARG;
+  if (slot < 0 || S < 1 || L > S || slot > S - L) return ATTN_ERR_INVALID_ARG;
+  if (d < 16 || d > 256 || (d & (d - 1)) != 0) return ATTN_ERR_UNSUPPORTED;
+  if ((rope_style != ATTN_ROPE_NONE) != (angles_k != nullptr)) return ATTN_ERR_INVALID_ARG;
+  if (q != nullptr && (rope_style != ATTN_ROPE_NONE) != (angles_q != nullptr)) return ATTN_ERR_INVALID_ARG;
+  for (const void* t : {q, static_cast<const void*>(q_out), k, v, static_cast<const void*>(k_cache),
+                        static_cast<const void*>(v_cache)})
+    if (t != nullptr && !aligned(t, 16)) return ATTN_ERR_INVALID_ARG;
+  for (const float* f : {gamma_q, gamma_k, angles_q, angles_k})
+    if (f != nullptr && !aligned(f, 4)) return ATTN_ERR_INVALID_ARG;
+  const long long tok_q = q ? 1LL * B * L : 0, tok_kv = 1LL * B * L;
+  if (tok_q + 2 * tok_kv > 0x7fffffffLL || 1LL * Hq * d > (1 << 20) || 1LL * Hkv * d > (1 << 20))
+    return ATTN_ERR_INVALID_ARG;
+  const size_t nq = static_cast<size_t>(tok_q) * Hq * d * 2, nkv = static_cast<size_t>(tok_kv) * Hkv * d * 2;
+  const size_t ncache = static_cast<size_t>(B) * S * Hkv * d * 2;
+  // the caches are written: they may overlap no input and not each other; q_out
+  // may be q (in place) and may overlap nothing else
+  if (overlap(k_cache, ncache, v_cache, ncache)) return ATTN_ERR_INVALID_ARG;
+  for (const void* c : {static_cast<const void*>(k_cache), static_cast<const void*>(v_cache)}) {
+    if (overlap(c, ncache, k, nkv) || overlap(c, ncache, v, nkv)) return ATTN_ERR_INVALID_ARG;
+    if (q != nullptr && (overlap(c, ncache, q, nq) || overlap(c, ncache, q_out, nq)))
+      return ATTN_ERR_INVALID_ARG;
+  }
+  if (q != nullptr) {
+    if (q_out != q && overlap(q_out, nq, q, nq)) return ATTN_ERR_INVALID_ARG;
+    if (overlap(q_out, nq, k, nkv) || overlap(q_out, nq, v, nkv)) return ATTN_ERR_INVALID_ARG;
+  }
+
+  ProParams p{};
+  p.t[0] = ProTensor{q, q_out, norm_scope ? gamma_q : nullptr, angles_q, L, Hq, L, 0, 0};
+  p.t[1] = ProTensor{k, k_cache, norm_scope ? gamma_k : nullptr, angles_k, L, Hkv, S, slot, 0};
+  p.t[2] = ProTensor{v, v_cache, nullptr, nullptr, L, Hkv, S, slot, 1};
+  p.tok_end[0] = static_cast<int>(tok_q);
+  p.tok_end[1] = static_cast<int>(tok_q + tok_kv);
+  p.tok_end[2] = static_cast<int>(tok_q + 2 * tok_kv);
+  p.d = d;
+  p.eps = eps;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  (void)cudaGetLastError();
+  launch_prologue(p, dtype == ATTN_DTYPE_BF16, norm_scope, rope_style,
+                  static_cast<unsigned>(p.tok_end[2]), s);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }

@@ -81,6 +81,16 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
              int causal, int kv_offset, int dtype, void* stream);
 
 /*
+ * attn_fwd_cache — attn_fwd with K and V read from the first Lk tokens of a
+ * [B, S, Hkv, d] cache (the rolling block cache of streaming self-attention,
+ * whose valid tokens are a prefix of its S slots): batch b's keys start at
+ * k_cache + b * S * Hkv * d. Lk <= S. Everything else as attn_fwd.
+ */
+int attn_fwd_cache(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
+                   int B, int Lq, int Lk, int S, int Hq, int Hkv, int d, float scale, int causal,
+                   int kv_offset, int dtype, void* stream);
+
+/*
  * attn_fwd_host — the same forward for operands in host memory: copies q, k, v
  * from host to the caller's device buffers, runs attn_fwd, and copies o (and
  * lse when both lse pointers are given) back to host memory, all queued on
@@ -150,6 +160,37 @@ int attn_qk_prologue(const void* q, void* q_out, const void* k, void* k_out,
                      const float* gamma_q, const float* gamma_k, const float* angles_q,
                      const float* angles_k, int B, int Lq, int Lk, int Hq, int Hkv, int d,
                      int norm_scope, float eps, int rope_style, int dtype, void* stream);
+
+/*
+ * attn_stream_update — the K/V cache update of one streaming self-attention
+ * step, with the query prologue, in one launch, asynchronous on `stream`.
+ *
+ * Operation (developer guide, "Generic Multi Head Attention Interface"; user
+ * guide, "Cache lifecycle"): the current chunk's K/V are written into the
+ * rolling block cache before the chunk is queried, keys with before-cache
+ * RoPE already rotated. For every batch b and chunk token i < L:
+ *   k_cache[b, slot + i] = RoPE(RMSNorm(k[b, i]))   (as attn_qk_prologue)
+ *   v_cache[b, slot + i] = v[b, i]                  (copied; V is never
+ *                                                    normalised or rotated)
+ *   q_out[b, i]          = RoPE(RMSNorm(q[b, i]))   (when q is given)
+ * The angle row of token i is i (the tables hold the chunk's positions).
+ *
+ * Arguments (16-bit tensors contiguous and 16-byte aligned):
+ *   q, q_out  device [B, L, Hq, d] of dtype, or both NULL; q_out may equal q
+ *   k, v      device [B, L, Hkv, d] of dtype (read)
+ *   k_cache, v_cache  device [B, S, Hkv, d] of dtype; tokens slot .. slot+L-1
+ *             of every batch are written, nothing else is touched
+ *   gamma_*, angles_*, norm_scope, eps, rope_style, d  as attn_qk_prologue
+ *             (angles_q / angles_k: [L, d])
+ *   0 <= slot and slot + L <= S
+ * Errors as attn_qk_prologue; additionally the caches may overlap no input and
+ * not each other. No allocation, no synchronisation.
+ */
+int attn_stream_update(const void* q, void* q_out, const void* k, const void* v, void* k_cache,
+                       void* v_cache, const float* gamma_q, const float* gamma_k,
+                       const float* angles_q, const float* angles_k, int B, int L, int S, int slot,
+                       int Hq, int Hkv, int d, int norm_scope, float eps, int rope_style, int dtype,
+                       void* stream);
 
 /* Short English text of a status code (static storage). */
 const char* attn_status_string(int status);

@@ -1,0 +1,103 @@
+"""Streaming self-attention through the rolling block K/V cache on a B200,
+against the FP64 oracle: before_update, attend (the chunk's Q/K RMSNorm and
+before-cache RoPE, its K/V written into the cache, attention over every valid
+cached key), after_update, for streams that fill the cache and then evict.
+
+Expected values: the prologue oracle on the 16-bit inputs, rounded to the
+16-bit type (the cache stores 16-bit K; Q enters the attention as 16 bits),
+then the rolling-cache oracle. Bars as in the attention parity tests.
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import head_attention_streaming_b200 as hasb
+import oracle
+from head_attention_streaming_b200.inputs import rope_angle_table
+from oracle import prologue as qp
+from oracle import rolling_cache as rc
+from test_parity_gpu import _check
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _device(cuda_ok):
+    torch.cuda.set_device(0)
+    yield
+    assert hasb.device_fault(clear=True) == 0
+
+
+def _round16(x: np.ndarray, dtype) -> np.ndarray:
+    return torch.from_numpy(x).to(dtype).to(torch.float64).numpy()
+
+
+def _stream(B, C, sink, window, Hq, Hkv, d, n_chunks, dtype, norm, style, seed, sample_rows=None):
+    g = torch.Generator().manual_seed(seed)
+    T = n_chunks * C
+    q = torch.randn(B, T, Hq, d, generator=g).to(dtype)
+    k = torch.randn(B, T, Hkv, d, generator=g).to(dtype)
+    v = torch.randn(B, T, Hkv, d, generator=g).to(dtype)
+    wq, wk = (d, d) if norm == qp.NORM_HEAD else (Hq * d, Hkv * d)
+    gq = (1.0 + 0.1 * torch.randn(wq, generator=g)) if norm else None
+    gk = (1.0 + 0.1 * torch.randn(wk, generator=g)) if norm else None
+    ang = rope_angle_table(T, d, style, 0) if style else None
+    scale = 1.0 / math.sqrt(d)
+    eps = 1e-6
+    f64 = lambda t: None if t is None else t.to(torch.float64).numpy()
+    kn = _round16(qp.qk_prologue(f64(k), f64(gk), eps, norm, f64(ang), style), dtype)
+    vn = f64(v)
+    cache = hasb.BlockKVCache(B, Hkv, d, C, window, sink, dtype=dtype)
+    dev = lambda t: None if t is None else t.cuda()
+    tag = "bf16" if dtype == torch.bfloat16 else "fp16"
+    for c in range(n_chunks):
+        sl = slice(c * C, (c + 1) * C)
+        cache.before_update(c)
+        o, lse = cache.attend(dev(q[:, sl].contiguous()), dev(k[:, sl].contiguous()),
+                              dev(v[:, sl].contiguous()), scale=scale, norm_scope=norm, eps=eps,
+                              gamma_q=dev(gq), gamma_k=dev(gk), rope_style=style,
+                              angles_q=dev(ang[sl].contiguous()) if style else None,
+                              angles_k=dev(ang[sl].contiguous()) if style else None)
+        torch.cuda.synchronize()
+        cache.after_update(c)
+        qn = _round16(qp.qk_prologue(f64(q[:, sl]), f64(gq), eps, norm,
+                                     None if ang is None else f64(ang[sl]), style), dtype)
+        idx = rc.visible_tokens(c, C, sink, window)
+        rows = sample_rows
+        o_ref, lse_ref = oracle.attention_fwd(qn, kn[:, idx], vn[:, idx], scale, oracle.MASK_NONE, 0,
+                                              rows=rows)
+        o_cpu, lse_cpu = o.cpu(), lse.cpu()
+        if rows is not None:
+            o_cpu, lse_cpu = o_cpu[:, rows], lse_cpu[:, :, rows]
+        _check(o_cpu, lse_cpu, o_ref, lse_ref, tag, what=f"chunk {c}", output_ulp=sample_rows is None)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+def test_fill_then_evict_with_sink_norm_and_rope(dtype):
+    """Chunk 64, one sink chunk, a three-chunk window: chunks 0-3 fill the
+    cache, chunks 4-6 evict the oldest window chunk each."""
+    _stream(2, 64, 64, 192, 4, 2, 128, 7, dtype, qp.NORM_HEAD, qp.ROPE_SPLIT, seed=1)
+
+
+def test_sliding_window_without_sink_interleaved_inner_norm():
+    _stream(1, 128, 0, 256, 4, 4, 64, 5, torch.bfloat16, qp.NORM_INNER, qp.ROPE_INTERLEAVED, seed=2)
+
+
+def test_ragged_chunk_no_prologue():
+    """A chunk length that is not a multiple of the 128-row tiles."""
+    _stream(1, 100, 100, 300, 2, 1, 128, 6, torch.bfloat16, qp.NORM_NONE, qp.ROPE_NONE, seed=3)
+
+
+def test_dit_stream_full_size_through_eviction():
+    """1785-token chunks of the DiT video stream, 40 query heads over 8 K/V
+    heads, a four-chunk window (7140 keys at steady state), head RMSNorm and
+    split-half RoPE: five chunks, the fifth evicting the first; 64 sampled
+    rows per chunk against the oracle."""
+    rows = np.sort(np.random.default_rng(7).choice(1785, size=64, replace=False))
+    _stream(1, 1785, 0, 7140, 40, 8, 128, 5, torch.bfloat16, qp.NORM_HEAD, qp.ROPE_SPLIT, seed=4,
+            sample_rows=rows)
