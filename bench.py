@@ -72,6 +72,9 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="minimum CPU time spent timing the oracle sample")
     ap.add_argument("--op", default="attention", choices=["attention", "prologue"])
+    ap.add_argument("--splitkv", type=int, default=None,
+                    help="time attn_fwd_splitkv with this many key ranges (0: chosen by the "
+                         "library) instead of attn_fwd")
     return ap.parse_args()
 
 
@@ -447,8 +450,22 @@ def main():
     lse = torch.empty((w.B, w.Hq, w.Lq), dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
 
-    def step():
-        hasb.attn_fwd(q, k, v, scale=w.scale, causal=w.mask, kv_offset=w.kv_offset, out=o, lse=lse)
+    split_used = None
+    if args.splitkv is None:
+        def step():
+            hasb.attn_fwd(q, k, v, scale=w.scale, causal=w.mask, kv_offset=w.kv_offset, out=o, lse=lse)
+    else:
+        tiles = (w.Lk + 127) // 128
+        cap = args.splitkv if args.splitkv > 0 else min(tiles, 32)
+        ws = torch.empty(max(1, hasb.splitkv_workspace_bytes(w.B, w.Lq, w.Hq, w.d, cap) // 4),
+                         dtype=torch.float32, device="cuda")
+        _, _, split_used = hasb.attn_fwd_splitkv(q, k, v, n_splits=args.splitkv, scale=w.scale,
+                                                 causal=w.mask, kv_offset=w.kv_offset, workspace=ws,
+                                                 out=o, lse=lse)
+
+        def step():
+            hasb.attn_fwd_splitkv(q, k, v, n_splits=args.splitkv, scale=w.scale, causal=w.mask,
+                                  kv_offset=w.kv_offset, workspace=ws, out=o, lse=lse)
 
     # ---- kernel-only timed region (inputs resident in HBM)
     for _ in range(max(3, args.warmup)):
@@ -526,6 +543,8 @@ def main():
     launch_avg = statistics.mean(launch_ms)
     achieved = w.flops() / (launch_avg * 1e-3) / 1e12
     traffic, traffic_src = profiled_traffic()
+    if split_used is not None:
+        traffic, traffic_src = None, "key-split path: no ncu summary of this kernel pair"
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": traffic,
                 "peak_source": f"bf16_tflops (burst) of {peak_src}",
@@ -544,10 +563,14 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": w.dtype, "data": "synthetic: seeded N(0,1) inputs of the workload's shape",
-            "config": workload_config(w, world),
+            "config": dict(workload_config(w, world),
+                           **({} if split_used is None else
+                              {"splitkv": split_used,
+                               "step": "attn_fwd_splitkv: split forward + merge, both timed"})),
             "pct_of_peak": 100.0 * value / world / peak,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": args.steps, "clocks": clock_info, "device_fault_bits": fault,
+            "gpu_launches": args.steps * (1 if split_used in (None, 1) else 2),
+            "clocks": clock_info, "device_fault_bits": fault,
         }
         print(json.dumps(line))
     if world > 1:

@@ -49,6 +49,10 @@ _SIGNATURES = {
                            [ctypes.c_int, ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
     "attn_fwd_cache": (ctypes.c_int, [ctypes.c_void_p] * 5 + [ctypes.c_int] * 7 +
                        [ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
+    "attn_splitkv_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int] * 5),
+    "attn_fwd_splitkv": (ctypes.c_int, [ctypes.c_void_p] * 6 + [ctypes.c_size_t] + [ctypes.c_int] * 7 +
+                         [ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                          ctypes.POINTER(ctypes.c_int), ctypes.c_void_p]),
     "attn_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "attn_device_fault": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint), ctypes.c_int]),
     "attn_set_wait_timeout_ns": (ctypes.c_int, [ctypes.c_ulonglong]),
@@ -266,6 +270,51 @@ def attn_fwd_cache(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor
     if st != ATTN_OK:
         raise AttnError(st, "attn_fwd_cache")
     return out, lse
+
+
+def splitkv_workspace_bytes(B: int, Lq: int, Hq: int, d: int, n_splits: int) -> int:
+    """Bytes of the float32 workspace attn_fwd_splitkv needs for n_splits ranges."""
+    return int(lib().attn_splitkv_workspace_bytes(B, Lq, Hq, d, n_splits))
+
+
+def attn_fwd_splitkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, n_splits: int = 0,
+                     scale: float | None = None, causal: int = MASK_NONE, kv_offset: int = 0,
+                     workspace: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                     lse: torch.Tensor | None = None, return_lse: bool = True, stream=None):
+    """Key-split attention forward through ``attn_fwd_splitkv`` of the C ABI
+    (masks 0 and 2). ``workspace`` (float32, CUDA) is allocated here when not
+    given, sized for the split count the library chooses. Returns
+    ``(out, lse, splits_used)``.
+    """
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_cuda or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError(f"{name} must be a contiguous 4-D CUDA tensor")
+    if q.dtype not in DTYPE_CODES or k.dtype != q.dtype or v.dtype != q.dtype or k.shape != v.shape:
+        raise ValueError("q, k, v must share one dtype (bf16/fp16); k and v one shape")
+    B, Lq, Hq, d = q.shape
+    Lk, Hkv = k.shape[1], k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
+    used = ctypes.c_int(0)
+    args = (B, Lq, Lk, Hq, Hkv, d, float(scale), int(causal), int(kv_offset), DTYPE_CODES[q.dtype])
+    if workspace is None:
+        # the largest split count the library could choose: one per 128-key tile, at most 32
+        tiles = (Lk + 127) // 128
+        cap = n_splits if n_splits > 0 else min(tiles, 32)
+        workspace = torch.empty(max(1, splitkv_workspace_bytes(B, Lq, Hq, d, max(1, cap)) // 4),
+                                dtype=torch.float32, device=q.device)
+    elif not workspace.is_cuda or workspace.dtype != torch.float32 or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous float32 CUDA tensor")
+    st = lib().attn_fwd_splitkv(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(workspace),
+                                workspace.numel() * 4, int(n_splits), *args[:9], args[9],
+                                ctypes.byref(used), _stream_handle(stream, q.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fwd_splitkv")
+    return out, lse, used.value
 
 
 def attn_fwd_host(q_host, k_host, v_host, o_host, lse_host, q_dev, k_dev, v_dev, o_dev, lse_dev, *,

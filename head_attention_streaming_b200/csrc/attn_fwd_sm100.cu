@@ -141,13 +141,20 @@ struct FwdParams {
   int B, Lq, Lk, Hq, Hkv, group, kv_offset;
   int kv_limit;      // keys visible to every row (masks 0 and 2): Lk or kv_offset + Lq
   int n_pairs;       // ceil(Lq / 256)
-  int n_units;       // B * Hq * n_pairs
+  int n_units;       // B * Hq * n_pairs * n_splits
   float sl2;         // scale * log2(e)
   unsigned long long timeout_ns;
+  // key split (masks 0 and 2 only): unit s of a query pair covers KV tiles
+  // s * split_tiles .. (s + 1) * split_tiles - 1 and writes float32 O / l and
+  // LSE of its keys to o_part [n_splits, B, Hq, Lq, d], lse_part [n_splits, B, Hq, Lq]
+  int n_splits, split_tiles;
+  float* o_part;
+  float* lse_part;
 };
 
 struct Unit {
   int b, hq, hkv, r0, n0, n1;  // n_t: KV tiles visited by query tile t
+  int j0, split;               // first KV tile, key split index
 };
 
 __device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
@@ -158,6 +165,8 @@ __device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
 template <bool CAUSAL>
 __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
   Unit x;
+  x.split = u % p.n_splits;
+  u /= p.n_splits;
   int pt = u % p.n_pairs;
   int t = u / p.n_pairs;
   int g = t % p.group;
@@ -170,8 +179,11 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
   if (CAUSAL) {
     x.n0 = cdiv(min(p.Lk, p.kv_offset + x.r0 + kTileRows), kTileRows);
     x.n1 = cdiv(min(p.Lk, p.kv_offset + x.r0 + 2 * kTileRows), kTileRows);
+    x.j0 = 0;
   } else {
-    x.n0 = x.n1 = cdiv(p.kv_limit, kTileRows);
+    const int total = cdiv(p.kv_limit, kTileRows);
+    x.j0 = x.split * p.split_tiles;
+    x.n0 = x.n1 = min(total, x.j0 + p.split_tiles) - x.j0;  // >= 1: the host never makes an empty split
   }
   return x;
 }
@@ -290,7 +302,7 @@ __device__ __forceinline__ void load_role(const CUtensorMap* tm_q, const CUtenso
 #pragma unroll
         for (int c = 0; c < C::kChunks; ++c)
           tma_load_4d(sKV + slot * C::kTileBytes + c * C::kChunkBytes, kv ? tm_v : tm_k, bf,
-                      c * 64, x.hkv, j * kTileRows, x.b, pol_kv);
+                      c * 64, x.hkv, (x.j0 + j) * kTileRows, x.b, pol_kv);
         ++kv_it;
       }
     }
@@ -465,7 +477,7 @@ __device__ __forceinline__ void store_role(const CUtensorMap* tm_o, const FwdPar
   bulk_wait_group0();  // every store complete before the CTA exits
 }
 
-template <int D, bool BF16, bool CAUSAL>
+template <int D, bool BF16, bool CAUSAL, bool SPLIT>
 __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, uint32_t tmem,
                                              uint32_t bars, uint32_t sstg, volatile int* abort_flag) {
   using C = Cfg<D>;
@@ -507,7 +519,7 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
       for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(tS + 32 * c, r + 32 * c);
       tmem_wait_ld_x128(r);
 
-      const int lim = row_lim - j * kTileRows;  // keys c < lim of this tile are visible
+      const int lim = row_lim - (x.j0 + j) * kTileRows;  // keys c < lim of this tile are visible
       const bool partial = lim < kTileRows;
       if (partial) {
 #pragma unroll
@@ -592,6 +604,36 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
       l += (sum[0] + sum[1]) + (sum[2] + sum[3]);
     }
 
+    if constexpr (SPLIT) {
+      // key split: float32 O / l of this split's keys, each thread its own
+      // row (d contiguous floats), straight from registers; LSE of the split
+      bool ok = mbar_wait(bar_o, ocnt & 1, abort_flag, kFaultSoftmaxOFull, p.timeout_ns);
+      if (!__all_sync(0xffffffffu, ok)) return;
+      ++ocnt;
+      tc_fence_after_sync();
+      const float inv_l = 1.f / l;
+      const bool in_range = row < p.Lq;
+      const size_t prow = ((static_cast<size_t>(x.split) * p.B + x.b) * p.Hq + x.hq) * p.Lq + row;
+      float* dst = p.o_part + prow * D;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t ov[32];
+        tmem_ld_32x32b_x32(tO + 32 * c, ov);
+        tmem_wait_ld_x32(ov);
+        if (in_range) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(dst + 32 * c + e) =
+                make_float4(__uint_as_float(ov[e]) * inv_l, __uint_as_float(ov[e + 1]) * inv_l,
+                            __uint_as_float(ov[e + 2]) * inv_l, __uint_as_float(ov[e + 3]) * inv_l);
+        }
+      }
+      if (in_range) p.lse_part[prow] = (ref + log2f(l)) * kLn2;
+      // every TMEM read of O_t is complete (wait::ld) before the next unit's
+      // P V overwrites it: that MMA waits for this warpgroup's next P
+      continue;
+    }
+
     // epilogue: O / l to 16 bits into the shared staging tile (128-byte
     // swizzle, the layout of the TMA box), handed to the store warp; LSE.
     // The staging buffer alternates between the two query tiles: tile t fills
@@ -632,7 +674,7 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
   }
 }
 
-template <int D, bool BF16, bool CAUSAL>
+template <int D, bool BF16, bool CAUSAL, bool SPLIT>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
@@ -698,14 +740,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < 8) {
     regs_increase<kRegsSoftmax>();
-    softmax_role<D, BF16, CAUSAL>(warp / 4, p, tmem, bars, sStg, abort_flag);
+    softmax_role<D, BF16, CAUSAL, SPLIT>(warp / 4, p, tmem, bars, sStg, abort_flag);
   } else {
     regs_decrease<kRegsProducer>();
     if (warp == 8) {
       if (lane == 0) load_role<D, BF16, CAUSAL>(&tm_q, &tm_k, &tm_v, p, sQ, sKV, bars, abort_flag);
     } else if (warp == 9 || warp == 10) {
       if (lane == 0) mma_role<D, BF16, CAUSAL>(warp - 9, p, tmem, sQ, sKV, bars, abort_flag);
-    } else {
+    } else if (!SPLIT) {
       if (lane == 0) store_role<D, BF16, CAUSAL>(&tm_o, p, sStg, bars, abort_flag);
     }
   }
@@ -716,6 +758,53 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after_sync();
     tmem_dealloc(tmem, C::kTmemCols);
   }
+}
+
+// ------------------------------------------------------------- key-split merge
+
+// Combines the key splits of attn_fwd_splitkv: for output row (b, i, hq),
+// lse = ln sum_g exp(lse_g) and O = sum_g exp(lse_g - lse) O_g (attention over
+// disjoint key ranges regrouped: the softmax of the developer guide's "Multi
+// Head Attention Definition" with its normaliser summed part by part). One warp
+// per output row; lane l holds d / 32 consecutive features. Reads
+// n_splits * (d + 1) floats and writes d 16-bit values per row: HBM-bound.
+template <int D, bool BF16>
+__global__ void __launch_bounds__(256) split_merge_kernel(const float* __restrict__ o_part,
+                                                          const float* __restrict__ lse_part, void* o,
+                                                          float* lse, int n_splits, int B, int Lq,
+                                                          int Hq) {
+  constexpr int kPer = D / 32;
+  const long long w = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) / 32;
+  const int lane = threadIdx.x % 32;
+  const long long rows = 1LL * B * Hq * Lq;
+  if (w >= rows) return;
+  // w = (b * Hq + hq) * Lq + i: the row index of the partial buffers
+  const int i = static_cast<int>(w % Lq);
+  const long long bh = w / Lq;
+  const int hq = static_cast<int>(bh % Hq);
+  const int b = static_cast<int>(bh / Hq);
+  const size_t split_rows = static_cast<size_t>(rows);
+  float m = -INFINITY;
+  for (int g = 0; g < n_splits; ++g) m = fmaxf(m, lse_part[g * split_rows + w]);
+  float acc[kPer];
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
+  float tot = 0.f;
+  for (int g = 0; g < n_splits; ++g) {
+    const float wg = expf(lse_part[g * split_rows + w] - m);
+    tot += wg;
+    const float* src = o_part + (g * split_rows + w) * D + lane * kPer;
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) acc[e] = fmaf(wg, src[e], acc[e]);
+  }
+  const float inv = 1.f / tot;
+  uint16_t* out = static_cast<uint16_t*>(o) + ((static_cast<size_t>(b) * Lq + i) * Hq + hq) * D + lane * kPer;
+#pragma unroll
+  for (int e = 0; e < kPer; e += 2) {
+    const uint32_t pk = pack2<BF16>(acc[e] * inv, acc[e + 1] * inv);
+    *reinterpret_cast<uint32_t*>(out + e) = pk;
+  }
+  if (lse != nullptr && lane == 0) lse[w] = m + logf(tot);
 }
 
 // ------------------------------------------------------------- diagnostics
@@ -908,7 +997,7 @@ bool encode_bl_hd(CUtensorMap* map, const void* ptr, int B, int L, int H, int d,
   return r == CUDA_SUCCESS;
 }
 
-template <int D, bool BF16, bool CAUSAL>
+template <int D, bool BF16, bool CAUSAL, bool SPLIT = false>
 int launch_fwd(const FwdParams& p, const void* q, const void* k, const void* v, int kv_rows, int grid,
                cudaStream_t stream) {
   using C = Cfg<D>;
@@ -918,7 +1007,7 @@ int launch_fwd(const FwdParams& p, const void* q, const void* k, const void* v, 
       !encode_bl_hd(&tv, v, p.B, p.Lk, p.Hkv, D, BF16, kv_rows) ||
       !encode_bl_hd(&to, p.o, p.B, p.Lq, p.Hq, D, BF16))
     return ATTN_ERR_CUDA;
-  auto kern = attn_fwd_sm100_kernel<D, BF16, CAUSAL>;
+  auto kern = attn_fwd_sm100_kernel<D, BF16, CAUSAL, SPLIT>;
   static std::once_flag attr_flags[kMaxDevices];
   static int attr_status[kMaxDevices];
   int dev = 0;
@@ -1046,6 +1135,10 @@ int attn_fwd_impl(const void* q, const void* k, const void* v, void* o, float* l
   p.n_units = static_cast<int>(n_units);
   p.sl2 = scale * kLog2e;
   p.timeout_ns = g_timeout_ns.load();
+  p.n_splits = 1;
+  p.split_tiles = (p.kv_limit + kTileRows - 1) / kTileRows;
+  p.o_part = nullptr;
+  p.lse_part = nullptr;
   const int grid = static_cast<int>(n_units < di.num_sms ? n_units : di.num_sms);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool bf16 = dtype == ATTN_DTYPE_BF16;
@@ -1056,6 +1149,34 @@ int attn_fwd_impl(const void* q, const void* k, const void* v, void* o, float* l
   }
   if (bf16) return cz ? launch_fwd<64, true, true>(p, q, k, v, kv_rows, grid, s) : launch_fwd<64, true, false>(p, q, k, v, kv_rows, grid, s);
   return cz ? launch_fwd<64, false, true>(p, q, k, v, kv_rows, grid, s) : launch_fwd<64, false, false>(p, q, k, v, kv_rows, grid, s);
+}
+
+// Key splits for attn_fwd_splitkv: `requested` (0 = choose) split count, the
+// KV tile count of the visible range, and the base unit count; returns the
+// split count actually used and the tiles per split (no split is empty).
+void choose_splits(int requested, int total_tiles, long long base_units, int num_sms, int* n_splits,
+                   int* split_tiles) {
+  long long want = requested;
+  if (want <= 0) {
+    // fewest waves per unit of work: ceil(units * n / SMs) / n, with 2 % per
+    // extra split for the partial outputs and the merge
+    double best = 1e300;
+    want = 1;
+    const int cap = total_tiles < 32 ? total_tiles : 32;
+    for (int n = 1; n <= cap; ++n) {
+      const long long waves = (base_units * n + num_sms - 1) / num_sms;
+      const double cost = static_cast<double>(waves) / n * (1.0 + 0.02 * (n - 1));
+      if (cost < best - 1e-12) {
+        best = cost;
+        want = n;
+      }
+    }
+  }
+  if (want > total_tiles) want = total_tiles;
+  if (want < 1) want = 1;
+  const int per = static_cast<int>((total_tiles + want - 1) / want);
+  *split_tiles = per;
+  *n_splits = (total_tiles + per - 1) / per;
 }
 
 }  // namespace hasb
@@ -1075,6 +1196,83 @@ int attn_fwd_cache(const void* q, const void* k_cache, const void* v_cache, void
   if (S < 1) return ATTN_ERR_INVALID_ARG;
   return attn_fwd_impl(q, k_cache, v_cache, o, lse, B, Lq, Lk, S, Hq, Hkv, d, scale, causal,
                        kv_offset, dtype, stream);
+}
+
+size_t attn_splitkv_workspace_bytes(int B, int Lq, int Hq, int d, int n_splits) {
+  if (B < 1 || Lq < 1 || Hq < 1 || d < 1 || n_splits < 1) return 0;
+  return static_cast<size_t>(n_splits) * B * Hq * Lq * (static_cast<size_t>(d) + 1) * sizeof(float);
+}
+
+int attn_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse,
+                     float* workspace, size_t workspace_bytes, int n_splits, int B, int Lq, int Lk,
+                     int Hq, int Hkv, int d, float scale, int causal, int kv_offset, int dtype,
+                     int* splits_used, void* stream) {
+  const int valid = attn_fwd_validate(q, k, v, o, lse, B, Lq, Lk, Hq, Hkv, d, scale, causal,
+                                      kv_offset, dtype, Lk);
+  if (valid != ATTN_OK) return valid;
+  if (causal == ATTN_MASK_CAUSAL || n_splits < 0) return ATTN_ERR_INVALID_ARG;
+  if (workspace != nullptr && (reinterpret_cast<uintptr_t>(workspace) & 15u) != 0)
+    return ATTN_ERR_INVALID_ARG;
+  const long long n_pairs = (Lq + 2LL * kTileRows - 1) / (2LL * kTileRows);
+  const long long base_units = n_pairs * B * Hq;
+  const int kv_limit = (causal == ATTN_MASK_CHUNK) ? kv_offset + Lq : Lk;
+  const int total_tiles = (kv_limit + kTileRows - 1) / kTileRows;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+  const DeviceInfo di = device_info(dev);
+  if (!di.ok) return ATTN_ERR_CUDA;
+  if (!di.sm100) return ATTN_ERR_UNSUPPORTED;
+  int ns = 1, per = total_tiles;
+  choose_splits(n_splits, total_tiles, base_units, di.num_sms, &ns, &per);
+  if (splits_used != nullptr) *splits_used = ns;
+  if (ns == 1)
+    return attn_fwd(q, k, v, o, lse, B, Lq, Lk, Hq, Hkv, d, scale, causal, kv_offset, dtype, stream);
+  const size_t need = attn_splitkv_workspace_bytes(B, Lq, Hq, d, ns);
+  if (workspace == nullptr || workspace_bytes < need) return ATTN_ERR_INVALID_ARG;
+  const size_t o_elems = static_cast<size_t>(ns) * B * Hq * Lq * d;
+  if (ranges_overlap(workspace, need, q, 2ull * B * Lq * Hq * d) ||
+      ranges_overlap(workspace, need, k, 2ull * B * Lk * Hkv * d) ||
+      ranges_overlap(workspace, need, v, 2ull * B * Lk * Hkv * d) ||
+      ranges_overlap(workspace, need, o, 2ull * B * Lq * Hq * d) ||
+      (lse != nullptr && ranges_overlap(workspace, need, lse, 4ull * B * Hq * Lq)))
+    return ATTN_ERR_INVALID_ARG;
+  if (base_units * ns > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+
+  FwdParams p;
+  p.o = o;
+  p.lse = lse;
+  p.B = B; p.Lq = Lq; p.Lk = Lk; p.Hq = Hq; p.Hkv = Hkv; p.group = Hq / Hkv;
+  p.kv_offset = kv_offset;
+  p.kv_limit = kv_limit;
+  p.n_pairs = static_cast<int>(n_pairs);
+  p.n_units = static_cast<int>(base_units * ns);
+  p.sl2 = scale * kLog2e;
+  p.timeout_ns = g_timeout_ns.load();
+  p.n_splits = ns;
+  p.split_tiles = per;
+  p.o_part = workspace;
+  p.lse_part = workspace + o_elems;
+  const int grid = static_cast<int>(p.n_units < di.num_sms ? p.n_units : di.num_sms);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool bf16 = dtype == ATTN_DTYPE_BF16;
+  int st;
+  if (d == 128)
+    st = bf16 ? launch_fwd<128, true, false, true>(p, q, k, v, Lk, grid, s)
+              : launch_fwd<128, false, false, true>(p, q, k, v, Lk, grid, s);
+  else
+    st = bf16 ? launch_fwd<64, true, false, true>(p, q, k, v, Lk, grid, s)
+              : launch_fwd<64, false, false, true>(p, q, k, v, Lk, grid, s);
+  if (st != ATTN_OK) return st;
+  const long long rows = 1LL * B * Hq * Lq;
+  const unsigned mgrid = static_cast<unsigned>((rows * 32 + 255) / 256);
+  if (d == 128) {
+    if (bf16) split_merge_kernel<128, true><<<mgrid, 256, 0, s>>>(p.o_part, p.lse_part, o, lse, ns, B, Lq, Hq);
+    else split_merge_kernel<128, false><<<mgrid, 256, 0, s>>>(p.o_part, p.lse_part, o, lse, ns, B, Lq, Hq);
+  } else {
+    if (bf16) split_merge_kernel<64, true><<<mgrid, 256, 0, s>>>(p.o_part, p.lse_part, o, lse, ns, B, Lq, Hq);
+    else split_merge_kernel<64, false><<<mgrid, 256, 0, s>>>(p.o_part, p.lse_part, o, lse, ns, B, Lq, Hq);
+  }
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 int attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, void* o_host,

@@ -73,6 +73,11 @@ WORKLOADS = {
                  MASK_CHUNK, 5355, 1.0 / math.sqrt(128), seed=4),
         Workload("video_20480x56x128", 1, 20480, 20480, 56, 56, 128, "bf16", MASK_NONE, 0,
                  1.0 / math.sqrt(128), seed=5, sample_rows=256),
+        # a short streaming chunk (256 tokens) against the same 7140-key cache:
+        # one 256-row query pair per head, 40 work units for 148 SMs unless the
+        # keys are split (attn_fwd_splitkv)
+        Workload("stream_chunk_256_vs_7140_gqa40x8", 1, 256, 7140, 40, 8, 128, "bf16",
+                 MASK_CHUNK, 6884, 1.0 / math.sqrt(128), seed=6),
     ]
 }
 

@@ -20,6 +20,8 @@
 #ifndef HEAD_ATTENTION_STREAMING_B200_ATTN_H_
 #define HEAD_ATTENTION_STREAMING_B200_ATTN_H_
 
+#include <stddef.h>
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -89,6 +91,37 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
 int attn_fwd_cache(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
                    int B, int Lq, int Lk, int S, int Hq, int Hkv, int d, float scale, int causal,
                    int kv_offset, int dtype, void* stream);
+
+/*
+ * attn_fwd_splitkv — attn_fwd with the visible keys of every query tile split
+ * into ranges that different CTAs process at once, then merged: for few query
+ * rows over many keys (a short chunk against a long cache), where one CTA per
+ * 256-row query pair would leave most SMs idle.
+ *
+ * Operation: attention over disjoint key ranges, combined exactly through the
+ * per-range log-sum-exp: lse = ln sum_g exp(lse_g), O = sum_g exp(lse_g - lse)
+ * O_g (the softmax of the developer guide's "Multi Head Attention Definition"
+ * with its normaliser summed range by range). Masks 0 and 2 only (every row
+ * sees the same key range); causal returns ATTN_ERR_INVALID_ARG.
+ *
+ * Arguments as attn_fwd, plus:
+ *   n_splits   requested number of key ranges, >= 1, or 0 to choose one from
+ *              the shape and the SM count; clipped to the number of 128-key
+ *              tiles, never an empty range
+ *   workspace  device float32 buffer of at least
+ *              attn_splitkv_workspace_bytes(B, Lq, Hq, d, n) bytes for the n
+ *              ranges used (partial O and LSE), 16-byte aligned, overlapping no
+ *              operand; may be NULL when no split happens (n = 1)
+ *   splits_used  if not NULL, receives n (written before any launch)
+ * With n = 1 the call is attn_fwd. Two launches otherwise (the split forward,
+ * then the merge), asynchronous on `stream`. The workspace is the caller's and
+ * must not be reused before the call's work on `stream` has completed.
+ */
+size_t attn_splitkv_workspace_bytes(int B, int Lq, int Hq, int d, int n_splits);
+int attn_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse,
+                     float* workspace, size_t workspace_bytes, int n_splits, int B, int Lq, int Lk,
+                     int Hq, int Hkv, int d, float scale, int causal, int kv_offset, int dtype,
+                     int* splits_used, void* stream);
 
 /*
  * attn_fwd_host — the same forward for operands in host memory: copies q, k, v

@@ -26,7 +26,7 @@ A = 0x10000  # 16-byte aligned fake addresses: never dereferenced (calls fail va
 def _declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"^\s*(?:int|const char\*)\s+(attn_\w+)\s*\(", text, flags=re.M)))
+    return sorted(set(re.findall(r"^\s*(?:int|const char\*|size_t)\s+(attn_\w+)\s*\(", text, flags=re.M)))
 
 
 def test_header_declares_the_entry_points():
@@ -150,3 +150,17 @@ def test_prologue_python_binding_rejects_cpu_tensors():
     q = torch.zeros(1, 4, 2, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         hasb.qk_prologue(q)
+
+
+def test_splitkv_argument_contract_before_any_cuda_call():
+    L = hasb.lib()
+    base = [A, A + 0x100000, A + 0x200000, A + 0x300000, None, A + 0x400000, 1 << 20]
+    tail = [1, 64, 512, 2, 1, 128, 0.1]
+    # causal is refused; a negative split count is refused; a misaligned workspace is refused
+    assert L.attn_fwd_splitkv(*base, 0, *tail, 1, 0, 0, None, None) == hasb.ATTN_ERR_INVALID_ARG
+    assert L.attn_fwd_splitkv(*base, -1, *tail, 0, 0, 0, None, None) == hasb.ATTN_ERR_INVALID_ARG
+    bad = list(base)
+    bad[5] = A + 0x400000 + 4
+    assert L.attn_fwd_splitkv(*bad, 2, *tail, 0, 0, 0, None, None) == hasb.ATTN_ERR_INVALID_ARG
+    assert L.attn_splitkv_workspace_bytes(1, 64, 2, 128, 4) == 4 * 1 * 2 * 64 * 129 * 4
+    assert L.attn_splitkv_workspace_bytes(0, 64, 2, 128, 4) == 0
