@@ -1179,40 +1179,32 @@ void choose_splits(int requested, int total_tiles, long long base_units, int num
   *n_splits = (total_tiles + per - 1) / per;
 }
 
-}  // namespace hasb
 
-extern "C" {
+// Scratch of attn_fwd_splitkv_static: float32 partial outputs and LSEs of the
+// key ranges, in a file-scope device array (64 MB, reserved when the module is
+// loaded); that entry point allocates nothing. Calls that use it must not
+// overlap in time (one stream, or ordered by the caller).
+constexpr size_t kStaticScratchFloats = size_t(16) << 20;
+__device__ __align__(256) float g_split_scratch[kStaticScratchFloats];
 
-int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Lq,
-             int Lk, int Hq, int Hkv, int d, float scale, int causal, int kv_offset, int dtype,
-             void* stream) {
-  return attn_fwd_impl(q, k, v, o, lse, B, Lq, Lk, Lk, Hq, Hkv, d, scale, causal, kv_offset, dtype,
-                       stream);
-}
-
-int attn_fwd_cache(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
-                   int B, int Lq, int Lk, int S, int Hq, int Hkv, int d, float scale, int causal,
-                   int kv_offset, int dtype, void* stream) {
-  if (S < 1) return ATTN_ERR_INVALID_ARG;
-  return attn_fwd_impl(q, k_cache, v_cache, o, lse, B, Lq, Lk, S, Hq, Hkv, d, scale, causal,
-                       kv_offset, dtype, stream);
-}
-
-size_t attn_splitkv_workspace_bytes(int B, int Lq, int Hq, int d, int n_splits) {
-  if (B < 1 || Lq < 1 || Hq < 1 || d < 1 || n_splits < 1) return 0;
-  return static_cast<size_t>(n_splits) * B * Hq * Lq * (static_cast<size_t>(d) + 1) * sizeof(float);
-}
-
-int attn_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse,
-                     float* workspace, size_t workspace_bytes, int n_splits, int B, int Lq, int Lk,
-                     int Hq, int Hkv, int d, float scale, int causal, int kv_offset, int dtype,
-                     int* splits_used, void* stream) {
+// Argument contract of the key-split entry points (no CUDA call).
+int splitkv_validate(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                     int n_splits, int B, int Lq, int Lk, int Hq, int Hkv, int d, float scale,
+                     int causal, int kv_offset, int dtype) {
   const int valid = attn_fwd_validate(q, k, v, o, lse, B, Lq, Lk, Hq, Hkv, d, scale, causal,
                                       kv_offset, dtype, Lk);
   if (valid != ATTN_OK) return valid;
   if (causal == ATTN_MASK_CAUSAL || n_splits < 0) return ATTN_ERR_INVALID_ARG;
-  if (workspace != nullptr && (reinterpret_cast<uintptr_t>(workspace) & 15u) != 0)
-    return ATTN_ERR_INVALID_ARG;
+  return ATTN_OK;
+}
+
+// The key-split forward after validation. fit: lower the split count until the
+// partials fit the workspace (down to one range, i.e. plain attn_fwd) instead
+// of refusing a workspace that is too small.
+int splitkv_run(const void* q, const void* k, const void* v, void* o, float* lse, float* workspace,
+                size_t workspace_bytes, bool fit, int n_splits, int B, int Lq, int Lk, int Hq,
+                int Hkv, int d, float scale, int causal, int kv_offset, int dtype, int* splits_used,
+                void* stream) {
   const long long n_pairs = (Lq + 2LL * kTileRows - 1) / (2LL * kTileRows);
   const long long base_units = n_pairs * B * Hq;
   const int kv_limit = (causal == ATTN_MASK_CHUNK) ? kv_offset + Lq : Lk;
@@ -1224,6 +1216,12 @@ int attn_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float
   if (!di.sm100) return ATTN_ERR_UNSUPPORTED;
   int ns = 1, per = total_tiles;
   choose_splits(n_splits, total_tiles, base_units, di.num_sms, &ns, &per);
+  if (fit) {
+    while (ns > 1 && attn_splitkv_workspace_bytes(B, Lq, Hq, d, ns) > workspace_bytes) {
+      per = (total_tiles + ns - 2) / (ns - 1);
+      ns = (total_tiles + per - 1) / per;
+    }
+  }
   if (splits_used != nullptr) *splits_used = ns;
   if (ns == 1)
     return attn_fwd(q, k, v, o, lse, B, Lq, Lk, Hq, Hkv, d, scale, causal, kv_offset, dtype, stream);
@@ -1273,6 +1271,57 @@ int attn_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float
     else split_merge_kernel<64, false><<<mgrid, 256, 0, s>>>(p.o_part, p.lse_part, o, lse, ns, B, Lq, Hq);
   }
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+
+
+}  // namespace hasb
+
+extern "C" {
+
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Lq,
+             int Lk, int Hq, int Hkv, int d, float scale, int causal, int kv_offset, int dtype,
+             void* stream) {
+  return attn_fwd_impl(q, k, v, o, lse, B, Lq, Lk, Lk, Hq, Hkv, d, scale, causal, kv_offset, dtype,
+                       stream);
+}
+
+int attn_fwd_cache(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
+                   int B, int Lq, int Lk, int S, int Hq, int Hkv, int d, float scale, int causal,
+                   int kv_offset, int dtype, void* stream) {
+  if (S < 1) return ATTN_ERR_INVALID_ARG;
+  return attn_fwd_impl(q, k_cache, v_cache, o, lse, B, Lq, Lk, S, Hq, Hkv, d, scale, causal,
+                       kv_offset, dtype, stream);
+}
+
+size_t attn_splitkv_workspace_bytes(int B, int Lq, int Hq, int d, int n_splits) {
+  if (B < 1 || Lq < 1 || Hq < 1 || d < 1 || n_splits < 1) return 0;
+  return static_cast<size_t>(n_splits) * B * Hq * Lq * (static_cast<size_t>(d) + 1) * sizeof(float);
+}
+
+int attn_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse,
+                     float* workspace, size_t workspace_bytes, int n_splits, int B, int Lq, int Lk,
+                     int Hq, int Hkv, int d, float scale, int causal, int kv_offset, int dtype,
+                     int* splits_used, void* stream) {
+  const int valid = splitkv_validate(q, k, v, o, lse, n_splits, B, Lq, Lk, Hq, Hkv, d, scale, causal,
+                                     kv_offset, dtype);
+  if (valid != ATTN_OK) return valid;
+  if (workspace != nullptr && (reinterpret_cast<uintptr_t>(workspace) & 15u) != 0)
+    return ATTN_ERR_INVALID_ARG;
+  return splitkv_run(q, k, v, o, lse, workspace, workspace_bytes, false, n_splits, B, Lq, Lk, Hq, Hkv,
+                     d, scale, causal, kv_offset, dtype, splits_used, stream);
+}
+
+int attn_fwd_splitkv_static(const void* q, const void* k, const void* v, void* o, float* lse,
+                            int n_splits, int B, int Lq, int Lk, int Hq, int Hkv, int d, float scale,
+                            int causal, int kv_offset, int dtype, int* splits_used, void* stream) {
+  const int valid = splitkv_validate(q, k, v, o, lse, n_splits, B, Lq, Lk, Hq, Hkv, d, scale, causal,
+                                     kv_offset, dtype);
+  if (valid != ATTN_OK) return valid;
+  void* ws = nullptr;
+  if (cudaGetSymbolAddress(&ws, g_split_scratch) != cudaSuccess) return ATTN_ERR_CUDA;
+  return splitkv_run(q, k, v, o, lse, static_cast<float*>(ws), sizeof(g_split_scratch), true, n_splits,
+                     B, Lq, Lk, Hq, Hkv, d, scale, causal, kv_offset, dtype, splits_used, stream);
 }
 
 int attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, void* o_host,

@@ -124,6 +124,19 @@ int attn_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float
                      int* splits_used, void* stream);
 
 /*
+ * attn_fwd_splitkv_static — attn_fwd_splitkv without a workspace argument: the
+ * partial outputs live in a 64 MB scratch array inside the library (device
+ * memory reserved when the library is loaded), so the call allocates nothing.
+ * If the chosen or requested split count needs more scratch, the count is
+ * lowered until it fits (down to one range, i.e. attn_fwd); *splits_used
+ * reports it. Calls must not overlap in time (one stream, or ordered by the
+ * caller): they share the scratch. Arguments and errors as attn_fwd_splitkv.
+ */
+int attn_fwd_splitkv_static(const void* q, const void* k, const void* v, void* o, float* lse,
+                            int n_splits, int B, int Lq, int Lk, int Hq, int Hkv, int d, float scale,
+                            int causal, int kv_offset, int dtype, int* splits_used, void* stream);
+
+/*
  * attn_fwd_host — the same forward for operands in host memory: copies q, k, v
  * from host to the caller's device buffers, runs attn_fwd, and copies o (and
  * lse when both lse pointers are given) back to host memory, all queued on
