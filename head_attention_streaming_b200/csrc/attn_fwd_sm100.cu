@@ -162,11 +162,15 @@ __device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
 // Work unit u -> (b, hq, row pair). Query heads of one GQA group are adjacent
 // and the row pairs of one head are adjacent, so CTAs running together read
 // the same K/V head (L2 reuse). Causal units run longest first.
-template <bool CAUSAL>
+template <bool CAUSAL, bool SPLIT>
 __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
   Unit x;
-  x.split = u % p.n_splits;
-  u /= p.n_splits;
+  if constexpr (SPLIT) {
+    x.split = u % p.n_splits;
+    u /= p.n_splits;
+  } else {
+    x.split = 0;
+  }
   int pt = u % p.n_pairs;
   int t = u / p.n_pairs;
   int g = t % p.group;
@@ -180,10 +184,13 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
     x.n0 = cdiv(min(p.Lk, p.kv_offset + x.r0 + kTileRows), kTileRows);
     x.n1 = cdiv(min(p.Lk, p.kv_offset + x.r0 + 2 * kTileRows), kTileRows);
     x.j0 = 0;
-  } else {
+  } else if constexpr (SPLIT) {
     const int total = cdiv(p.kv_limit, kTileRows);
     x.j0 = x.split * p.split_tiles;
     x.n0 = x.n1 = min(total, x.j0 + p.split_tiles) - x.j0;  // >= 1: the host never makes an empty split
+  } else {
+    x.j0 = 0;
+    x.n0 = x.n1 = cdiv(p.kv_limit, kTileRows);
   }
   return x;
 }
@@ -263,7 +270,7 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint3
   issue_pv_half<D, BF16, 1>(d_tmem, p_tmem, v_lo, 1u);
 }
 
-template <int D, bool BF16, bool CAUSAL>
+template <int D, bool BF16, bool CAUSAL, bool SPLIT>
 __device__ __forceinline__ void load_role(const CUtensorMap* tm_q, const CUtensorMap* tm_k,
                                           const CUtensorMap* tm_v, const FwdParams& p,
                                           uint32_t sQ, uint32_t sKV, uint32_t bars,
@@ -274,7 +281,7 @@ __device__ __forceinline__ void load_role(const CUtensorMap* tm_q, const CUtenso
   int kv_it = 0, uit = 0;
   bool aborted = false;
   for (int u = blockIdx.x; u < p.n_units && !aborted; u += gridDim.x, ++uit) {
-    const Unit x = decode_unit<CAUSAL>(p, u);
+    const Unit x = decode_unit<CAUSAL, SPLIT>(p, u);
     for (int t = 0; t < 2; ++t) {
       const uint32_t bq = bars + 8 * (kBarQEmpty + t);
       if (!mbar_wait(bq, (uit & 1) ^ 1, abort_flag, kFaultLoadQEmpty, p.timeout_ns)) {
@@ -323,7 +330,7 @@ __device__ __forceinline__ void load_role(const CUtensorMap* tm_q, const CUtenso
 // issuing the other's GEMMs. With one thread per tile, the tensor core runs
 // whichever tile has work. Both threads read the same K/V ring slots; each slot
 // use is released by both (kv_empty takes two arrivals).
-template <int D, bool BF16, bool CAUSAL>
+template <int D, bool BF16, bool CAUSAL, bool SPLIT>
 __device__ __forceinline__ void mma_role(const int t, const FwdParams& p, uint32_t tmem, uint32_t sQ,
                                          uint32_t sKV, uint32_t bars, volatile int* abort_flag) {
   using C = Cfg<D>;
@@ -344,7 +351,7 @@ __device__ __forceinline__ void mma_role(const int t, const FwdParams& p, uint32
   int kv_it = 0, uit = 0, pcnt = 0;
   bool ok = true;
   for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++uit) {
-    const Unit x = decode_unit<CAUSAL>(p, u);
+    const Unit x = decode_unit<CAUSAL, SPLIT>(p, u);
     const int n = t ? x.n1 : x.n0;  // KV tiles this query tile uses (n0 <= n1)
     ok = mbar_wait(bar(kBarQFull + t), uit & 1, abort_flag, kFaultMmaQFull, p.timeout_ns) &&
          kv_full(kv_it);
@@ -454,14 +461,14 @@ __device__ __forceinline__ void exp_tile(const uint32_t (&r)[128], float sl2, fl
 // buffer to global memory with a TMA store (rows past Lq are clipped by the
 // tensor map), then hands the buffer to the other query tile. Order per unit:
 // tile 0, then tile 1, the same order the softmax warpgroups fill it in.
-template <int D, bool BF16, bool CAUSAL>
+template <int D, bool BF16, bool CAUSAL, bool SPLIT>
 __device__ __forceinline__ void store_role(const CUtensorMap* tm_o, const FwdParams& p, uint32_t sStg,
                                            uint32_t bars, volatile int* abort_flag) {
   using C = Cfg<D>;
   int scnt = 0;
   bool ok = true;
   for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-    const Unit x = decode_unit<CAUSAL>(p, u);
+    const Unit x = decode_unit<CAUSAL, SPLIT>(p, u);
     for (int t = 0; t < 2 && ok; ++t) {
       ok = mbar_wait(bars + 8 * kBarStgFull, scnt & 1, abort_flag, kFaultStore, p.timeout_ns);
       if (!ok) break;
@@ -501,7 +508,7 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
   int scnt = 0, ocnt = 0;
 
   for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
-    const Unit x = decode_unit<CAUSAL>(p, u);
+    const Unit x = decode_unit<CAUSAL, SPLIT>(p, u);
     const int n = t ? x.n1 : x.n0;
     const int row = x.r0 + t * kTileRows + r_in;
     const int row_lim = CAUSAL ? min(p.Lk, p.kv_offset + row + 1) : p.kv_limit;
@@ -744,11 +751,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     regs_decrease<kRegsProducer>();
     if (warp == 8) {
-      if (lane == 0) load_role<D, BF16, CAUSAL>(&tm_q, &tm_k, &tm_v, p, sQ, sKV, bars, abort_flag);
+      if (lane == 0) load_role<D, BF16, CAUSAL, SPLIT>(&tm_q, &tm_k, &tm_v, p, sQ, sKV, bars, abort_flag);
     } else if (warp == 9 || warp == 10) {
-      if (lane == 0) mma_role<D, BF16, CAUSAL>(warp - 9, p, tmem, sQ, sKV, bars, abort_flag);
+      if (lane == 0) mma_role<D, BF16, CAUSAL, SPLIT>(warp - 9, p, tmem, sQ, sKV, bars, abort_flag);
     } else if (!SPLIT) {
-      if (lane == 0) store_role<D, BF16, CAUSAL>(&tm_o, p, sStg, bars, abort_flag);
+      if (lane == 0) store_role<D, BF16, CAUSAL, SPLIT>(&tm_o, p, sStg, bars, abort_flag);
     }
   }
   __syncwarp();
