@@ -238,6 +238,53 @@ def select_workload(args):
     return w
 
 
+class Ranks:
+    """One process per GPU under torchrun (RANK, WORLD_SIZE, LOCAL_RANK from the
+    environment, rendezvous at MASTER_ADDR/MASTER_PORT). Every rank runs its own
+    instance of the workload (weak scaling); the process group carries only the
+    timing reduction. NCCL on GPUs; the tests drive the same code with gloo."""
+
+    def __init__(self, backend: str = "nccl"):
+        import torch.distributed as dist
+        self.dist = dist
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+        self.backend = backend
+        if self.world > 1:
+            import datetime
+            import torch
+            kw = {"device_id": torch.device("cuda", self.local_rank)} if backend == "nccl" else {}
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
+
+    def barrier(self):
+        if self.world > 1:
+            self.dist.barrier()
+
+    def max(self, x: float, device) -> float:
+        """The largest x over all ranks (every rank gets it)."""
+        if self.world == 1:
+            return float(x)
+        import torch
+        t = torch.tensor([float(x)], device=device)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.world > 1:
+            self.dist.destroy_process_group()
+
+
+def rank_seed(base: int, rank: int) -> int:
+    """Seed of a rank's own problem instance (distinct per rank)."""
+    return base + 7919 * rank
+
+
+def job_rate(world: int, work_per_rank: float, ms_per_step: float) -> float:
+    """Whole-job throughput: the work of all ranks over the slowest rank's step time."""
+    return world * work_per_rank / (ms_per_step * 1e-3)
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -275,21 +322,16 @@ def run_prologue(args):
     """Time attn_qk_prologue on Q and K of the 1785-token DiT workload (rank 0 of
     each replica; weak scaling like the attention bench)."""
     import torch
-    import torch.distributed as dist
 
     import head_attention_streaming_b200 as hasb
     from head_attention_streaming_b200 import inputs
 
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local_rank)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local_rank))
+    ranks = Ranks("nccl")
+    rank, world = ranks.rank, ranks.world
     B, L, H, d, pos0, eps = 1, 1785, 40, 128, 5355, 1e-6
-    g = torch.Generator().manual_seed(31 + 7919 * rank)
+    g = torch.Generator().manual_seed(rank_seed(31, rank))
     q_cpu = torch.randn(B, L, H, d, generator=g).to(torch.bfloat16)
     k_cpu = torch.randn(B, L, H, d, generator=g).to(torch.bfloat16)
     gq_cpu = 1.0 + 0.1 * torch.randn(d, generator=g)
@@ -306,9 +348,7 @@ def run_prologue(args):
         hasb.qk_prologue(q, k, norm_scope=hasb.NORM_HEAD, eps=eps, gamma_q=gq, gamma_k=gk,
                          rope_style=hasb.ROPE_SPLIT, angles_q=ang, angles_k=ang, out_q=oq, out_k=ok)
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
+    barrier = ranks.barrier
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -330,12 +370,8 @@ def run_prologue(args):
     torch.cuda.synchronize()
     clock_info = clocks.stop()
     launch_ms = [a.elapsed_time(b) for a, b in ev]
-    ms_step = statistics.mean(launch_ms)
-    if world > 1:
-        t = torch.tensor([ms_step], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step = float(t.item())
-    value = world * algo_bytes / (ms_step * 1e-3) / 1e9
+    ms_step = ranks.max(statistics.mean(launch_ms), "cuda")
+    value = job_rate(world, algo_bytes, ms_step) / 1e9
 
     # end to end: pinned host Q, K in, prologue, Q, K out, every step
     qh, kh = q_cpu.pin_memory(), k_cpu.pin_memory()
@@ -357,12 +393,8 @@ def run_prologue(args):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e_ms = e0.elapsed_time(e1) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e_ms = float(t.item())
-    e2e = {"value": world * algo_bytes / (e_ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": e_ms,
+    e_ms = ranks.max(e0.elapsed_time(e1) / e2e_steps, "cuda")
+    e2e = {"value": job_rate(world, algo_bytes, e_ms) / 1e9, "unit": "GB/s", "ms_per_step": e_ms,
            "h2d_bytes_per_step": tensor_bytes, "d2h_bytes_per_step": tensor_bytes,
            "path": "pinned host Q, K -> device, attn_qk_prologue, Q, K -> host, one stream"}
 
@@ -411,8 +443,7 @@ def run_prologue(args):
             "clocks": clock_info, "device_fault_bits": hasb.device_fault(clear=True),
         }
         print(json.dumps(line))
-    if world > 1:
-        dist.destroy_process_group()
+    ranks.close()
     return 0
 
 
@@ -424,27 +455,19 @@ def main():
         return run_reference(args)
 
     import torch
-    import torch.distributed as dist
 
     import head_attention_streaming_b200 as hasb
     from head_attention_streaming_b200 import inputs
 
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local_rank)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local_rank))
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
+    ranks = Ranks("nccl")
+    rank, world = ranks.rank, ranks.world
+    barrier = ranks.barrier
 
     w = select_workload(args)
     q_cpu, k_cpu, v_cpu = inputs.make_qkv(w.B, w.Lq, w.Lk, w.Hq, w.Hkv, w.d, w.torch_dtype,
-                                          seed=w.seed + 7919 * rank, qk_rmsnorm=w.qk_rmsnorm)
+                                          seed=rank_seed(w.seed, rank), qk_rmsnorm=w.qk_rmsnorm)
     q, k, v = q_cpu.cuda(), k_cpu.cuda(), v_cpu.cuda()
     o = torch.empty_like(q)
     lse = torch.empty((w.B, w.Hq, w.Lq), dtype=torch.float32, device="cuda")
@@ -495,12 +518,8 @@ def main():
     fault = hasb.device_fault(clear=True)
     ms_total = t_start.elapsed_time(t_end)
     launch_ms = [a.elapsed_time(b) for a, b in ev]
-    ms_step = statistics.mean(launch_ms) if flush else ms_total / args.steps
-    if world > 1:
-        t = torch.tensor([ms_step], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step = float(t.item())
-    value = world * w.flops() / (ms_step * 1e-3) / 1e12
+    ms_step = ranks.max(statistics.mean(launch_ms) if flush else ms_total / args.steps, "cuda")
+    value = job_rate(world, w.flops(), ms_step) / 1e12
 
     # ---- end to end through the host-buffer C ABI entry point
     e2e = None
@@ -526,14 +545,10 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize()
         barrier()
-        e_ms = e0.elapsed_time(e1) / args.e2e_steps
-        if world > 1:
-            t = torch.tensor([e_ms], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms = ranks.max(e0.elapsed_time(e1) / args.e2e_steps, "cuda")
         h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
         d2h = oh.numel() * oh.element_size() + lh.numel() * lh.element_size()
-        e2e = {"value": world * w.flops() / (e_ms * 1e-3) / 1e12, "unit": "TFLOPS",
+        e2e = {"value": job_rate(world, w.flops(), e_ms) / 1e12, "unit": "TFLOPS",
                "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "path": "attn_fwd_host (pinned host -> device, forward, device -> host), one stream"}
 
@@ -573,8 +588,7 @@ def main():
             "clocks": clock_info, "device_fault_bits": fault,
         }
         print(json.dumps(line))
-    if world > 1:
-        dist.destroy_process_group()
+    ranks.close()
     return 0
 
 
