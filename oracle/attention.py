@@ -60,6 +60,7 @@ import numpy as np
 MASK_NONE = 0
 MASK_CAUSAL = 1
 MASK_CHUNK = 2
+MASK_WINDOW = 3
 
 
 def kv_head(hq: int, Hq: int, Hkv: int) -> int:
@@ -90,8 +91,26 @@ def visible_limit(mask: int, i: int, Lq: int, Lk: int, kv_offset: int) -> int:
     raise ValueError(f"unknown mask mode {mask}")
 
 
+def visible_range(mask: int, i: int, Lq: int, Lk: int, kv_offset: int, window=(-1, -1)):
+    """Visible keys of query row ``i`` as a half-open range ``[lo, hi)``.
+
+    Modes 0-2: ``[0, visible_limit(...))``. Mode 3 (sliding window, skill page
+    "optimizing-attention-flash", "Sliding window attention": flash-attn's
+    ``window_size=(left, right)``, -1 for no limit on that side): with the row's
+    position ``p = kv_offset + i`` in key coordinates, keys
+    ``p - left <= j <= p + right`` are visible.
+    """
+    if mask != MASK_WINDOW:
+        return 0, visible_limit(mask, i, Lq, Lk, kv_offset)
+    left, right = window
+    p = kv_offset + i
+    lo = 0 if left < 0 else max(0, p - left)
+    hi = Lk if right < 0 else min(Lk, p + right + 1)
+    return lo, hi
+
+
 def attention_fwd(q, k, v, scale: float, mask: int = MASK_NONE, kv_offset: int = 0,
-                  rows=None, return_weights: bool = False):
+                  rows=None, return_weights: bool = False, window=(-1, -1)):
     """Scaled dot-product attention forward in float64.
 
     developer guide, "Multi Head Attention Definition" (per-head SDPA equation);
@@ -101,8 +120,10 @@ def attention_fwd(q, k, v, scale: float, mask: int = MASK_NONE, kv_offset: int =
       q: ``[B, Lq, Hq, d]`` array (any real dtype; widened to float64).
       k, v: ``[B, Lk, Hkv, d]``.
       scale: multiplier of the dot products (1/sqrt(d) in the pages).
-      mask: 0 none, 1 causal, 2 streaming chunk (see ``visible_limit``).
-      kv_offset: cache position of query row 0 (masks 1 and 2).
+      mask: 0 none, 1 causal, 2 streaming chunk, 3 sliding window (see
+        ``visible_limit`` and ``visible_range``).
+      kv_offset: cache position of query row 0 (masks 1, 2 and 3).
+      window: ``(left, right)`` of mask 3.
       rows: optional 1-D sequence of query rows to compute (all rows if None).
       return_weights: also return the softmax weights ``[B, Hq, R, Lk]`` (zero
         at invisible keys); meant for tiny inputs.
@@ -128,8 +149,9 @@ def attention_fwd(q, k, v, scale: float, mask: int = MASK_NONE, kv_offset: int =
     lse = np.zeros((B, Hq, R), dtype=np.float64)
     weights = np.zeros((B, Hq, R, Lk), dtype=np.float64) if return_weights else None
 
-    limits = np.array([visible_limit(mask, int(i), Lq, Lk, kv_offset) for i in rows],
-                      dtype=np.int64)
+    ranges = [visible_range(mask, int(i), Lq, Lk, kv_offset, window) for i in rows]
+    if any(hi <= lo for lo, hi in ranges):
+        raise ValueError("every query row must see at least one key")
     for b in range(B):
         for hq in range(Hq):
             hkv = kv_head(hq, Hq, Hkv)
@@ -137,17 +159,17 @@ def attention_fwd(q, k, v, scale: float, mask: int = MASK_NONE, kv_offset: int =
             V = v[b, :, hkv, :]
             Q = q[b, rows, hq, :]
             scores = scale * (Q @ K.T)  # [R, Lk]
-            # rows that share one visible prefix are handled together
-            for lim in np.unique(limits):
-                sel = np.nonzero(limits == lim)[0]
-                s = scores[sel, :lim]                       # visible keys only
+            # rows that share one visible key range are handled together
+            for lo, hi in sorted(set(ranges)):
+                sel = np.array([n for n, r in enumerate(ranges) if r == (lo, hi)], dtype=np.int64)
+                s = scores[sel, lo:hi]                      # visible keys only
                 m = s.max(axis=1, keepdims=True)            # pass 1: row max
                 e = np.exp(s - m)                           # pass 2: weights
                 l = e.sum(axis=1, keepdims=True)
-                o[b, sel, hq, :] = (e @ V[:lim]) / l
+                o[b, sel, hq, :] = (e @ V[lo:hi]) / l
                 lse[b, hq, sel] = m[:, 0] + np.log(l[:, 0])
                 if return_weights:
-                    weights[b, hq, sel, :lim] = e / l
+                    weights[b, hq, sel, lo:hi] = e / l
     if return_weights:
         return o, lse, weights
     return o, lse
@@ -162,3 +184,9 @@ def flops(B: int, Lq: int, Lk: int, Hq: int, d: int, mask: int) -> float:
     """
     f = 4.0 * B * Hq * Lq * Lk * d
     return f / 2.0 if mask == MASK_CAUSAL else f
+
+
+def visible_pairs(Lq: int, Lk: int, mask: int, kv_offset: int = 0, window=(-1, -1)) -> int:
+    """Number of visible (query row, key) pairs of one (batch, head)."""
+    return sum(hi - lo for lo, hi in (visible_range(mask, i, Lq, Lk, kv_offset, window)
+                                      for i in range(Lq)))
