@@ -56,6 +56,9 @@ _SIGNATURES = {
     "attn_fwd_splitkv_static": (ctypes.c_int, [ctypes.c_void_p] * 5 + [ctypes.c_int] * 7 +
                                 [ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                  ctypes.POINTER(ctypes.c_int), ctypes.c_void_p]),
+    "attn_fwd_window": (ctypes.c_int, [ctypes.c_void_p] * 5 + [ctypes.c_int] * 6 +
+                        [ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                         ctypes.c_void_p]),
     "attn_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "attn_device_fault": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint), ctypes.c_int]),
     "attn_set_wait_timeout_ns": (ctypes.c_int, [ctypes.c_ulonglong]),
@@ -348,6 +351,34 @@ def attn_fwd_splitkv_static(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *
     if st != ATTN_OK:
         raise AttnError(st, "attn_fwd_splitkv_static")
     return out, lse, used.value
+
+
+def attn_fwd_window(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, window=(-1, -1),
+                    scale: float | None = None, kv_offset: int = 0, out: torch.Tensor | None = None,
+                    lse: torch.Tensor | None = None, return_lse: bool = True, stream=None):
+    """Sliding-window attention through ``attn_fwd_window`` of the C ABI: row i
+    (key position kv_offset + i) sees keys within ``window = (left, right)`` of
+    it, -1 = unbounded on that side. Returns ``(out, lse)``."""
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_cuda or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError(f"{name} must be a contiguous 4-D CUDA tensor")
+    if q.dtype not in DTYPE_CODES or k.dtype != q.dtype or v.dtype != q.dtype or k.shape != v.shape:
+        raise ValueError("q, k, v must share one dtype (bf16/fp16); k and v one shape")
+    B, Lq, Hq, d = q.shape
+    Lk, Hkv = k.shape[1], k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
+    left, right = window
+    st = lib().attn_fwd_window(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Lq, Lk, Hq, Hkv, d,
+                               float(scale), int(left), int(right), int(kv_offset), DTYPE_CODES[q.dtype],
+                               _stream_handle(stream, q.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fwd_window")
+    return out, lse
 
 
 def attn_fwd_host(q_host, k_host, v_host, o_host, lse_host, q_dev, k_dev, v_dev, o_dev, lse_dev, *,

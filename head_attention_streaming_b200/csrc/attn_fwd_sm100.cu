@@ -150,11 +150,18 @@ struct FwdParams {
   int n_splits, split_tiles;
   float* o_part;
   float* lse_part;
+  // sliding window (left, right; -1 = unbounded): row i sees keys
+  // p - left <= j <= p + right, p = kv_offset + i
+  int win_left, win_right;
 };
 
+// KV tiles of a work unit: the loader streams tiles j0 .. j0 + nu - 1 (the
+// union of both query tiles' ranges); query tile t uses n_t of them, starting
+// s_t tiles in. Without a window both ranges start at j0 and n0 <= n1 = nu.
 struct Unit {
-  int b, hq, hkv, r0, n0, n1;  // n_t: KV tiles visited by query tile t
-  int j0, split;               // first KV tile, key split index
+  int b, hq, hkv, r0, n0, n1;
+  int j0, split;  // first KV tile, key split index
+  int s0, s1, nu;
 };
 
 __device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
@@ -162,7 +169,7 @@ __device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
 // Work unit u -> (b, hq, row pair). Query heads of one GQA group are adjacent
 // and the row pairs of one head are adjacent, so CTAs running together read
 // the same K/V head (L2 reuse). Causal units run longest first.
-template <bool CAUSAL, bool SPLIT>
+template <bool CAUSAL, bool SPLIT, bool WINDOW>
 __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
   Unit x;
   if constexpr (SPLIT) {
@@ -180,6 +187,26 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
   x.hq = x.hkv * p.group + g;
   if (CAUSAL) pt = p.n_pairs - 1 - pt;
   x.r0 = pt * 2 * kTileRows;
+  x.s0 = x.s1 = 0;
+  if constexpr (WINDOW) {
+    // key range of each query tile from its first and last real rows
+    int a[2], e[2];
+    for (int t = 0; t < 2; ++t) {
+      const int first = min(x.r0 + t * kTileRows, p.Lq - 1);
+      const int last = min(x.r0 + t * kTileRows + kTileRows - 1, p.Lq - 1);
+      const int lo = p.win_left < 0 ? 0 : max(0, p.kv_offset + first - p.win_left);
+      const int hi = p.win_right < 0 ? p.Lk : min(p.Lk, p.kv_offset + last + p.win_right + 1);
+      a[t] = lo / kTileRows;
+      e[t] = cdiv(hi, kTileRows);
+    }
+    x.j0 = a[0];  // a[0] <= a[1] and e[0] <= e[1]: tile 1's rows come later
+    x.s0 = 0;
+    x.s1 = a[1] - a[0];
+    x.n0 = e[0] - a[0];
+    x.n1 = e[1] - a[1];
+    x.nu = e[1] - a[0];
+    return x;
+  }
   if (CAUSAL) {
     x.n0 = cdiv(min(p.Lk, p.kv_offset + x.r0 + kTileRows), kTileRows);
     x.n1 = cdiv(min(p.Lk, p.kv_offset + x.r0 + 2 * kTileRows), kTileRows);
@@ -192,6 +219,7 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
     x.j0 = 0;
     x.n0 = x.n1 = cdiv(p.kv_limit, kTileRows);
   }
+  x.nu = x.n1;
   return x;
 }
 
@@ -270,7 +298,7 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint3
   issue_pv_half<D, BF16, 1>(d_tmem, p_tmem, v_lo, 1u);
 }
 
-template <int D, bool BF16, bool CAUSAL, bool SPLIT>
+template <int D, bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW>
 __device__ __forceinline__ void load_role(const CUtensorMap* tm_q, const CUtensorMap* tm_k,
                                           const CUtensorMap* tm_v, const FwdParams& p,
                                           uint32_t sQ, uint32_t sKV, uint32_t bars,
@@ -281,7 +309,7 @@ __device__ __forceinline__ void load_role(const CUtensorMap* tm_q, const CUtenso
   int kv_it = 0, uit = 0;
   bool aborted = false;
   for (int u = blockIdx.x; u < p.n_units && !aborted; u += gridDim.x, ++uit) {
-    const Unit x = decode_unit<CAUSAL, SPLIT>(p, u);
+    const Unit x = decode_unit<CAUSAL, SPLIT, WINDOW>(p, u);
     for (int t = 0; t < 2; ++t) {
       const uint32_t bq = bars + 8 * (kBarQEmpty + t);
       if (!mbar_wait(bq, (uit & 1) ^ 1, abort_flag, kFaultLoadQEmpty, p.timeout_ns)) {
@@ -295,7 +323,7 @@ __device__ __forceinline__ void load_role(const CUtensorMap* tm_q, const CUtenso
         tma_load_4d(sQ + t * C::kTileBytes + c * C::kChunkBytes, tm_q, bf, c * 64, x.hq,
                     x.r0 + t * kTileRows, x.b, pol_q);
     }
-    for (int j = 0; j < x.n1 && !aborted; ++j) {
+    for (int j = 0; j < x.nu && !aborted; ++j) {
       for (int kv = 0; kv < 2; ++kv) {
         const int slot = kv_it % C::kStages;
         const uint32_t be = bars + 8 * (kBarKvEmpty + slot);
@@ -330,7 +358,7 @@ __device__ __forceinline__ void load_role(const CUtensorMap* tm_q, const CUtenso
 // issuing the other's GEMMs. With one thread per tile, the tensor core runs
 // whichever tile has work. Both threads read the same K/V ring slots; each slot
 // use is released by both (kv_empty takes two arrivals).
-template <int D, bool BF16, bool CAUSAL, bool SPLIT>
+template <int D, bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW>
 __device__ __forceinline__ void mma_role(const int t, const FwdParams& p, uint32_t tmem, uint32_t sQ,
                                          uint32_t sKV, uint32_t bars, volatile int* abort_flag) {
   using C = Cfg<D>;
@@ -351,18 +379,29 @@ __device__ __forceinline__ void mma_role(const int t, const FwdParams& p, uint32
   int kv_it = 0, uit = 0, pcnt = 0;
   bool ok = true;
   for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++uit) {
-    const Unit x = decode_unit<CAUSAL, SPLIT>(p, u);
-    const int n = t ? x.n1 : x.n0;  // KV tiles this query tile uses (n0 <= n1)
-    ok = mbar_wait(bar(kBarQFull + t), uit & 1, abort_flag, kFaultMmaQFull, p.timeout_ns) &&
-         kv_full(kv_it);
+    const Unit x = decode_unit<CAUSAL, SPLIT, WINDOW>(p, u);
+    const int n = t ? x.n1 : x.n0;  // KV tiles this query tile uses
+    const int s = t ? x.s1 : x.s0;  // ... starting this many tiles into the unit's stream
+    ok = mbar_wait(bar(kBarQFull + t), uit & 1, abort_flag, kFaultMmaQFull, p.timeout_ns);
+    // window: tiles before this query tile's range pass through the ring;
+    // release this thread's share once each has landed
+    for (int j = 0; j < s && ok; ++j) {
+      for (int kv = 0; kv < 2 && ok; ++kv) {
+        const int idx = kv_it + 2 * j + kv;
+        if (!kv_full(idx)) { ok = false; break; }
+        mbar_arrive(bar(kBarKvEmpty + idx % C::kStages));
+      }
+    }
+    const int kb = kv_it + 2 * s;  // ring index of this query tile's first K
+    ok = ok && kv_full(kb);
     if (!ok) break;
     // S_t(0) = Q_t K_0^T
-    issue_qk<D, BF16>(s_t, q_lo, k_lo(kv_it));
+    issue_qk<D, BF16>(s_t, q_lo, k_lo(kb));
     mma_commit(bar(kBarSFull + t));
-    mma_commit(bar(kBarKvEmpty + kv_it % C::kStages));
+    mma_commit(bar(kBarKvEmpty + kb % C::kStages));
     if (n == 1) mma_commit(bar(kBarQEmpty + t));
     for (int j = 0; j < n; ++j) {
-      const int vidx = kv_it + 2 * j + 1;  // V_j
+      const int vidx = kb + 2 * j + 1;  // V_j
       const int knext = vidx + 1;          // K_{j+1}
       // O_t += P_t V_j: the first 64 keys as soon as their half of P is in
       // tensor memory, the rest once all of P is
@@ -391,17 +430,17 @@ __device__ __forceinline__ void mma_role(const int t, const FwdParams& p, uint32
         if (j + 1 == n - 1) mma_commit(bar(kBarQEmpty + t));
       }
     }
-    // causal: tiles this query tile never sees (n <= j < n1) still pass through
+    // causal / window: tiles after this query tile's range still pass through
     // the ring; release this thread's share once each has landed (waiting for
     // the landing keeps the arrival in the slot's current phase)
-    for (int j = n; j < x.n1 && ok; ++j) {
+    for (int j = s + n; j < x.nu && ok; ++j) {
       for (int kv = 0; kv < 2 && ok; ++kv) {
         const int idx = kv_it + 2 * j + kv;
         if (!kv_full(idx)) { ok = false; break; }
         mbar_arrive(bar(kBarKvEmpty + idx % C::kStages));
       }
     }
-    kv_it += 2 * x.n1;
+    kv_it += 2 * x.nu;
   }
   if (!ok) {
     // every MMA this thread issued must finish before tensor memory is freed
@@ -419,7 +458,7 @@ __device__ __forceinline__ void mma_role(const int t, const FwdParams& p, uint32
 // exponential (their -inf scores times a zero scale, or -inf + inf when the
 // row has no visible key yet, would give NaN).
 template <bool BF16, bool MASKED>
-__device__ __forceinline__ void exp_tile(const uint32_t (&r)[128], float sl2, float nref, int lim,
+__device__ __forceinline__ void exp_tile(const uint32_t (&r)[128], float sl2, float nref, int lim, int lim_lo,
                                          float (&sum)[4], uint32_t tS, uint32_t bar_half,
                                          uint32_t bar_full, uint32_t bar_turn_other, bool hand_over,
                                          int lane) {
@@ -438,8 +477,8 @@ __device__ __forceinline__ void exp_tile(const uint32_t (&r)[128], float sl2, fl
         p1 = ex2_approx(fmaf(__uint_as_float(r[c + 1]), sl2, nref));
       }
       if (MASKED) {
-        p0 = c < lim ? p0 : 0.f;
-        p1 = c + 1 < lim ? p1 : 0.f;
+        p0 = (c < lim && c >= lim_lo) ? p0 : 0.f;
+        p1 = (c + 1 < lim && c + 1 >= lim_lo) ? p1 : 0.f;
       }
       sum[(2 * cc) & 3] += p0;
       sum[(2 * cc + 1) & 3] += p1;
@@ -461,14 +500,14 @@ __device__ __forceinline__ void exp_tile(const uint32_t (&r)[128], float sl2, fl
 // buffer to global memory with a TMA store (rows past Lq are clipped by the
 // tensor map), then hands the buffer to the other query tile. Order per unit:
 // tile 0, then tile 1, the same order the softmax warpgroups fill it in.
-template <int D, bool BF16, bool CAUSAL, bool SPLIT>
+template <int D, bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW>
 __device__ __forceinline__ void store_role(const CUtensorMap* tm_o, const FwdParams& p, uint32_t sStg,
                                            uint32_t bars, volatile int* abort_flag) {
   using C = Cfg<D>;
   int scnt = 0;
   bool ok = true;
   for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-    const Unit x = decode_unit<CAUSAL, SPLIT>(p, u);
+    const Unit x = decode_unit<CAUSAL, SPLIT, WINDOW>(p, u);
     for (int t = 0; t < 2 && ok; ++t) {
       ok = mbar_wait(bars + 8 * kBarStgFull, scnt & 1, abort_flag, kFaultStore, p.timeout_ns);
       if (!ok) break;
@@ -484,7 +523,7 @@ __device__ __forceinline__ void store_role(const CUtensorMap* tm_o, const FwdPar
   bulk_wait_group0();  // every store complete before the CTA exits
 }
 
-template <int D, bool BF16, bool CAUSAL, bool SPLIT>
+template <int D, bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW>
 __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, uint32_t tmem,
                                              uint32_t bars, uint32_t sstg, volatile int* abort_flag) {
   using C = Cfg<D>;
@@ -508,10 +547,18 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
   int scnt = 0, ocnt = 0;
 
   for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
-    const Unit x = decode_unit<CAUSAL, SPLIT>(p, u);
+    const Unit x = decode_unit<CAUSAL, SPLIT, WINDOW>(p, u);
     const int n = t ? x.n1 : x.n0;
+    const int s = t ? x.s1 : x.s0;  // first KV tile of this query tile, relative to x.j0
     const int row = x.r0 + t * kTileRows + r_in;
-    const int row_lim = CAUSAL ? min(p.Lk, p.kv_offset + row + 1) : p.kv_limit;
+    // visible keys of this row: [row_lo, row_lim)
+    int row_lim = CAUSAL ? min(p.Lk, p.kv_offset + row + 1) : p.kv_limit;
+    int row_lo = 0;
+    if constexpr (WINDOW) {
+      const int pos = p.kv_offset + row;
+      row_lo = p.win_left < 0 ? 0 : max(0, pos - p.win_left);
+      row_lim = p.win_right < 0 ? p.Lk : min(p.Lk, pos + p.win_right + 1);
+    }
     float ref = -INFINITY;  // scaled (log2) max the exponentials are taken against
     float l = 0.f;          // running row sum of exp2(s * sl2 - ref)
 
@@ -526,12 +573,14 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
       for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(tS + 32 * c, r + 32 * c);
       tmem_wait_ld_x128(r);
 
-      const int lim = row_lim - (x.j0 + j) * kTileRows;  // keys c < lim of this tile are visible
-      const bool partial = lim < kTileRows;
+      const int key0 = (x.j0 + s + j) * kTileRows;  // first key of this tile
+      const int lim = row_lim - key0;                // keys c < lim of this tile are visible ...
+      const int lim_lo = WINDOW ? row_lo - key0 : 0;  // ... and c >= lim_lo
+      const bool partial = lim < kTileRows || lim_lo > 0;
       if (partial) {
 #pragma unroll
         for (int c = 0; c < 128; ++c)
-          if (c >= lim) r[c] = __float_as_uint(-INFINITY);
+          if (c >= lim || c < lim_lo) r[c] = __float_as_uint(-INFINITY);
       }
       // row max: a three-input max tree (depth 5) over the 128 scores
       float m_tile;
@@ -586,17 +635,19 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
       // Ping-pong: the two softmax warpgroups take turns for their exponentials
       // (tile 0 of KV tile j, then tile 1 of j, then tile 0 of j + 1, ...), so
       // the MUFU serves one of them at a time and each tile's GEMMs run on the
-      // tensor core while the other tile computes. Waits and arrivals pair up:
-      // turn[1] gets one arrival per KV tile tile 0 processes (n0 per unit),
-      // turn[0] one per tile 1 processes below n0 - 1.
-      if (t == 0 ? j >= 1 : j < x.n0) {
+      // tensor core while the other tile computes. Step j of tile 0 hands over
+      // if tile 1 has a step j; step j of tile 1 hands over if tile 0 has a
+      // step j + 1; each waits exactly for the hand-overs it is owed, so
+      // arrivals and waits pair up per unit: min(n0, n1) on turn[1] and
+      // min(n0 - 1, n1) on turn[0] (n0 > n1 can happen with a window).
+      if (t == 0 ? (j >= 1 && j - 1 < x.n1) : j < x.n0) {
         bool ok_turn = mbar_wait(bar_turn_mine, tcnt & 1, abort_flag, kFaultSoftmaxTurn, p.timeout_ns);
         if (!__all_sync(0xffffffffu, ok_turn)) return;
         ++tcnt;
       }
 
       const float nref = -ref;
-      const bool hand_over = (t == 0 || j + 1 < x.n0);
+      const bool hand_over = t == 0 ? j < x.n1 : j + 1 < x.n0;
       float sum[4] = {0.f, 0.f, 0.f, 0.f};
       // the masked variant is a separate instantiation so full tiles carry no
       // per-score compare/select. exp_tile holds warp-collective instructions
@@ -604,9 +655,11 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
       // warp: rows of one warp can differ (causal), and a lane whose keys are
       // all visible is unaffected by the masked variant.
       if (__any_sync(0xffffffffu, partial)) {
-        exp_tile<BF16, true>(r, sl2, nref, lim, sum, tS, bar_ph, bar_p, bar_turn_other, hand_over, lane);
+        exp_tile<BF16, true>(r, sl2, nref, lim, lim_lo, sum, tS, bar_ph, bar_p, bar_turn_other, hand_over,
+                             lane);
       } else {
-        exp_tile<BF16, false>(r, sl2, nref, lim, sum, tS, bar_ph, bar_p, bar_turn_other, hand_over, lane);
+        exp_tile<BF16, false>(r, sl2, nref, lim, lim_lo, sum, tS, bar_ph, bar_p, bar_turn_other, hand_over,
+                              lane);
       }
       l += (sum[0] + sum[1]) + (sum[2] + sum[3]);
     }
@@ -681,7 +734,7 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
   }
 }
 
-template <int D, bool BF16, bool CAUSAL, bool SPLIT>
+template <int D, bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
@@ -747,15 +800,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < 8) {
     regs_increase<kRegsSoftmax>();
-    softmax_role<D, BF16, CAUSAL, SPLIT>(warp / 4, p, tmem, bars, sStg, abort_flag);
+    softmax_role<D, BF16, CAUSAL, SPLIT, WINDOW>(warp / 4, p, tmem, bars, sStg, abort_flag);
   } else {
     regs_decrease<kRegsProducer>();
     if (warp == 8) {
-      if (lane == 0) load_role<D, BF16, CAUSAL, SPLIT>(&tm_q, &tm_k, &tm_v, p, sQ, sKV, bars, abort_flag);
+      if (lane == 0) load_role<D, BF16, CAUSAL, SPLIT, WINDOW>(&tm_q, &tm_k, &tm_v, p, sQ, sKV, bars, abort_flag);
     } else if (warp == 9 || warp == 10) {
-      if (lane == 0) mma_role<D, BF16, CAUSAL, SPLIT>(warp - 9, p, tmem, sQ, sKV, bars, abort_flag);
+      if (lane == 0) mma_role<D, BF16, CAUSAL, SPLIT, WINDOW>(warp - 9, p, tmem, sQ, sKV, bars, abort_flag);
     } else if (!SPLIT) {
-      if (lane == 0) store_role<D, BF16, CAUSAL, SPLIT>(&tm_o, p, sStg, bars, abort_flag);
+      if (lane == 0) store_role<D, BF16, CAUSAL, SPLIT, WINDOW>(&tm_o, p, sStg, bars, abort_flag);
     }
   }
   __syncwarp();
@@ -1004,7 +1057,7 @@ bool encode_bl_hd(CUtensorMap* map, const void* ptr, int B, int L, int H, int d,
   return r == CUDA_SUCCESS;
 }
 
-template <int D, bool BF16, bool CAUSAL, bool SPLIT = false>
+template <int D, bool BF16, bool CAUSAL, bool SPLIT = false, bool WINDOW = false>
 int launch_fwd(const FwdParams& p, const void* q, const void* k, const void* v, int kv_rows, int grid,
                cudaStream_t stream) {
   using C = Cfg<D>;
@@ -1014,7 +1067,7 @@ int launch_fwd(const FwdParams& p, const void* q, const void* k, const void* v, 
       !encode_bl_hd(&tv, v, p.B, p.Lk, p.Hkv, D, BF16, kv_rows) ||
       !encode_bl_hd(&to, p.o, p.B, p.Lq, p.Hq, D, BF16))
     return ATTN_ERR_CUDA;
-  auto kern = attn_fwd_sm100_kernel<D, BF16, CAUSAL, SPLIT>;
+  auto kern = attn_fwd_sm100_kernel<D, BF16, CAUSAL, SPLIT, WINDOW>;
   static std::once_flag attr_flags[kMaxDevices];
   static int attr_status[kMaxDevices];
   int dev = 0;
@@ -1117,11 +1170,14 @@ int attn_fwd_validate(const void* q, const void* k, const void* v, const void* o
 // attn_fwd over K/V whose consecutive batches are kv_rows rows apart.
 int attn_fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Lq,
                   int Lk, int kv_rows, int Hq, int Hkv, int d, float scale, int causal, int kv_offset,
-                  int dtype, void* stream) {
-  // ---- argument contract (no CUDA call before it passes)
-  const int valid = attn_fwd_validate(q, k, v, o, lse, B, Lq, Lk, Hq, Hkv, d, scale, causal,
-                                      kv_offset, dtype, kv_rows);
+                  int dtype, void* stream, bool window = false, int win_left = -1,
+                  int win_right = -1) {
+  // ---- argument contract (no CUDA call before it passes); a window uses the
+  // offset rule of masks 1 and 2 (0 <= kv_offset, kv_offset + Lq <= Lk)
+  const int valid = attn_fwd_validate(q, k, v, o, lse, B, Lq, Lk, Hq, Hkv, d, scale,
+                                      window ? ATTN_MASK_CHUNK : causal, kv_offset, dtype, kv_rows);
   if (valid != ATTN_OK) return valid;
+  if (window && (win_left < -1 || win_right < -1)) return ATTN_ERR_INVALID_ARG;
   const long long n_pairs = (Lq + 2LL * kTileRows - 1) / (2LL * kTileRows);
   const long long n_units = n_pairs * B * Hq;
 
@@ -1146,9 +1202,19 @@ int attn_fwd_impl(const void* q, const void* k, const void* v, void* o, float* l
   p.split_tiles = (p.kv_limit + kTileRows - 1) / kTileRows;
   p.o_part = nullptr;
   p.lse_part = nullptr;
+  p.win_left = win_left;
+  p.win_right = win_right;
   const int grid = static_cast<int>(n_units < di.num_sms ? n_units : di.num_sms);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool bf16 = dtype == ATTN_DTYPE_BF16;
+  if (window) {
+    p.kv_limit = Lk;
+    if (d == 128)
+      return bf16 ? launch_fwd<128, true, false, false, true>(p, q, k, v, kv_rows, grid, s)
+                  : launch_fwd<128, false, false, false, true>(p, q, k, v, kv_rows, grid, s);
+    return bf16 ? launch_fwd<64, true, false, false, true>(p, q, k, v, kv_rows, grid, s)
+                : launch_fwd<64, false, false, false, true>(p, q, k, v, kv_rows, grid, s);
+  }
   const bool cz = causal == ATTN_MASK_CAUSAL;
   if (d == 128) {
     if (bf16) return cz ? launch_fwd<128, true, true>(p, q, k, v, kv_rows, grid, s) : launch_fwd<128, true, false>(p, q, k, v, kv_rows, grid, s);
@@ -1257,6 +1323,7 @@ int splitkv_run(const void* q, const void* k, const void* v, void* o, float* lse
   p.split_tiles = per;
   p.o_part = workspace;
   p.lse_part = workspace + o_elems;
+  p.win_left = p.win_right = -1;
   const int grid = static_cast<int>(p.n_units < di.num_sms ? p.n_units : di.num_sms);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool bf16 = dtype == ATTN_DTYPE_BF16;
@@ -1291,6 +1358,13 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
              void* stream) {
   return attn_fwd_impl(q, k, v, o, lse, B, Lq, Lk, Lk, Hq, Hkv, d, scale, causal, kv_offset, dtype,
                        stream);
+}
+
+int attn_fwd_window(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Lq,
+                    int Lk, int Hq, int Hkv, int d, float scale, int window_left, int window_right,
+                    int kv_offset, int dtype, void* stream) {
+  return attn_fwd_impl(q, k, v, o, lse, B, Lq, Lk, Lk, Hq, Hkv, d, scale, ATTN_MASK_NONE, kv_offset,
+                       dtype, stream, true, window_left, window_right);
 }
 
 int attn_fwd_cache(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,

@@ -83,6 +83,20 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
              int causal, int kv_offset, int dtype, void* stream);
 
 /*
+ * attn_fwd_window — attn_fwd with a sliding window (local attention): query
+ * row i, at key position p = kv_offset + i, sees keys p - window_left <= j <=
+ * p + window_right; -1 leaves that side unbounded (skill page
+ * "optimizing-attention-flash", "Sliding window attention": flash-attn's
+ * window_size=(left, right)). (-1, 0) is causal, (-1, -1) is no mask. KV tiles
+ * outside every row's window are neither loaded nor multiplied.
+ * Arguments as attn_fwd with 0 <= kv_offset, kv_offset + Lq <= Lk, and
+ * window_left, window_right >= -1 (so every row sees its own position).
+ */
+int attn_fwd_window(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Lq,
+                    int Lk, int Hq, int Hkv, int d, float scale, int window_left, int window_right,
+                    int kv_offset, int dtype, void* stream);
+
+/*
  * attn_fwd_cache — attn_fwd with K and V read from the first Lk tokens of a
  * [B, S, Hkv, d] cache (the rolling block cache of streaming self-attention,
  * whose valid tokens are a prefix of its S slots): batch b's keys start at

@@ -164,3 +164,12 @@ def test_splitkv_argument_contract_before_any_cuda_call():
     assert L.attn_fwd_splitkv(*bad, 2, *tail, 0, 0, 0, None, None) == hasb.ATTN_ERR_INVALID_ARG
     assert L.attn_splitkv_workspace_bytes(1, 64, 2, 128, 4) == 4 * 1 * 2 * 64 * 129 * 4
     assert L.attn_splitkv_workspace_bytes(0, 64, 2, 128, 4) == 0
+
+
+@pytest.mark.parametrize("kw", [dict(wl=-2), dict(wr=-3), dict(off=-1), dict(off=5), dict(Lq=0)])
+def test_window_argument_contract(kw):
+    a = dict(wl=4, wr=0, off=0, Lq=4)
+    a.update(kw)
+    st = hasb.lib().attn_fwd_window(A, A + 0x100000, A + 0x200000, A + 0x300000, None, 1, a["Lq"], 8, 2,
+                                    1, 128, 0.1, a["wl"], a["wr"], a["off"], 0, None)
+    assert st == hasb.ATTN_ERR_INVALID_ARG
