@@ -381,15 +381,17 @@ __device__ __forceinline__ void mma_role(const int t, const FwdParams& p, uint32
   for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++uit) {
     const Unit x = decode_unit<CAUSAL, SPLIT, WINDOW>(p, u);
     const int n = t ? x.n1 : x.n0;  // KV tiles this query tile uses
-    const int s = t ? x.s1 : x.s0;  // ... starting this many tiles into the unit's stream
+    const int s = WINDOW ? (t ? x.s1 : x.s0) : 0;  // ... starting this many tiles into the stream
     ok = mbar_wait(bar(kBarQFull + t), uit & 1, abort_flag, kFaultMmaQFull, p.timeout_ns);
-    // window: tiles before this query tile's range pass through the ring;
-    // release this thread's share once each has landed
-    for (int j = 0; j < s && ok; ++j) {
-      for (int kv = 0; kv < 2 && ok; ++kv) {
-        const int idx = kv_it + 2 * j + kv;
-        if (!kv_full(idx)) { ok = false; break; }
-        mbar_arrive(bar(kBarKvEmpty + idx % C::kStages));
+    if constexpr (WINDOW) {
+      // tiles before this query tile's range pass through the ring; release
+      // this thread's share once each has landed
+      for (int j = 0; j < s && ok; ++j) {
+        for (int kv = 0; kv < 2 && ok; ++kv) {
+          const int idx = kv_it + 2 * j + kv;
+          if (!kv_full(idx)) { ok = false; break; }
+          mbar_arrive(bar(kBarKvEmpty + idx % C::kStages));
+        }
       }
     }
     const int kb = kv_it + 2 * s;  // ring index of this query tile's first K
@@ -549,7 +551,7 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
   for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
     const Unit x = decode_unit<CAUSAL, SPLIT, WINDOW>(p, u);
     const int n = t ? x.n1 : x.n0;
-    const int s = t ? x.s1 : x.s0;  // first KV tile of this query tile, relative to x.j0
+    const int s = WINDOW ? (t ? x.s1 : x.s0) : 0;  // first KV tile of this query tile, relative to x.j0
     const int row = x.r0 + t * kTileRows + r_in;
     // visible keys of this row: [row_lo, row_lim)
     int row_lim = CAUSAL ? min(p.Lk, p.kv_offset + row + 1) : p.kv_limit;
@@ -640,14 +642,16 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
       // step j + 1; each waits exactly for the hand-overs it is owed, so
       // arrivals and waits pair up per unit: min(n0, n1) on turn[1] and
       // min(n0 - 1, n1) on turn[0] (n0 > n1 can happen with a window).
-      if (t == 0 ? (j >= 1 && j - 1 < x.n1) : j < x.n0) {
+      const bool wait_turn = WINDOW ? (t == 0 ? (j >= 1 && j - 1 < x.n1) : j < x.n0)
+                                    : (t == 0 ? j >= 1 : j < x.n0);  // n0 <= n1 without a window
+      if (wait_turn) {
         bool ok_turn = mbar_wait(bar_turn_mine, tcnt & 1, abort_flag, kFaultSoftmaxTurn, p.timeout_ns);
         if (!__all_sync(0xffffffffu, ok_turn)) return;
         ++tcnt;
       }
 
       const float nref = -ref;
-      const bool hand_over = t == 0 ? j < x.n1 : j + 1 < x.n0;
+      const bool hand_over = WINDOW ? (t == 0 ? j < x.n1 : j + 1 < x.n0) : (t == 0 || j + 1 < x.n0);
       float sum[4] = {0.f, 0.f, 0.f, 0.f};
       // the masked variant is a separate instantiation so full tiles carry no
       // per-score compare/select. exp_tile holds warp-collective instructions
