@@ -26,6 +26,11 @@ Also reported on the same JSON line:
 --impl reference times the FP64 CPU oracle (the only reference this build has)
 on the same workload, metric and unit, each step a bounded sample of it.
 
+--op stream times one steady-state streaming self-attention step through the
+rolling block cache (BlockKVCache: 1785-token chunks, a 7140-key window, 40
+query heads over 8 K/V heads, head RMSNorm + split-half RoPE): attn_stream_update
+then attn_fwd_cache, reported as attention TFLOPS over the whole step.
+
 --op prologue times the Q/K prologue instead (attn_qk_prologue: head-scope
 RMSNorm, eps 1e-6, then split-half RoPE, on Q and the new K chunk of the
 1785-token DiT workload, BF16 [1, 1785, 40, 128] each): an HBM-bound pass,
@@ -71,7 +76,7 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="minimum CPU time spent timing the oracle sample")
-    ap.add_argument("--op", default="attention", choices=["attention", "prologue"])
+    ap.add_argument("--op", default="attention", choices=["attention", "prologue", "stream"])
     ap.add_argument("--window", default=None,
                     help="LEFT,RIGHT: time attn_fwd_window with this sliding window (-1 = unbounded "
                          "side) instead of attn_fwd; FLOPs count the visible (row, key) pairs")
@@ -450,10 +455,100 @@ def run_prologue(args):
     return 0
 
 
+
+def run_stream(args):
+    """Steady-state streaming steps through the rolling block K/V cache."""
+    import torch
+
+    import head_attention_streaming_b200 as hasb
+    from head_attention_streaming_b200 import inputs
+
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    ranks = Ranks("nccl")
+    rank, world = ranks.rank, ranks.world
+    C, window, Hq, Hkv, d = 1785, 7140, 40, 8, 128
+    scale = 1.0 / math.sqrt(d)
+    n_chunks = 4 + max(3, args.warmup) + args.steps      # fill, warm-up, timed
+    g = torch.Generator().manual_seed(rank_seed(41, rank))
+    gq = (1.0 + 0.1 * torch.randn(d, generator=g)).cuda()
+    gk = (1.0 + 0.1 * torch.randn(d, generator=g)).cuda()
+    # one chunk's worth of inputs, reused with fresh positions every step
+    q = torch.randn(1, C, Hq, d, generator=g).to(torch.bfloat16).cuda()
+    k = torch.randn(1, C, Hkv, d, generator=g).to(torch.bfloat16).cuda()
+    v = torch.randn(1, C, Hkv, d, generator=g).to(torch.bfloat16).cuda()
+    angles = [inputs.rope_angle_table(C, d, hasb.ROPE_SPLIT, c * C).cuda() for c in range(n_chunks)]
+    cache = hasb.BlockKVCache(1, Hkv, d, C, window, 0)
+    o = torch.empty_like(q)
+    lse = torch.empty(1, Hq, C, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+    flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+
+    def step(c):
+        cache.before_update(c)
+        cache.attend(q, k, v, scale=scale, norm_scope=hasb.NORM_HEAD, gamma_q=gq, gamma_k=gk,
+                     rope_style=hasb.ROPE_SPLIT, angles_q=angles[c], angles_k=angles[c], out=o, lse=lse)
+        cache.after_update(c)
+
+    c = 0
+    for _ in range(4 + max(3, args.warmup)):   # fill the window, then warm up at steady state
+        step(c)
+        c += 1
+    torch.cuda.synchronize()
+    ranks.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    time.sleep(0.3)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    for a, b in ev:
+        flush_buf.add_(1)  # chunk inputs and cache (55 MB) fit in L2: evict them between steps
+        a.record(stream)
+        step(c)
+        b.record(stream)
+        c += 1
+    torch.cuda.synchronize()
+    ranks.barrier()
+    torch.cuda.synchronize()
+    clock_info = clocks.stop()
+    launch_ms = [a.elapsed_time(b) for a, b in ev]
+    ms_step = ranks.max(statistics.mean(launch_ms), "cuda")
+    flops = 4.0 * Hq * C * window * d
+    value = job_rate(world, flops, ms_step) / 1e12
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    achieved = flops / (statistics.mean(launch_ms) * 1e-3) / 1e12
+    if rank == 0:
+        line = {
+            "metric": "streaming self-attention step TFLOPS (rolling cache update + attention) on 1 B200",
+            "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic: seeded N(0,1) chunk Q/K/V, gamma = 1 + 0.1 N(0,1), per-chunk RoPE angles",
+            "config": {"workload": "stream_step_1785_window_7140_gqa40x8", "chunk": C, "window": window,
+                       "sink": 0, "Hq": Hq, "Hkv": Hkv, "d": d, "norm": "head", "rope": "split",
+                       "step": "attn_stream_update + attn_fwd_cache over the full window, both timed",
+                       "l2": "inputs 55 MB vs 126 MB L2: L2 flushed between steps",
+                       "parallelism": "single GPU" if world == 1 else f"{world} independent replicas"},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": None,
+                         "traffic_source": "no ncu summary of this two-kernel step",
+                         "peak_source": f"bf16_tflops (burst) of {peak_src}",
+                         "launch_ms_mean": statistics.mean(launch_ms)},
+            "cpu_baseline": None, "e2e": None, "gpu_launches": 2 * args.steps, "clocks": clock_info,
+            "device_fault_bits": hasb.device_fault(clear=True),
+        }
+        print(json.dumps(line))
+    ranks.close()
+    return 0
+
+
 def main():
     args = parse_args()
     if args.op == "prologue":
         return run_prologue(args)
+    if args.op == "stream":
+        return run_stream(args)
     if args.impl == "reference":
         return run_reference(args)
 

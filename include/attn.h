@@ -120,8 +120,9 @@ int attn_fwd_cache(const void* q, const void* k_cache, const void* v_cache, void
  *
  * Arguments as attn_fwd, plus:
  *   n_splits   requested number of key ranges, >= 1, or 0 to choose one from
- *              the shape and the SM count; clipped to the number of 128-key
- *              tiles, never an empty range
+ *              the shape and the SM count. Ranges are whole 128-key tiles,
+ *              ceil(tiles / n_splits) each, so the count used can be lower than
+ *              requested (4 tiles asked for 3 ranges give 2); never an empty range
  *   workspace  device float32 buffer of at least
  *              attn_splitkv_workspace_bytes(B, Lq, Hq, d, n) bytes for the n
  *              ranges used (partial O and LSE), 16-byte aligned, overlapping no
