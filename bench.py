@@ -76,7 +76,7 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="minimum CPU time spent timing the oracle sample")
-    ap.add_argument("--op", default="attention", choices=["attention", "prologue", "stream"])
+    ap.add_argument("--op", default="attention", choices=["attention", "prologue", "stream", "fp8"])
     ap.add_argument("--window", default=None,
                     help="LEFT,RIGHT: time attn_fwd_window with this sliding window (-1 = unbounded "
                          "side) instead of attn_fwd; FLOPs count the visible (row, key) pairs")
@@ -543,12 +543,145 @@ def run_stream(args):
     return 0
 
 
+def run_fp8(args):
+    """Unscaled FP8 attention: each step casts Q, K (attn_fp8_cast) and V
+    (attn_fp8_cast_vt, transposed) from bf16 to e4m3 and runs attn_fwd_fp8,
+    all four launches timed; the attention launch is also timed alone."""
+    import torch
+
+    import head_attention_streaming_b200 as hasb
+    from head_attention_streaming_b200 import inputs
+
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    ranks = Ranks("nccl")
+    rank, world = ranks.rank, ranks.world
+    w = select_workload(args)
+    if w.d != 128 or w.dtype != "bf16":
+        raise SystemExit("--op fp8 runs bf16 workloads with head_dim 128")
+    q_cpu, k_cpu, v_cpu = inputs.make_qkv(w.B, w.Lq, w.Lk, w.Hq, w.Hkv, w.d, w.torch_dtype,
+                                          seed=rank_seed(w.seed, rank), qk_rmsnorm=w.qk_rmsnorm)
+    q, k, v = q_cpu.cuda(), k_cpu.cuda(), v_cpu.cuda()
+    q8 = torch.empty(q.shape, dtype=hasb.binding.E4M3, device="cuda")
+    k8 = torch.empty(k.shape, dtype=hasb.binding.E4M3, device="cuda")
+    pitch = (w.Lk + 15) // 16 * 16
+    vt8 = torch.empty((w.B, w.Hkv, w.d, pitch), dtype=hasb.binding.E4M3, device="cuda")
+    o = torch.empty(q.shape, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((w.B, w.Hq, w.Lq), dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def casts():
+        hasb.fp8_cast(q, out=q8)
+        hasb.fp8_cast(k, out=k8)
+        hasb.fp8_cast_vt(v, pitch=pitch, out=vt8)
+
+    def attend():
+        hasb.attn_fwd_fp8(q8, k8, vt8, scale=w.scale, causal=w.mask, kv_offset=w.kv_offset, out=o, lse=lse)
+
+    for _ in range(max(3, args.warmup)):
+        casts()
+        attend()
+    torch.cuda.synchronize()
+    ranks.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    time.sleep(0.3)
+    flush = needs_flush(w)
+    flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda") if flush else None
+    ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(args.steps)]
+    for a, m, b in ev:
+        if flush:
+            flush_buf.add_(1)
+        a.record(stream)
+        casts()
+        m.record(stream)
+        attend()
+        b.record(stream)
+    torch.cuda.synchronize()
+    ranks.barrier()
+    torch.cuda.synchronize()
+    clock_info = clocks.stop()
+    step_ms = [a.elapsed_time(b) for a, _, b in ev]
+    attn_ms = [m.elapsed_time(b) for _, m, b in ev]
+    ms_step = ranks.max(statistics.mean(step_ms), "cuda")
+    flops = w.flops()
+    value = job_rate(world, flops, ms_step) / 1e12
+
+    e2e = None
+    if args.e2e_steps > 0:
+        qh, kh, vh = q_cpu.pin_memory(), k_cpu.pin_memory(), v_cpu.pin_memory()
+        oh = torch.empty(q_cpu.shape, dtype=torch.bfloat16).pin_memory()
+        lh = torch.empty((w.B, w.Hq, w.Lq), dtype=torch.float32).pin_memory()
+
+        def e2e_step():
+            q.copy_(qh, non_blocking=True)
+            k.copy_(kh, non_blocking=True)
+            v.copy_(vh, non_blocking=True)
+            casts()
+            attend()
+            oh.copy_(o, non_blocking=True)
+            lh.copy_(lse, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        ranks.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ranks.barrier()
+        e_ms = ranks.max(e0.elapsed_time(e1) / args.e2e_steps, "cuda")
+        e2e = {"value": job_rate(world, flops, e_ms) / 1e12, "unit": "TFLOPS", "ms_per_step": e_ms,
+               "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in (qh, kh, vh)),
+               "d2h_bytes_per_step": oh.numel() * oh.element_size() + lh.numel() * lh.element_size(),
+               "path": "pinned bf16 host Q/K/V -> device, fp8_cast x2 + fp8_cast_vt + attn_fwd_fp8, "
+                       "O and LSE -> host, one stream"}
+
+    peaks, peak_src = load_peaks()
+    peak16 = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    peak16_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    ci = clock_info or {}
+    capped = ("sw_power_cap" in ci.get("reasons", []) and "sm_mhz" in ci
+              and ci["sm_mhz"] < 0.97 * ci.get("sm_max_mhz", ci["sm_mhz"]))
+    peak = 2.0 * (peak16_sus if capped else peak16)   # e4m3 dense = 2 x bf16 dense (4.5 vs 2.25 PF)
+    achieved = flops / (statistics.mean(attn_ms) * 1e-3) / 1e12
+    if rank == 0:
+        line = {
+            "metric": "FP8 (e4m3) attention forward TFLOPS incl. the Q/K/V casts on 1 B200",
+            "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 (f32 accumulate, bf16 out)",
+            "data": "synthetic: seeded N(0,1) inputs of the workload's shape",
+            "config": dict(workload_config(w, world),
+                           step="fp8_cast(Q), fp8_cast(K), fp8_cast_vt(V), attn_fwd_fp8: all timed"),
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": None,
+                         "traffic_source": "no ncu summary of the FP8 kernel",
+                         "peak_source": ("2 x bf16_tflops_sustained" if capped else "2 x bf16_tflops (burst)")
+                                        + f" of {peak_src} (nominal e4m3 / bf16 dense ratio)",
+                         "kernel": "attn_fwd_sm100_kernel (e4m3)",
+                         "launch_ms_mean": statistics.mean(attn_ms),
+                         "casts_ms_mean": statistics.mean(step_ms) - statistics.mean(attn_ms)},
+            "cpu_baseline": None, "e2e": e2e, "gpu_launches": 4 * args.steps, "clocks": clock_info,
+            "device_fault_bits": hasb.device_fault(clear=True),
+        }
+        print(json.dumps(line))
+    ranks.close()
+    return 0
+
+
 def main():
     args = parse_args()
     if args.op == "prologue":
         return run_prologue(args)
     if args.op == "stream":
         return run_stream(args)
+    if args.op == "fp8":
+        return run_fp8(args)
     if args.impl == "reference":
         return run_reference(args)
 

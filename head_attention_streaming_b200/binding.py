@@ -59,6 +59,10 @@ _SIGNATURES = {
     "attn_fwd_window": (ctypes.c_int, [ctypes.c_void_p] * 5 + [ctypes.c_int] * 6 +
                         [ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                          ctypes.c_void_p]),
+    "attn_fp8_cast": (ctypes.c_int, [ctypes.c_void_p] * 2 + [ctypes.c_longlong, ctypes.c_int, ctypes.c_void_p]),
+    "attn_fp8_cast_vt": (ctypes.c_int, [ctypes.c_void_p] * 2 + [ctypes.c_int] * 6 + [ctypes.c_void_p]),
+    "attn_fwd_fp8": (ctypes.c_int, [ctypes.c_void_p] * 5 + [ctypes.c_int] * 7 +
+                     [ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
     "attn_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "attn_device_fault": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint), ctypes.c_int]),
     "attn_set_wait_timeout_ns": (ctypes.c_int, [ctypes.c_ulonglong]),
@@ -378,6 +382,85 @@ def attn_fwd_window(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, window
                                _stream_handle(stream, q.device))
     if st != ATTN_OK:
         raise AttnError(st, "attn_fwd_window")
+    return out, lse
+
+
+E4M3 = torch.float8_e4m3fn
+
+
+def _check_cuda(name, t, dim):
+    if not t.is_cuda or not t.is_contiguous() or t.dim() != dim:
+        raise ValueError(f"{name} must be a contiguous {dim}-D CUDA tensor")
+
+
+def fp8_cast(x: torch.Tensor, *, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """e4m3 copy of a 16-bit tensor (round to nearest even, saturated at +-448)
+    through ``attn_fp8_cast``; x.numel() must be a multiple of 8."""
+    _check_cuda("x", x, x.dim())
+    if x.dtype not in DTYPE_CODES:
+        raise ValueError("x must be bf16 or fp16")
+    if out is None:
+        out = torch.empty(x.shape, dtype=E4M3, device=x.device)
+    elif out.dtype != E4M3 or out.numel() != x.numel() or not out.is_contiguous() or not out.is_cuda:
+        raise ValueError("out must be a contiguous float8_e4m3fn CUDA tensor with x's size")
+    st = lib().attn_fp8_cast(_ptr(x), _ptr(out), x.numel(), DTYPE_CODES[x.dtype],
+                             _stream_handle(stream, x.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fp8_cast")
+    return out
+
+
+def fp8_cast_vt(v: torch.Tensor, *, pitch: int | None = None, out: torch.Tensor | None = None,
+                stream=None) -> torch.Tensor:
+    """V [B, Lk, Hkv, d] (16-bit) to e4m3 V^T [B, Hkv, d, pitch] through
+    ``attn_fp8_cast_vt``; pitch defaults to Lk rounded up to 16. Bytes at keys
+    >= Lk of a row are left as they were."""
+    _check_cuda("v", v, 4)
+    if v.dtype not in DTYPE_CODES:
+        raise ValueError("v must be bf16 or fp16")
+    B, Lk, Hkv, d = v.shape
+    if pitch is None:
+        pitch = (Lk + 15) // 16 * 16
+    if out is None:
+        out = torch.empty((B, Hkv, d, pitch), dtype=E4M3, device=v.device)
+    elif (out.dtype != E4M3 or tuple(out.shape) != (B, Hkv, d, pitch) or not out.is_contiguous()
+          or not out.is_cuda):
+        raise ValueError("out must be a contiguous float8_e4m3fn CUDA tensor [B, Hkv, d, pitch]")
+    st = lib().attn_fp8_cast_vt(_ptr(v), _ptr(out), B, Lk, Hkv, d, int(pitch), DTYPE_CODES[v.dtype],
+                                _stream_handle(stream, v.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fp8_cast_vt")
+    return out
+
+
+def attn_fwd_fp8(q8: torch.Tensor, k8: torch.Tensor, vt8: torch.Tensor, *, scale: float | None = None,
+                 causal: int = MASK_NONE, kv_offset: int = 0, out: torch.Tensor | None = None,
+                 lse: torch.Tensor | None = None, return_lse: bool = True, stream=None):
+    """Attention on e4m3 operands through ``attn_fwd_fp8``: q8 [B, Lq, Hq, d],
+    k8 [B, Lk, Hkv, d], vt8 [B, Hkv, d, pitch] (``fp8_cast_vt``), all
+    float8_e4m3fn. Returns ``(out, lse)``, out bf16 [B, Lq, Hq, d]."""
+    for name, t in (("q8", q8), ("k8", k8), ("vt8", vt8)):
+        _check_cuda(name, t, 4)
+        if t.dtype != E4M3:
+            raise ValueError(f"{name} must be float8_e4m3fn")
+    B, Lq, Hq, d = q8.shape
+    Bk, Lk, Hkv, dk = k8.shape
+    if Bk != B or dk != d or tuple(vt8.shape[:3]) != (B, Hkv, d):
+        raise ValueError("q8, k8, vt8 shapes disagree")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((B, Lq, Hq, d), dtype=torch.bfloat16, device=q8.device)
+    elif (out.dtype != torch.bfloat16 or tuple(out.shape) != (B, Lq, Hq, d) or not out.is_contiguous()
+          or not out.is_cuda):
+        raise ValueError("out must be a contiguous bf16 CUDA tensor [B, Lq, Hq, d]")
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q8.device)
+    st = lib().attn_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(vt8), _ptr(out), _ptr(lse), B, Lq, Lk,
+                            vt8.shape[3], Hq, Hkv, d, float(scale), int(causal), int(kv_offset),
+                            _stream_handle(stream, q8.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fwd_fp8")
     return out, lse
 
 

@@ -17,7 +17,8 @@ PKG_DIR = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(PKG_DIR, "csrc")
 INCLUDE = os.path.join(os.path.dirname(PKG_DIR), "include")
 SO_PATH = os.path.join(PKG_DIR, "libattn_sm100.so")
-SOURCES = [os.path.join(CSRC, "attn_fwd_sm100.cu"), os.path.join(CSRC, "qk_prologue.cu")]
+SOURCES = [os.path.join(CSRC, "attn_fwd_sm100.cu"), os.path.join(CSRC, "qk_prologue.cu"),
+           os.path.join(CSRC, "fp8_pack.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, "sm100_ptx.cuh"), os.path.join(CSRC, "tmem_ldst.inc"),
                   os.path.join(INCLUDE, "attn.h")]
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]

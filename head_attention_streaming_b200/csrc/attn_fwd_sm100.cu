@@ -67,7 +67,7 @@ constexpr float kRescaleTau = 8.0f;    // lazy rescale threshold, log2 units (P 
 constexpr float kLn2 = 0.69314718055994531f;
 constexpr float kLog2e = 1.4426950408889634f;
 
-template <int D>
+template <int D, bool F8 = false>
 struct Cfg {
   static constexpr int kChunks = D / 64;              // 128-byte swizzle chunks per row
   static constexpr int kChunkBytes = kTileRows * 128;  // one chunk of a 128-row tile
@@ -81,6 +81,30 @@ struct Cfg {
   // tensor-memory columns of S_t (P_t aliased) and O_t
   static __device__ __forceinline__ uint32_t col_s(int t) { return t ? 128u : 0u; }
   static __device__ __forceinline__ uint32_t col_o(int t) { return t ? 256u + D : 256u; }
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr int kOChunks = D / 64;  // 64-column chunks of the 16-bit O staging tile
+  static constexpr int kOffP = 0;          // P lives in tensor memory
+};
+
+// e4m3 operands, d = 128: a Q / K row is one 128-byte swizzle chunk (16 KB per
+// 128-row tile), V arrives transposed (a tile is 128 d-rows of 128 keys) so
+// both P V operands are K-major, and P goes through shared memory (two 16 KB
+// buffers, K-major with the same swizzle) instead of tensor memory.
+template <>
+struct Cfg<128, true> {
+  static constexpr int kChunks = 1;
+  static constexpr int kChunkBytes = kTileRows * 128;
+  static constexpr int kTileBytes = kTileRows * 128;
+  static constexpr int kStages = 8;
+  static constexpr int kOChunks = 2;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffKV = 2 * kTileBytes;
+  static constexpr int kOffP = kOffKV + kStages * kTileBytes;
+  static constexpr int kOffStg = kOffP + 2 * kTileBytes;
+  static constexpr int kOffBar = kOffStg + kOChunks * kChunkBytes;
+  static constexpr int kSmemBytes = kOffBar + 512 + 1024;
+  static __device__ __forceinline__ uint32_t col_s(int t) { return t ? 128u : 0u; }
+  static __device__ __forceinline__ uint32_t col_o(int t) { return t ? 384u : 256u; }
   static constexpr uint32_t kTmemCols = 512;
 };
 
@@ -261,6 +285,27 @@ __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
 // Q and K tiles are K-major with the 128-byte swizzle (TMA boxes of 64 elements
 // x 128 rows): 16 elements = 32 bytes along K inside a chunk, then the next
 // chunk. Descriptor address fields count 16-byte units.
+// e4m3 Q K^T: D/32 MMAs of 128x128x32 (kind::f8f6f4), 32 bytes along K each,
+// inside the single 128-byte swizzle chunk of a row.
+template <int D>
+__device__ __forceinline__ void issue_qk_f8(uint32_t d_tmem, uint32_t q_lo, uint32_t k_lo) {
+  constexpr uint32_t idesc = mma_idesc_f16(false, 128, 128, false, false);
+#pragma unroll
+  for (int kk = 0; kk < D / 32; ++kk)
+    mma_f8_ss_lo_flag(d_tmem, q_lo + 2 * kk, k_lo + 2 * kk, idesc, kk > 0 ? 1u : 0u);
+}
+
+// e4m3 O += P V for half HALF of the 128 keys: A = P (shared memory, K-major),
+// B = V^T (K-major): two MMAs of 128xDx32, 32 keys (bytes) each.
+template <int D, int HALF>
+__device__ __forceinline__ void issue_pv_half_f8(uint32_t d_tmem, uint32_t p_lo, uint32_t vt_lo,
+                                                 uint32_t accumulate) {
+  constexpr uint32_t idesc = mma_idesc_f16(false, 128, D, false, false);
+#pragma unroll
+  for (int kk = 2 * HALF; kk < 2 * HALF + 2; ++kk)
+    mma_f8_ss_lo_flag(d_tmem, p_lo + 2 * kk, vt_lo + 2 * kk, idesc, kk == 0 ? accumulate : 1u);
+}
+
 template <int D, bool BF16>
 __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_lo, uint32_t k_lo) {
   constexpr uint32_t idesc = mma_idesc_f16(BF16, 128, 128, false, false);
@@ -298,12 +343,12 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint3
   issue_pv_half<D, BF16, 1>(d_tmem, p_tmem, v_lo, 1u);
 }
 
-template <int D, bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW>
+template <int D, bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW, bool F8>
 __device__ __forceinline__ void load_role(const CUtensorMap* tm_q, const CUtensorMap* tm_k,
                                           const CUtensorMap* tm_v, const FwdParams& p,
                                           uint32_t sQ, uint32_t sKV, uint32_t bars,
                                           volatile int* abort_flag) {
-  using C = Cfg<D>;
+  using C = Cfg<D, F8>;
   const uint64_t pol_q = l2_policy_evict_first();
   const uint64_t pol_kv = l2_policy_evict_last();
   int kv_it = 0, uit = 0;
@@ -334,10 +379,20 @@ __device__ __forceinline__ void load_role(const CUtensorMap* tm_q, const CUtenso
         }
         const uint32_t bf = bars + 8 * (kBarKvFull + slot);
         mbar_arrive_expect_tx(bf, C::kTileBytes);
+        if constexpr (F8) {
+          // K: (d, head, key, batch); transposed V: (key, d, head, batch)
+          if (kv)
+            tma_load_4d(sKV + slot * C::kTileBytes, tm_v, bf, (x.j0 + j) * kTileRows, 0, x.hkv, x.b,
+                        pol_kv);
+          else
+            tma_load_4d(sKV + slot * C::kTileBytes, tm_k, bf, 0, x.hkv, (x.j0 + j) * kTileRows, x.b,
+                        pol_kv);
+        } else {
 #pragma unroll
-        for (int c = 0; c < C::kChunks; ++c)
-          tma_load_4d(sKV + slot * C::kTileBytes + c * C::kChunkBytes, kv ? tm_v : tm_k, bf,
-                      c * 64, x.hkv, (x.j0 + j) * kTileRows, x.b, pol_kv);
+          for (int c = 0; c < C::kChunks; ++c)
+            tma_load_4d(sKV + slot * C::kTileBytes + c * C::kChunkBytes, kv ? tm_v : tm_k, bf,
+                        c * 64, x.hkv, (x.j0 + j) * kTileRows, x.b, pol_kv);
+        }
         ++kv_it;
       }
     }
@@ -358,10 +413,13 @@ __device__ __forceinline__ void load_role(const CUtensorMap* tm_q, const CUtenso
 // issuing the other's GEMMs. With one thread per tile, the tensor core runs
 // whichever tile has work. Both threads read the same K/V ring slots; each slot
 // use is released by both (kv_empty takes two arrivals).
-template <int D, bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW>
+template <int D, bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW, bool F8>
 __device__ __forceinline__ void mma_role(const int t, const FwdParams& p, uint32_t tmem, uint32_t sQ,
-                                         uint32_t sKV, uint32_t bars, volatile int* abort_flag) {
-  using C = Cfg<D>;
+                                         uint32_t sKV, uint32_t sP, uint32_t bars,
+                                         volatile int* abort_flag) {
+  using C = Cfg<D, F8>;
+  // e4m3: P_t in shared memory (K-major, 128-byte swizzle)
+  const uint32_t p_lo = smem_desc_lo(sP + t * C::kTileBytes, 16);
   auto bar = [&](int i) { return bars + 8 * i; };
   // low descriptor halves: Q and K tiles K-major (LBO unused, 16), V tiles MN-major (LBO = chunk)
   const uint32_t q_lo = smem_desc_lo(sQ + t * C::kTileBytes, 16);
@@ -398,7 +456,8 @@ __device__ __forceinline__ void mma_role(const int t, const FwdParams& p, uint32
     ok = ok && kv_full(kb);
     if (!ok) break;
     // S_t(0) = Q_t K_0^T
-    issue_qk<D, BF16>(s_t, q_lo, k_lo(kb));
+    if constexpr (F8) issue_qk_f8<D>(s_t, q_lo, k_lo(kb));
+    else issue_qk<D, BF16>(s_t, q_lo, k_lo(kb));
     mma_commit(bar(kBarSFull + t));
     mma_commit(bar(kBarKvEmpty + kb % C::kStages));
     if (n == 1) mma_commit(bar(kBarQEmpty + t));
@@ -413,20 +472,23 @@ __device__ __forceinline__ void mma_role(const int t, const FwdParams& p, uint32
         break;
       }
       tc_fence_after_sync();
-      issue_pv_half<D, BF16, 0>(o_t, s_t, v_lo(vidx), j > 0 ? 1u : 0u);
+      if constexpr (F8) issue_pv_half_f8<D, 0>(o_t, p_lo, k_lo(vidx), j > 0 ? 1u : 0u);
+      else issue_pv_half<D, BF16, 0>(o_t, s_t, v_lo(vidx), j > 0 ? 1u : 0u);
       if (!mbar_wait(bar(kBarPFull + t), pcnt & 1, abort_flag, kFaultMmaPFull, p.timeout_ns)) {
         ok = false;
         break;
       }
       ++pcnt;
       tc_fence_after_sync();
-      issue_pv_half<D, BF16, 1>(o_t, s_t, v_lo(vidx), 1u);
+      if constexpr (F8) issue_pv_half_f8<D, 1>(o_t, p_lo, k_lo(vidx), 1u);
+      else issue_pv_half<D, BF16, 1>(o_t, s_t, v_lo(vidx), 1u);
       mma_commit(bar(kBarKvEmpty + vidx % C::kStages));
       if (j == n - 1) {
         mma_commit(bar(kBarOFull + t));
       } else {
         if (!kv_full(knext)) { ok = false; break; }
-        issue_qk<D, BF16>(s_t, q_lo, k_lo(knext));
+        if constexpr (F8) issue_qk_f8<D>(s_t, q_lo, k_lo(knext));
+        else issue_qk<D, BF16>(s_t, q_lo, k_lo(knext));
         mma_commit(bar(kBarSFull + t));
         mma_commit(bar(kBarKvEmpty + knext % C::kStages));
         if (j + 1 == n - 1) mma_commit(bar(kBarQEmpty + t));
@@ -459,6 +521,51 @@ __device__ __forceinline__ void mma_role(const int t, const FwdParams& p, uint32
 // moves on the ALU pipe here). MASKED: keys c >= lim are zeroed after the
 // exponential (their -inf scores times a zero scale, or -inf + inf when the
 // row has no visible key yet, would give NaN).
+// e4m3 variant of exp_tile: P = exp2(s * sl2 - ref) rounded to e4m3 (four keys
+// per 32-bit word) into this row of the P_t buffer in shared memory (128 bytes
+// per row, K-major with the 128-byte swizzle: 16-byte unit u of row r at
+// r * 128 + ((u ^ (r % 8)) * 16)), in two halves of 64 keys, each handed to the
+// MMA issuer once it is visible to the tensor core (proxy fence). The row sum
+// uses the unrounded P.
+template <bool MASKED>
+__device__ __forceinline__ void exp_tile_f8(const uint32_t (&r)[128], float sl2, float nref, int lim,
+                                            int lim_lo, float (&sum)[4], uint32_t prow, int r_in,
+                                            uint32_t bar_half, uint32_t bar_full, uint32_t bar_turn_other,
+                                            bool hand_over, int lane) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t w[16];
+#pragma unroll
+    for (int cc = 0; cc < 16; ++cc) {
+      float pv[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int c = 64 * h + 4 * cc + e;
+        float pe = ex2_approx(fmaf(__uint_as_float(r[c]), sl2, nref));
+        if (MASKED) pe = (c < lim && c >= lim_lo) ? pe : 0.f;
+        sum[e] += pe;
+        pv[e] = pe;
+      }
+      w[cc] = pack_e4m3x2(pv[0], pv[1]) | (pack_e4m3x2(pv[2], pv[3]) << 16);
+    }
+    if (h == 1 && hand_over) {  // exponentials done: hand over the turn
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_turn_other);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const uint32_t unit = static_cast<uint32_t>((4 * h + u) ^ (r_in & 7));
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow + unit * 16), "r"(w[4 * u]),
+                   "r"(w[4 * u + 1]), "r"(w[4 * u + 2]), "r"(w[4 * u + 3])
+                   : "memory");
+    }
+    fence_proxy_async_smem();
+    tc_fence_before_sync();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(h == 0 ? bar_half : bar_full);
+  }
+}
+
 template <bool BF16, bool MASKED>
 __device__ __forceinline__ void exp_tile(const uint32_t (&r)[128], float sl2, float nref, int lim, int lim_lo,
                                          float (&sum)[4], uint32_t tS, uint32_t bar_half,
@@ -502,10 +609,10 @@ __device__ __forceinline__ void exp_tile(const uint32_t (&r)[128], float sl2, fl
 // buffer to global memory with a TMA store (rows past Lq are clipped by the
 // tensor map), then hands the buffer to the other query tile. Order per unit:
 // tile 0, then tile 1, the same order the softmax warpgroups fill it in.
-template <int D, bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW>
+template <int D, bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW, bool F8>
 __device__ __forceinline__ void store_role(const CUtensorMap* tm_o, const FwdParams& p, uint32_t sStg,
                                            uint32_t bars, volatile int* abort_flag) {
-  using C = Cfg<D>;
+  using C = Cfg<D, F8>;
   int scnt = 0;
   bool ok = true;
   for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
@@ -515,7 +622,7 @@ __device__ __forceinline__ void store_role(const CUtensorMap* tm_o, const FwdPar
       if (!ok) break;
       ++scnt;
 #pragma unroll
-      for (int c = 0; c < C::kChunks; ++c)
+      for (int c = 0; c < C::kOChunks; ++c)
         tma_store_4d(tm_o, sStg + c * C::kChunkBytes, c * 64, x.hq, x.r0 + t * kTileRows, x.b);
       bulk_commit_group();
       bulk_wait_group_read0();
@@ -525,10 +632,12 @@ __device__ __forceinline__ void store_role(const CUtensorMap* tm_o, const FwdPar
   bulk_wait_group0();  // every store complete before the CTA exits
 }
 
-template <int D, bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW>
+template <int D, bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW, bool F8>
 __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, uint32_t tmem,
-                                             uint32_t bars, uint32_t sstg, volatile int* abort_flag) {
-  using C = Cfg<D>;
+                                             uint32_t bars, uint32_t sstg, uint32_t sP,
+                                             volatile int* abort_flag) {
+  using C = Cfg<D, F8>;
+  const uint32_t prow = sP + t * C::kTileBytes + (threadIdx.x % kTileRows) * 128;  // e4m3 P row
   const int warp = threadIdx.x / 32;
   const int r_in = threadIdx.x % kTileRows;                      // row in tile = TMEM lane
   const uint32_t lane_bits = static_cast<uint32_t>((warp % 4) * 32) << 16;
@@ -658,7 +767,15 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
       // (tcgen05.st, __syncwarp), so the choice must be the same for the whole
       // warp: rows of one warp can differ (causal), and a lane whose keys are
       // all visible is unaffected by the masked variant.
-      if (__any_sync(0xffffffffu, partial)) {
+      if constexpr (F8) {
+        if (__any_sync(0xffffffffu, partial)) {
+          exp_tile_f8<true>(r, sl2, nref, lim, lim_lo, sum, prow, r_in, bar_ph, bar_p, bar_turn_other,
+                            hand_over, lane);
+        } else {
+          exp_tile_f8<false>(r, sl2, nref, lim, lim_lo, sum, prow, r_in, bar_ph, bar_p, bar_turn_other,
+                             hand_over, lane);
+        }
+      } else if (__any_sync(0xffffffffu, partial)) {
         exp_tile<BF16, true>(r, sl2, nref, lim, lim_lo, sum, tS, bar_ph, bar_p, bar_turn_other, hand_over,
                              lane);
       } else {
@@ -738,13 +855,13 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
   }
 }
 
-template <int D, bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW>
+template <int D, bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v,
                           const __grid_constant__ CUtensorMap tm_o, const FwdParams p) {
-  using C = Cfg<D>;
+  using C = Cfg<D, F8>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -752,6 +869,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sQ = sbase + C::kOffQ;
   const uint32_t sKV = sbase + C::kOffKV;
   const uint32_t sStg = sbase + C::kOffStg;
+  const uint32_t sP = sbase + C::kOffP;  // e4m3 P buffers (unused otherwise)
   const uint32_t bars = sbase + C::kOffBar;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffBar + 448);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffBar + 452);
@@ -804,15 +922,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < 8) {
     regs_increase<kRegsSoftmax>();
-    softmax_role<D, BF16, CAUSAL, SPLIT, WINDOW>(warp / 4, p, tmem, bars, sStg, abort_flag);
+    softmax_role<D, BF16, CAUSAL, SPLIT, WINDOW, F8>(warp / 4, p, tmem, bars, sStg, sP, abort_flag);
   } else {
     regs_decrease<kRegsProducer>();
     if (warp == 8) {
-      if (lane == 0) load_role<D, BF16, CAUSAL, SPLIT, WINDOW>(&tm_q, &tm_k, &tm_v, p, sQ, sKV, bars, abort_flag);
+      if (lane == 0) load_role<D, BF16, CAUSAL, SPLIT, WINDOW, F8>(&tm_q, &tm_k, &tm_v, p, sQ, sKV, bars, abort_flag);
     } else if (warp == 9 || warp == 10) {
-      if (lane == 0) mma_role<D, BF16, CAUSAL, SPLIT, WINDOW>(warp - 9, p, tmem, sQ, sKV, bars, abort_flag);
+      if (lane == 0) mma_role<D, BF16, CAUSAL, SPLIT, WINDOW, F8>(warp - 9, p, tmem, sQ, sKV, sP, bars,
+                                                                    abort_flag);
     } else if (!SPLIT) {
-      if (lane == 0) store_role<D, BF16, CAUSAL, SPLIT, WINDOW>(&tm_o, p, sStg, bars, abort_flag);
+      if (lane == 0) store_role<D, BF16, CAUSAL, SPLIT, WINDOW, F8>(&tm_o, p, sStg, bars, abort_flag);
     }
   }
   __syncwarp();
@@ -1061,17 +1180,56 @@ bool encode_bl_hd(CUtensorMap* map, const void* ptr, int B, int L, int H, int d,
   return r == CUDA_SUCCESS;
 }
 
-template <int D, bool BF16, bool CAUSAL, bool SPLIT = false, bool WINDOW = false>
+// [B, L, H, d] e4m3 tensor (d = 128 bytes per head row) as a 4-D TMA map:
+// box = the whole 128-byte row of one head x 128 rows, 128-byte swizzle.
+bool encode_e4m3_bl_hd(CUtensorMap* map, const void* ptr, int B, int L, int H, int d) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)L, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)d, (cuuint64_t)H * d, (cuuint64_t)L * H * d};
+  const cuuint32_t box[4] = {128, 1, (cuuint32_t)kTileRows, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Transposed e4m3 V, [B, Hkv, d, pitch] bytes (key index innermost, rows of
+// `pitch` >= Lk bytes): box = 128 keys x 128 d-rows, 128-byte swizzle.
+bool encode_e4m3_vt(CUtensorMap* map, const void* ptr, int B, int Lk, int pitch, int Hkv, int d) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)Lk, (cuuint64_t)d, (cuuint64_t)Hkv, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)pitch, (cuuint64_t)d * pitch, (cuuint64_t)Hkv * d * pitch};
+  const cuuint32_t box[4] = {(cuuint32_t)kTileRows, 128, 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, bool BF16, bool CAUSAL, bool SPLIT = false, bool WINDOW = false, bool F8 = false>
 int launch_fwd(const FwdParams& p, const void* q, const void* k, const void* v, int kv_rows, int grid,
                cudaStream_t stream) {
-  using C = Cfg<D>;
+  using C = Cfg<D, F8>;
   CUtensorMap tq, tk, tv, to;
-  if (!encode_bl_hd(&tq, q, p.B, p.Lq, p.Hq, D, BF16) ||
-      !encode_bl_hd(&tk, k, p.B, p.Lk, p.Hkv, D, BF16, kv_rows) ||
-      !encode_bl_hd(&tv, v, p.B, p.Lk, p.Hkv, D, BF16, kv_rows) ||
-      !encode_bl_hd(&to, p.o, p.B, p.Lq, p.Hq, D, BF16))
-    return ATTN_ERR_CUDA;
-  auto kern = attn_fwd_sm100_kernel<D, BF16, CAUSAL, SPLIT, WINDOW>;
+  if constexpr (F8) {
+    // e4m3 Q / K (box: the 128-byte row of a head, 128 rows); V transposed,
+    // [B, Hkv, d, kv_rows] bytes with kv_rows a multiple of 16 (box: 128 keys
+    // x 128 d-rows); O bf16 as usual
+    if (!encode_e4m3_bl_hd(&tq, q, p.B, p.Lq, p.Hq, D) ||
+        !encode_e4m3_bl_hd(&tk, k, p.B, p.Lk, p.Hkv, D) ||
+        !encode_e4m3_vt(&tv, v, p.B, p.Lk, kv_rows, p.Hkv, D) ||
+        !encode_bl_hd(&to, p.o, p.B, p.Lq, p.Hq, D, true))
+      return ATTN_ERR_CUDA;
+  } else {
+    if (!encode_bl_hd(&tq, q, p.B, p.Lq, p.Hq, D, BF16) ||
+        !encode_bl_hd(&tk, k, p.B, p.Lk, p.Hkv, D, BF16, kv_rows) ||
+        !encode_bl_hd(&tv, v, p.B, p.Lk, p.Hkv, D, BF16, kv_rows) ||
+        !encode_bl_hd(&to, p.o, p.B, p.Lq, p.Hq, D, BF16))
+      return ATTN_ERR_CUDA;
+  }
+  auto kern = attn_fwd_sm100_kernel<D, BF16, CAUSAL, SPLIT, WINDOW, F8>;
   static std::once_flag attr_flags[kMaxDevices];
   static int attr_status[kMaxDevices];
   int dev = 0;
@@ -1369,6 +1527,62 @@ int attn_fwd_window(const void* q, const void* k, const void* v, void* o, float*
                     int kv_offset, int dtype, void* stream) {
   return attn_fwd_impl(q, k, v, o, lse, B, Lq, Lk, Lk, Hq, Hkv, d, scale, ATTN_MASK_NONE, kv_offset,
                        dtype, stream, true, window_left, window_right);
+}
+
+int attn_fwd_fp8(const void* q8, const void* k8, const void* vt8, void* o, float* lse, int B, int Lq,
+                 int Lk, int vt_pitch, int Hq, int Hkv, int d, float scale, int causal, int kv_offset,
+                 void* stream) {
+  // ---- argument contract (no CUDA call before it passes)
+  if (q8 == nullptr || k8 == nullptr || vt8 == nullptr || o == nullptr) return ATTN_ERR_INVALID_ARG;
+  if (B < 1 || Lq < 1 || Lk < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (d < 16 || d > 256 || (d & (d - 1)) != 0) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || scale < 0.f) return ATTN_ERR_INVALID_ARG;
+  if (causal != ATTN_MASK_NONE && causal != ATTN_MASK_CAUSAL && causal != ATTN_MASK_CHUNK)
+    return ATTN_ERR_INVALID_ARG;
+  if (causal == ATTN_MASK_NONE ? kv_offset != 0
+                               : (kv_offset < 0 || static_cast<long long>(kv_offset) + Lq > Lk))
+    return ATTN_ERR_INVALID_ARG;
+  if (vt_pitch < Lk || vt_pitch % 16 != 0) return ATTN_ERR_INVALID_ARG;
+  const auto a16 = [](const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; };
+  if (!a16(q8) || !a16(k8) || !a16(vt8) || !a16(o) || (reinterpret_cast<uintptr_t>(lse) & 3u) != 0)
+    return ATTN_ERR_INVALID_ARG;
+  const unsigned long long q_elems = 1ull * B * Lq * Hq * d, k_elems = 1ull * B * Lk * Hkv * d;
+  const unsigned long long vt_bytes = 1ull * B * Hkv * d * vt_pitch;
+  if (q_elems * 2 >= (1ull << 40) || k_elems >= (1ull << 40) || vt_bytes >= (1ull << 40))
+    return ATTN_ERR_INVALID_ARG;
+  const long long n_pairs = (Lq + 2LL * kTileRows - 1) / (2LL * kTileRows);
+  const long long n_units = n_pairs * B * Hq;
+  if (n_units > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+  if (ranges_overlap(o, q_elems * 2, q8, q_elems) || ranges_overlap(o, q_elems * 2, k8, k_elems) ||
+      ranges_overlap(o, q_elems * 2, vt8, vt_bytes))
+    return ATTN_ERR_INVALID_ARG;
+  if (d != 128) return ATTN_ERR_UNSUPPORTED;
+  // ---- device
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+  const DeviceInfo di = device_info(dev);
+  if (!di.ok) return ATTN_ERR_CUDA;
+  if (!di.sm100) return ATTN_ERR_UNSUPPORTED;
+  FwdParams p;
+  p.o = o;
+  p.lse = lse;
+  p.B = B; p.Lq = Lq; p.Lk = Lk; p.Hq = Hq; p.Hkv = Hkv; p.group = Hq / Hkv;
+  p.kv_offset = kv_offset;
+  p.kv_limit = (causal == ATTN_MASK_CHUNK) ? kv_offset + Lq : Lk;
+  p.n_pairs = static_cast<int>(n_pairs);
+  p.n_units = static_cast<int>(n_units);
+  p.sl2 = scale * kLog2e;
+  p.timeout_ns = g_timeout_ns.load();
+  p.n_splits = 1;
+  p.split_tiles = (p.kv_limit + kTileRows - 1) / kTileRows;
+  p.o_part = nullptr;
+  p.lse_part = nullptr;
+  p.win_left = p.win_right = -1;
+  const int grid = static_cast<int>(n_units < di.num_sms ? n_units : di.num_sms);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return causal == ATTN_MASK_CAUSAL
+             ? launch_fwd<128, true, true, false, false, true>(p, q8, k8, vt8, vt_pitch, grid, s)
+             : launch_fwd<128, true, false, false, false, true>(p, q8, k8, vt8, vt_pitch, grid, s);
 }
 
 int attn_fwd_cache(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,

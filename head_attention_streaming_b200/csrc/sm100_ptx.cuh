@@ -217,6 +217,30 @@ __device__ __forceinline__ void mma_f16_ts_lo_flag(uint32_t d_tmem, uint32_t a_t
       : "memory");
 }
 
+// D[tmem] (+)= A[smem] * B[smem]^T for 8-bit e4m3 operands (kind::f8f6f4; one
+// instruction covers K = 32). Type code 0 in the A / B type fields of the
+// instruction descriptor is e4m3 for this kind, so mma_idesc_f16(false, ...)
+// describes it.
+__device__ __forceinline__ void mma_f8_ss_lo_flag(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo,
+                                                  uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "mov.b64 da, {%1, %3};\n\t"
+      "mov.b64 db, {%2, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], da, db, %4, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_lo), "r"(b_lo), "n"(kSmemDescHiSw128), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
+// Two floats to two e4m3 bytes, round to nearest even, saturating at +-448:
+// lo in bits 0-7, hi in bits 8-15.
+__device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
+  unsigned short r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
 // Arrive once on `bar` when every tcgen05 operation this thread issued so far
 // has completed.
 __device__ __forceinline__ void mma_commit(uint32_t bar) {

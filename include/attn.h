@@ -97,6 +97,34 @@ int attn_fwd_window(const void* q, const void* k, const void* v, void* o, float*
                     int kv_offset, int dtype, void* stream);
 
 /*
+ * Unscaled FP8 attention (developer guide, "OptimizedImplConfig":
+ * quantized_sdpa casts Q, K and V directly to float8_e4m3fn, keeps the K/V
+ * cache in that type, and uses FP8 probabilities for the P V product).
+ *
+ * attn_fp8_cast — y[i] = e4m3(x[i]) for n 16-bit values (dtype), rounded to
+ * nearest even and saturated at +-448. n % 8 == 0; x 16-byte and y 8-byte
+ * aligned; no overlap. Asynchronous on `stream`.
+ *
+ * attn_fp8_cast_vt — V [B, Lk, Hkv, d] (16-bit, dtype) to e4m3 transposed:
+ * vt[b, h, c, j] = e4m3(v[b, j, h, c]) in [B, Hkv, d, pitch] bytes, pitch >= Lk
+ * and a multiple of 16 (bytes j >= Lk of a row are not written); d a multiple
+ * of 64. The transposed layout makes V's tiles the K-major operand of P V.
+ *
+ * attn_fwd_fp8 — attention forward on e4m3 operands: q8 [B, Lq, Hq, d] and
+ * k8 [B, Lk, Hkv, d] e4m3, vt8 as written by attn_fp8_cast_vt (pitch
+ * vt_pitch); S = scale q8 k8^T and the softmax in float32; P rounded to e4m3
+ * for the P V product (the row sum uses the unrounded P); o [B, Lq, Hq, d]
+ * bfloat16 and lse as attn_fwd. Masks, GQA, kv_offset and errors as attn_fwd;
+ * this build runs d = 128 (other head dims: ATTN_ERR_UNSUPPORTED).
+ */
+int attn_fp8_cast(const void* x, void* y, long long n, int dtype, void* stream);
+int attn_fp8_cast_vt(const void* v, void* vt, int B, int Lk, int Hkv, int d, int pitch, int dtype,
+                     void* stream);
+int attn_fwd_fp8(const void* q8, const void* k8, const void* vt8, void* o, float* lse, int B, int Lq,
+                 int Lk, int vt_pitch, int Hq, int Hkv, int d, float scale, int causal, int kv_offset,
+                 void* stream);
+
+/*
  * attn_fwd_cache — attn_fwd with K and V read from the first Lk tokens of a
  * [B, S, Hkv, d] cache (the rolling block cache of streaming self-attention,
  * whose valid tokens are a prefix of its S slots): batch b's keys start at

@@ -18,10 +18,21 @@ Readings (listed in DESIGN.md):
 * The cast rounds to nearest even and saturates at +-448 (the largest finite
   e4m3 value; the type has no infinities).
 * P is rounded to e4m3 before the P V product while the row sum l uses the
-  unrounded P. The oracle does not model that rounding; ``p_rounding_bound``
-  gives the per-element bound it implies: each weight w_j carries a relative
-  error of at most 2^-4 (half an e4m3 unit), so
-  |O_gpu - O| <= 2^-4 sum_j w_j |v_j| (+ the 16-bit rounding of O).
+  unrounded P. The oracle does not model that rounding (where it happens
+  depends on the running reference of the online softmax); it gives two
+  per-element figures the rounding implies, for any reference at or below the
+  row max (so every P <= 1, or <= 2^8 with a lagging reference: no
+  saturation). With w the exact softmax weights, w_max their row maximum and
+  P_j = w_j / w_max times a power of the reference gap that is <= 1:
+
+  - ``p_rounding_bound``: a normal e4m3 value has 3 mantissa bits, so rounding
+    moves it by at most 2^-4 of itself; below the smallest normal (2^-6) the
+    spacing is 2^-9 and the error at most 2^-10, i.e. 2^-10 w_max in weight
+    units. Hence |O_gpu - O| <= sum_j max(2^-4 w_j, 2^-10 w_max) |v_j|.
+  - ``p_rounding_var``: the same errors taken as independent and uniform over
+    one spacing (relative spacing at most 2^-3 for normal values, absolute
+    2^-9 w_max below them) give the variance bound
+    sum_j max(2^-6 w_j^2, 2^-18 w_max^2) v_j^2 / 12 of each output element.
 """
 
 from __future__ import annotations
@@ -47,17 +58,45 @@ def attention_fp8(q, k, v, scale: float, mask: int = 0, kv_offset: int = 0, rows
     return attention_fwd(e4m3(q), e4m3(k), e4m3(v), scale, mask, kv_offset, rows=rows)
 
 
-def p_rounding_bound(q, k, v, scale: float, mask: int = 0, kv_offset: int = 0) -> np.ndarray:
-    """Per-element bound [B, Lq, Hq, d] on |O| error from rounding P to e4m3:
-    2^-4 * sum_j w_j |v_j| with w the exact softmax weights (tiny inputs)."""
+def _weights_and_v(q, k, v, scale, mask, kv_offset, rows):
+    """Yield (b, hq, w [R, Lk], v8 [Lk, d]) per (batch, head) of the cast
+    inputs, w the exact softmax weights of the rows (one head at a time, so
+    long sequences need only R x Lk weights at once)."""
     q8, k8, v8 = e4m3(q), e4m3(k), e4m3(v)
-    _, _, w = attention_fwd(q8, k8, v8, scale, mask, kv_offset, return_weights=True)
     B, Lq, Hq, d = q8.shape
     Hkv = k8.shape[2]
     rep = Hq // Hkv
-    av = np.abs(v8)
-    out = np.zeros((B, Lq, Hq, d))
     for b in range(B):
         for h in range(Hq):
-            out[b, :, h, :] = w[b, h] @ av[b, :, h // rep, :]
-    return 2.0 ** -4 * out
+            hk = h // rep
+            _, _, w = attention_fwd(q8[b:b + 1, :, h:h + 1], k8[b:b + 1, :, hk:hk + 1],
+                                    v8[b:b + 1, :, hk:hk + 1], scale, mask, kv_offset, rows=rows,
+                                    return_weights=True)
+            yield b, h, w[0, 0], v8[b, :, hk, :]
+
+
+def p_rounding_bound(q, k, v, scale: float, mask: int = 0, kv_offset: int = 0, rows=None) -> np.ndarray:
+    """Per-element bound [B, R, Hq, d] on |O| error from rounding P to e4m3:
+    sum_j max(2^-4 w_j, 2^-10 w_max) |v_j| over the visible keys j."""
+    B, Lq, Hq, d = np.shape(q)
+    R = Lq if rows is None else len(rows)
+    out = np.zeros((B, R, Hq, d))
+    for b, h, w, v8 in _weights_and_v(q, k, v, scale, mask, kv_offset, rows):
+        wmax = w.max(axis=1, keepdims=True)
+        per_key = np.where(w > 0, np.maximum(2.0 ** -4 * w, 2.0 ** -10 * wmax), 0.0)
+        out[b, :, h, :] = per_key @ np.abs(v8)
+    return out
+
+
+def p_rounding_var(q, k, v, scale: float, mask: int = 0, kv_offset: int = 0, rows=None) -> np.ndarray:
+    """Per-element variance bound [B, R, Hq, d] of the O error from rounding P
+    to e4m3, errors independent and uniform over one e4m3 spacing:
+    sum_j max(2^-6 w_j^2, 2^-18 w_max^2) v_j^2 / 12 over the visible keys j."""
+    B, Lq, Hq, d = np.shape(q)
+    R = Lq if rows is None else len(rows)
+    out = np.zeros((B, R, Hq, d))
+    for b, h, w, v8 in _weights_and_v(q, k, v, scale, mask, kv_offset, rows):
+        wmax = w.max(axis=1, keepdims=True)
+        per_key = np.where(w > 0, np.maximum(2.0 ** -6 * w * w, 2.0 ** -18 * wmax * wmax), 0.0)
+        out[b, :, h, :] = per_key @ (v8 * v8) / 12.0
+    return out

@@ -173,3 +173,48 @@ def test_window_argument_contract(kw):
     st = hasb.lib().attn_fwd_window(A, A + 0x100000, A + 0x200000, A + 0x300000, None, 1, a["Lq"], 8, 2,
                                     1, 128, 0.1, a["wl"], a["wr"], a["off"], 0, None)
     assert st == hasb.ATTN_ERR_INVALID_ARG
+
+
+def _fp8_args(**kw):
+    a = dict(q=A, k=A + 0x100000, vt=A + 0x200000, o=A + 0x300000, lse=None, B=1, Lq=64, Lk=256,
+             pitch=256, Hq=2, Hkv=1, d=128, scale=0.1, mask=0, off=0)
+    a.update(kw)
+    return [a[n] for n in ("q", "k", "vt", "o", "lse", "B", "Lq", "Lk", "pitch", "Hq", "Hkv", "d",
+                           "scale", "mask", "off")] + [None]
+
+
+@pytest.mark.parametrize("kw", [dict(pitch=255), dict(pitch=240), dict(q=A + 8), dict(vt=A + 4),
+                                dict(Hq=3, Hkv=2), dict(mask=3), dict(mask=0, off=1),
+                                dict(mask=2, off=250), dict(scale=-1.0), dict(Lk=0),
+                                dict(o=A + 0x100000 + 64)])
+def test_fp8_attention_argument_contract(kw):
+    assert hasb.lib().attn_fwd_fp8(*_fp8_args(**kw)) == hasb.ATTN_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("d", [64, 256])
+def test_fp8_attention_other_head_dims_are_unsupported(d):
+    assert hasb.lib().attn_fwd_fp8(*_fp8_args(d=d)) == hasb.ATTN_ERR_UNSUPPORTED
+
+
+def test_fp8_cast_argument_contract():
+    L = hasb.lib()
+    assert L.attn_fp8_cast(A, A + 0x100000, 12, 0, None) == hasb.ATTN_ERR_INVALID_ARG   # n % 8
+    assert L.attn_fp8_cast(A + 8, A + 0x100000, 16, 0, None) == hasb.ATTN_ERR_INVALID_ARG  # x alignment
+    assert L.attn_fp8_cast(A, A + 0x100004, 16, 0, None) == hasb.ATTN_ERR_INVALID_ARG   # y alignment
+    assert L.attn_fp8_cast(A, A + 16, 16, 0, None) == hasb.ATTN_ERR_INVALID_ARG         # overlap
+    assert L.attn_fp8_cast(A, A + 0x100000, 16, 2, None) == hasb.ATTN_ERR_INVALID_ARG   # dtype
+    assert L.attn_fp8_cast(A, A + 0x100000, 0, 0, None) == hasb.ATTN_OK                 # empty: no launch
+    vt = [A, A + 0x100000]
+    assert L.attn_fp8_cast_vt(*vt, 1, 100, 1, 128, 96, 0, None) == hasb.ATTN_ERR_INVALID_ARG  # pitch < Lk
+    assert L.attn_fp8_cast_vt(*vt, 1, 100, 1, 128, 120, 0, None) == hasb.ATTN_ERR_INVALID_ARG  # pitch % 16
+    assert L.attn_fp8_cast_vt(*vt, 1, 100, 1, 96, 112, 0, None) == hasb.ATTN_ERR_INVALID_ARG   # d % 64
+    assert L.attn_fp8_cast_vt(A, A + 0x100, 1, 100, 1, 128, 112, 0, None) == hasb.ATTN_ERR_INVALID_ARG
+
+
+def test_fp8_binding_rejects_cpu_and_wrong_types():
+    import torch
+    q = torch.zeros(1, 4, 2, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        hasb.fp8_cast(q)
+    with pytest.raises(ValueError):
+        hasb.attn_fwd_fp8(q, q, q)

@@ -78,19 +78,57 @@ def test_fp8_attention_is_attention_of_the_cast_values():
     np.testing.assert_array_equal(a[0], c[0])
 
 
-@pytest.mark.parametrize("seed", [3, 4])
-def test_p_rounding_bound_covers_a_simulation(seed):
-    g = np.random.default_rng(seed)
-    q, k, v = (g.standard_normal(s) for s in ((1, 9, 2, 32), (1, 200, 2, 32), (1, 200, 2, 32)))
-    scale = 1 / np.sqrt(32)
-    o_exact, _ = fp8.attention_fp8(q, k, v, scale)
-    bound = fp8.p_rounding_bound(q, k, v, scale)
+def _simulate(q, k, v, scale, shift=0.0):
+    """O with P = e4m3(exp(s - m - shift)) and the unrounded row sum, m the row
+    max: the rounding the bounds describe, with the reference `shift` nats
+    below or above the max."""
     q8, k8, v8 = fp8.e4m3(q), fp8.e4m3(k), fp8.e4m3(v)
-    o_sim = np.zeros_like(o_exact)
-    for h in range(2):
-        s = scale * q8[0, :, h] @ k8[0, :, h].T
-        p = np.exp(s - s.max(axis=1, keepdims=True))
-        o_sim[0, :, h] = (fp8.e4m3(p) @ v8[0, :, h]) / p.sum(axis=1, keepdims=True)
+    o = np.zeros((q.shape[0], q.shape[1], q.shape[2], q.shape[3]))
+    rep = q.shape[2] // k.shape[2]
+    for b in range(q.shape[0]):
+        for h in range(q.shape[2]):
+            s = scale * q8[b, :, h] @ k8[b, :, h // rep].T
+            p = np.exp(s - s.max(axis=1, keepdims=True) - shift)
+            o[b, :, h] = (fp8.e4m3(p) @ v8[b, :, h // rep]) / p.sum(axis=1, keepdims=True)
+    return o
+
+
+@pytest.mark.parametrize("seed,scale,shift", [(3, 32 ** -0.5, 0.0), (4, 32 ** -0.5, 0.0),
+                                              (5, 1.5, 0.0), (6, 32 ** -0.5, 0.3)])
+def test_p_rounding_bound_and_variance_cover_a_simulation(seed, scale, shift):
+    """scale 1.5 spreads the scores so most weights fall below e4m3's smallest
+    normal (2^-6): the subnormal term of the bound is what covers them."""
+    g = np.random.default_rng(seed)
+    q, k, v = (g.standard_normal(s) for s in ((1, 9, 2, 32), (1, 400, 2, 32), (1, 400, 2, 32)))
+    o_exact, _ = fp8.attention_fp8(q, k, v, scale)
+    o_sim = _simulate(q, k, v, scale, shift)
+    bound = fp8.p_rounding_bound(q, k, v, scale)
+    var = fp8.p_rounding_var(q, k, v, scale)
     err = np.abs(o_sim - o_exact)
     assert np.all(err <= bound + 1e-12)
     assert err.max() > 0  # the rounding is visible, the bound is not vacuous
+    ratio = np.mean(err ** 2) / np.mean(var)
+    assert 0.02 < ratio <= 1.0, ratio  # the variance bound holds and is not loose by orders
+
+
+def test_subnormal_weights_need_the_absolute_term():
+    g = np.random.default_rng(5)
+    q, k, v = (g.standard_normal(s) for s in ((1, 9, 2, 32), (1, 400, 2, 32), (1, 400, 2, 32)))
+    o_exact, _, w = attention_fwd(fp8.e4m3(q), fp8.e4m3(k), fp8.e4m3(v), 1.5, MASK_NONE, 0,
+                                  return_weights=True)
+    rel_only = 2.0 ** -4 * np.einsum("bhrk,bkhd->brhd", w, np.abs(fp8.e4m3(v)))
+    err = np.abs(_simulate(q, k, v, 1.5) - o_exact)
+    assert np.any(err > rel_only)  # a relative-only bound would not hold here
+
+
+def test_bound_rows_are_the_rows_of_the_full_bound():
+    g = np.random.default_rng(7)
+    q, k, v = (g.standard_normal(s) for s in ((2, 20, 4, 16), (2, 30, 2, 16), (2, 30, 2, 16)))
+    rows = [0, 7, 19]
+    for mask, off in ((0, 0), (1, 10), (2, 5)):
+        full = fp8.p_rounding_bound(q, k, v, 0.4, mask, off)
+        part = fp8.p_rounding_bound(q, k, v, 0.4, mask, off, rows=rows)
+        np.testing.assert_allclose(part, full[:, rows], rtol=1e-12, atol=0)
+        fv = fp8.p_rounding_var(q, k, v, 0.4, mask, off)
+        pv = fp8.p_rounding_var(q, k, v, 0.4, mask, off, rows=rows)
+        np.testing.assert_allclose(pv, fv[:, rows], rtol=1e-12, atol=0)
