@@ -80,6 +80,9 @@ def parse_args():
     ap.add_argument("--window", default=None,
                     help="LEFT,RIGHT: time attn_fwd_window with this sliding window (-1 = unbounded "
                          "side) instead of attn_fwd; FLOPs count the visible (row, key) pairs")
+    ap.add_argument("--scaled", action="store_true",
+                    help="with --op fp8: per-token scaled codes (fp8_quantize_tokens for Q and K, "
+                         "fp8_quantize_vt for V) and attn_fwd_fp8_scaled")
     ap.add_argument("--splitkv", type=int, default=None,
                     help="time attn_fwd_splitkv with this many key ranges (0: chosen by the "
                          "library) instead of attn_fwd")
@@ -570,13 +573,29 @@ def run_fp8(args):
     lse = torch.empty((w.B, w.Hq, w.Lq), dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
 
-    def casts():
-        hasb.fp8_cast(q, out=q8)
-        hasb.fp8_cast(k, out=k8)
-        hasb.fp8_cast_vt(v, pitch=pitch, out=vt8)
+    spitch_q, spitch_k = (w.Lq + 3) // 4 * 4, (w.Lk + 3) // 4 * 4
+    sq = torch.empty((w.B, w.Hq, spitch_q), dtype=torch.float32, device="cuda")
+    sk = torch.empty((w.B, w.Hkv, spitch_k), dtype=torch.float32, device="cuda")
+    sv = torch.empty((w.B, w.Hkv, w.d), dtype=torch.float32, device="cuda")
 
-    def attend():
-        hasb.attn_fwd_fp8(q8, k8, vt8, scale=w.scale, causal=w.mask, kv_offset=w.kv_offset, out=o, lse=lse)
+    if args.scaled:
+        def casts():
+            hasb.fp8_quantize_tokens(q, out=q8, scales=sq)
+            hasb.fp8_quantize_tokens(k, out=k8, scales=sk)
+            hasb.fp8_quantize_vt(v, pitch=pitch, out=vt8, scales=sv)
+
+        def attend():
+            hasb.attn_fwd_fp8_scaled(q8, sq, k8, sk, vt8, sv, scale=w.scale, causal=w.mask,
+                                     kv_offset=w.kv_offset, out=o, lse=lse)
+    else:
+        def casts():
+            hasb.fp8_cast(q, out=q8)
+            hasb.fp8_cast(k, out=k8)
+            hasb.fp8_cast_vt(v, pitch=pitch, out=vt8)
+
+        def attend():
+            hasb.attn_fwd_fp8(q8, k8, vt8, scale=w.scale, causal=w.mask, kv_offset=w.kv_offset, out=o,
+                              lse=lse)
 
     for _ in range(max(3, args.warmup)):
         casts()
@@ -651,22 +670,27 @@ def run_fp8(args):
     achieved = flops / (statistics.mean(attn_ms) * 1e-3) / 1e12
     if rank == 0:
         line = {
-            "metric": "FP8 (e4m3) attention forward TFLOPS incl. the Q/K/V casts on 1 B200",
+            "metric": ("per-token scaled FP8 (e4m3) attention forward TFLOPS incl. the Q/K/V quantization"
+                       if args.scaled else
+                       "FP8 (e4m3) attention forward TFLOPS incl. the Q/K/V casts") + " on 1 B200",
             "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 (f32 accumulate, bf16 out)",
             "data": "synthetic: seeded N(0,1) inputs of the workload's shape",
             "config": dict(workload_config(w, world),
-                           step="fp8_cast(Q), fp8_cast(K), fp8_cast_vt(V), attn_fwd_fp8: all timed"),
+                           step=("fp8_quantize_tokens(Q), fp8_quantize_tokens(K), fp8_quantize_vt(V), "
+                                 "attn_fwd_fp8_scaled: all timed") if args.scaled else
+                                "fp8_cast(Q), fp8_cast(K), fp8_cast_vt(V), attn_fwd_fp8: all timed"),
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": None,
                          "traffic_source": "no ncu summary of the FP8 kernel",
                          "peak_source": ("2 x bf16_tflops_sustained" if capped else "2 x bf16_tflops (burst)")
                                         + f" of {peak_src} (nominal e4m3 / bf16 dense ratio)",
-                         "kernel": "attn_fwd_sm100_kernel (e4m3)",
+                         "kernel": "attn_fwd_sm100_kernel (e4m3" + (", per-token scales)" if args.scaled else ")"),
                          "launch_ms_mean": statistics.mean(attn_ms),
                          "casts_ms_mean": statistics.mean(step_ms) - statistics.mean(attn_ms)},
-            "cpu_baseline": None, "e2e": e2e, "gpu_launches": 4 * args.steps, "clocks": clock_info,
+            "cpu_baseline": None, "e2e": e2e, "gpu_launches": (6 if args.scaled else 4) * args.steps,
+            "clocks": clock_info,
             "device_fault_bits": hasb.device_fault(clear=True),
         }
         print(json.dumps(line))

@@ -63,6 +63,10 @@ _SIGNATURES = {
     "attn_fp8_cast_vt": (ctypes.c_int, [ctypes.c_void_p] * 2 + [ctypes.c_int] * 6 + [ctypes.c_void_p]),
     "attn_fwd_fp8": (ctypes.c_int, [ctypes.c_void_p] * 5 + [ctypes.c_int] * 7 +
                      [ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
+    "attn_fp8_quantize_tokens": (ctypes.c_int, [ctypes.c_void_p] * 3 + [ctypes.c_int] * 6 + [ctypes.c_void_p]),
+    "attn_fp8_quantize_vt": (ctypes.c_int, [ctypes.c_void_p] * 3 + [ctypes.c_int] * 6 + [ctypes.c_void_p]),
+    "attn_fwd_fp8_scaled": (ctypes.c_int, [ctypes.c_void_p] * 8 + [ctypes.c_int] * 9 +
+                            [ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
     "attn_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "attn_device_fault": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint), ctypes.c_int]),
     "attn_set_wait_timeout_ns": (ctypes.c_int, [ctypes.c_ulonglong]),
@@ -461,6 +465,101 @@ def attn_fwd_fp8(q8: torch.Tensor, k8: torch.Tensor, vt8: torch.Tensor, *, scale
                             _stream_handle(stream, q8.device))
     if st != ATTN_OK:
         raise AttnError(st, "attn_fwd_fp8")
+    return out, lse
+
+
+def fp8_quantize_tokens(x: torch.Tensor, *, s_pitch: int | None = None, out: torch.Tensor | None = None,
+                        scales: torch.Tensor | None = None, stream=None):
+    """Per-token scaled e4m3 codes of x [B, L, H, d] through
+    ``attn_fp8_quantize_tokens``. Returns (codes [B, L, H, d] float8_e4m3fn,
+    scales [B, H, s_pitch] float32; s_pitch defaults to L rounded up to 4)."""
+    _check_cuda("x", x, 4)
+    if x.dtype not in DTYPE_CODES:
+        raise ValueError("x must be bf16 or fp16")
+    B, L, H, d = x.shape
+    if s_pitch is None:
+        s_pitch = (L + 3) // 4 * 4
+    if out is None:
+        out = torch.empty(x.shape, dtype=E4M3, device=x.device)
+    elif out.dtype != E4M3 or out.shape != x.shape or not out.is_contiguous() or not out.is_cuda:
+        raise ValueError("out must be a contiguous float8_e4m3fn CUDA tensor shaped like x")
+    if scales is None:
+        scales = torch.empty((B, H, s_pitch), dtype=torch.float32, device=x.device)
+    elif (scales.dtype != torch.float32 or tuple(scales.shape) != (B, H, s_pitch)
+          or not scales.is_contiguous() or not scales.is_cuda):
+        raise ValueError("scales must be a contiguous float32 CUDA tensor [B, H, s_pitch]")
+    st = lib().attn_fp8_quantize_tokens(_ptr(x), _ptr(out), _ptr(scales), B, L, H, d, int(s_pitch),
+                                        DTYPE_CODES[x.dtype], _stream_handle(stream, x.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fp8_quantize_tokens")
+    return out, scales
+
+
+def fp8_quantize_vt(v: torch.Tensor, *, pitch: int | None = None, out: torch.Tensor | None = None,
+                    scales: torch.Tensor | None = None, stream=None):
+    """Per-channel scaled e4m3 codes of V [B, Lk, Hkv, d], transposed to
+    [B, Hkv, d, pitch], through ``attn_fp8_quantize_vt``. Returns (codes,
+    scales [B, Hkv, d] float32)."""
+    _check_cuda("v", v, 4)
+    if v.dtype not in DTYPE_CODES:
+        raise ValueError("v must be bf16 or fp16")
+    B, Lk, Hkv, d = v.shape
+    if pitch is None:
+        pitch = (Lk + 15) // 16 * 16
+    if out is None:
+        out = torch.empty((B, Hkv, d, pitch), dtype=E4M3, device=v.device)
+    elif (out.dtype != E4M3 or tuple(out.shape) != (B, Hkv, d, pitch) or not out.is_contiguous()
+          or not out.is_cuda):
+        raise ValueError("out must be a contiguous float8_e4m3fn CUDA tensor [B, Hkv, d, pitch]")
+    if scales is None:
+        scales = torch.empty((B, Hkv, d), dtype=torch.float32, device=v.device)
+    elif (scales.dtype != torch.float32 or tuple(scales.shape) != (B, Hkv, d) or not scales.is_contiguous()
+          or not scales.is_cuda):
+        raise ValueError("scales must be a contiguous float32 CUDA tensor [B, Hkv, d]")
+    st = lib().attn_fp8_quantize_vt(_ptr(v), _ptr(out), _ptr(scales), B, Lk, Hkv, d, int(pitch),
+                                    DTYPE_CODES[v.dtype], _stream_handle(stream, v.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fp8_quantize_vt")
+    return out, scales
+
+
+def attn_fwd_fp8_scaled(q8: torch.Tensor, sq: torch.Tensor, k8: torch.Tensor, sk: torch.Tensor,
+                        vt8: torch.Tensor, sv: torch.Tensor | None = None, *, scale: float | None = None,
+                        causal: int = MASK_NONE, kv_offset: int = 0, out: torch.Tensor | None = None,
+                        lse: torch.Tensor | None = None, return_lse: bool = True, stream=None):
+    """Per-token scaled FP8 attention through ``attn_fwd_fp8_scaled``: codes
+    and scales as ``fp8_quantize_tokens`` (Q, K) and ``fp8_quantize_vt`` (V;
+    sv None: V cast without scales by ``fp8_cast_vt``). Returns ``(out, lse)``."""
+    for name, t in (("q8", q8), ("k8", k8), ("vt8", vt8)):
+        _check_cuda(name, t, 4)
+        if t.dtype != E4M3:
+            raise ValueError(f"{name} must be float8_e4m3fn")
+    B, Lq, Hq, d = q8.shape
+    Bk, Lk, Hkv, dk = k8.shape
+    if Bk != B or dk != d or tuple(vt8.shape[:3]) != (B, Hkv, d):
+        raise ValueError("q8, k8, vt8 shapes disagree")
+    for name, t, lead in (("sq", sq, (B, Hq)), ("sk", sk, (B, Hkv))):
+        _check_cuda(name, t, 3)
+        if t.dtype != torch.float32 or tuple(t.shape[:2]) != lead:
+            raise ValueError(f"{name} must be float32 [{lead[0]}, {lead[1]}, pitch]")
+    if sv is not None:
+        _check_cuda("sv", sv, 3)
+        if sv.dtype != torch.float32 or tuple(sv.shape) != (B, Hkv, d):
+            raise ValueError("sv must be float32 [B, Hkv, d]")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((B, Lq, Hq, d), dtype=torch.bfloat16, device=q8.device)
+    elif (out.dtype != torch.bfloat16 or tuple(out.shape) != (B, Lq, Hq, d) or not out.is_contiguous()
+          or not out.is_cuda):
+        raise ValueError("out must be a contiguous bf16 CUDA tensor [B, Lq, Hq, d]")
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q8.device)
+    st = lib().attn_fwd_fp8_scaled(_ptr(q8), _ptr(k8), _ptr(vt8), _ptr(sq), _ptr(sk), _ptr(sv), _ptr(out),
+                                   _ptr(lse), B, Lq, Lk, vt8.shape[3], sq.shape[2], sk.shape[2], Hq, Hkv, d,
+                                   float(scale), int(causal), int(kv_offset), _stream_handle(stream, q8.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fwd_fp8_scaled")
     return out, lse
 
 

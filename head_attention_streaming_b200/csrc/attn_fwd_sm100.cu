@@ -67,7 +67,7 @@ constexpr float kRescaleTau = 8.0f;    // lazy rescale threshold, log2 units (P 
 constexpr float kLn2 = 0.69314718055994531f;
 constexpr float kLog2e = 1.4426950408889634f;
 
-template <int D, bool F8 = false>
+template <int D, int F8 = 0>
 struct Cfg {
   static constexpr int kChunks = D / 64;              // 128-byte swizzle chunks per row
   static constexpr int kChunkBytes = kTileRows * 128;  // one chunk of a 128-row tile
@@ -84,29 +84,37 @@ struct Cfg {
   static constexpr uint32_t kTmemCols = 512;
   static constexpr int kOChunks = D / 64;  // 64-column chunks of the 16-bit O staging tile
   static constexpr int kOffP = 0;          // P lives in tensor memory
+  static constexpr int kOffSk = 0;         // no key scales
 };
 
 // e4m3 operands, d = 128: a Q / K row is one 128-byte swizzle chunk (16 KB per
 // 128-row tile), V arrives transposed (a tile is 128 d-rows of 128 keys) so
 // both P V operands are K-major, and P goes through shared memory (two 16 KB
-// buffers, K-major with the same swizzle) instead of tensor memory.
-template <>
-struct Cfg<128, true> {
+// buffers, K-major with the same swizzle) instead of tensor memory. MODE 2
+// (per-token scales) adds one 512-byte buffer of key scales per softmax warp
+// and gives up one ring stage for it.
+template <int MODE>
+struct CfgE4m3 {
   static constexpr int kChunks = 1;
   static constexpr int kChunkBytes = kTileRows * 128;
   static constexpr int kTileBytes = kTileRows * 128;
-  static constexpr int kStages = 8;
+  static constexpr int kStages = MODE == 2 ? 7 : 8;
   static constexpr int kOChunks = 2;
   static constexpr int kOffQ = 0;
   static constexpr int kOffKV = 2 * kTileBytes;
   static constexpr int kOffP = kOffKV + kStages * kTileBytes;
   static constexpr int kOffStg = kOffP + 2 * kTileBytes;
-  static constexpr int kOffBar = kOffStg + kOChunks * kChunkBytes;
+  static constexpr int kOffSk = kOffStg + kOChunks * kChunkBytes;
+  static constexpr int kOffBar = kOffSk + (MODE == 2 ? 8 * 512 : 0);
   static constexpr int kSmemBytes = kOffBar + 512 + 1024;
   static __device__ __forceinline__ uint32_t col_s(int t) { return t ? 128u : 0u; }
   static __device__ __forceinline__ uint32_t col_o(int t) { return t ? 384u : 256u; }
   static constexpr uint32_t kTmemCols = 512;
 };
+template <>
+struct Cfg<128, 1> : CfgE4m3<1> {};
+template <>
+struct Cfg<128, 2> : CfgE4m3<2> {};
 
 // barrier slots (8 bytes each) in the barrier area
 enum Bar : int {
@@ -130,6 +138,14 @@ enum Bar : int {
 // the MUFU, so the default is 0; the polynomial stays available (and tested)
 // for shapes where the MUFU saturates.
 constexpr int kPolyPairsPer8 = POLY_PAIRS_PER8;
+// The same split for the e4m3 path, whose GEMMs take half the time.
+#ifndef F8_PACKED_KEY_SCALE
+#define F8_PACKED_KEY_SCALE 1
+#endif
+#ifndef F8_POLY_PAIRS_PER8
+#define F8_POLY_PAIRS_PER8 0
+#endif
+constexpr int kF8PolyPairsPer8 = F8_POLY_PAIRS_PER8;
 
 // 2^x for a pair of floats on the FMA pipe: x = j + f with j = round(x) and
 // f in [-1/2, 1/2]; 2^f from a degree-3 polynomial minimising the maximum
@@ -177,6 +193,13 @@ struct FwdParams {
   // sliding window (left, right; -1 = unbounded): row i sees keys
   // p - left <= j <= p + right, p = kv_offset + i
   int win_left, win_right;
+  // per-token scaled e4m3: the score of (row i, key j) is
+  // scale * sq[b, hq, i] * sk[b, hkv, j] * (q8_i . k8_j); O column c is
+  // multiplied by sv[b, hkv, c] (nullptr: 1)
+  const float* sq;
+  const float* sk;
+  const float* sv;
+  int sq_pitch, sk_pitch;
 };
 
 // KV tiles of a work unit: the loader streams tiles j0 .. j0 + nu - 1 (the
@@ -343,7 +366,7 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint3
   issue_pv_half<D, BF16, 1>(d_tmem, p_tmem, v_lo, 1u);
 }
 
-template <int D, bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW, bool F8>
+template <int D, bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW, int F8>
 __device__ __forceinline__ void load_role(const CUtensorMap* tm_q, const CUtensorMap* tm_k,
                                           const CUtensorMap* tm_v, const FwdParams& p,
                                           uint32_t sQ, uint32_t sKV, uint32_t bars,
@@ -379,7 +402,7 @@ __device__ __forceinline__ void load_role(const CUtensorMap* tm_q, const CUtenso
         }
         const uint32_t bf = bars + 8 * (kBarKvFull + slot);
         mbar_arrive_expect_tx(bf, C::kTileBytes);
-        if constexpr (F8) {
+        if constexpr (F8 != 0) {
           // K: (d, head, key, batch); transposed V: (key, d, head, batch)
           if (kv)
             tma_load_4d(sKV + slot * C::kTileBytes, tm_v, bf, (x.j0 + j) * kTileRows, 0, x.hkv, x.b,
@@ -413,7 +436,7 @@ __device__ __forceinline__ void load_role(const CUtensorMap* tm_q, const CUtenso
 // issuing the other's GEMMs. With one thread per tile, the tensor core runs
 // whichever tile has work. Both threads read the same K/V ring slots; each slot
 // use is released by both (kv_empty takes two arrivals).
-template <int D, bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW, bool F8>
+template <int D, bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW, int F8>
 __device__ __forceinline__ void mma_role(const int t, const FwdParams& p, uint32_t tmem, uint32_t sQ,
                                          uint32_t sKV, uint32_t sP, uint32_t bars,
                                          volatile int* abort_flag) {
@@ -456,7 +479,7 @@ __device__ __forceinline__ void mma_role(const int t, const FwdParams& p, uint32
     ok = ok && kv_full(kb);
     if (!ok) break;
     // S_t(0) = Q_t K_0^T
-    if constexpr (F8) issue_qk_f8<D>(s_t, q_lo, k_lo(kb));
+    if constexpr (F8 != 0) issue_qk_f8<D>(s_t, q_lo, k_lo(kb));
     else issue_qk<D, BF16>(s_t, q_lo, k_lo(kb));
     mma_commit(bar(kBarSFull + t));
     mma_commit(bar(kBarKvEmpty + kb % C::kStages));
@@ -472,7 +495,7 @@ __device__ __forceinline__ void mma_role(const int t, const FwdParams& p, uint32
         break;
       }
       tc_fence_after_sync();
-      if constexpr (F8) issue_pv_half_f8<D, 0>(o_t, p_lo, k_lo(vidx), j > 0 ? 1u : 0u);
+      if constexpr (F8 != 0) issue_pv_half_f8<D, 0>(o_t, p_lo, k_lo(vidx), j > 0 ? 1u : 0u);
       else issue_pv_half<D, BF16, 0>(o_t, s_t, v_lo(vidx), j > 0 ? 1u : 0u);
       if (!mbar_wait(bar(kBarPFull + t), pcnt & 1, abort_flag, kFaultMmaPFull, p.timeout_ns)) {
         ok = false;
@@ -480,14 +503,14 @@ __device__ __forceinline__ void mma_role(const int t, const FwdParams& p, uint32
       }
       ++pcnt;
       tc_fence_after_sync();
-      if constexpr (F8) issue_pv_half_f8<D, 1>(o_t, p_lo, k_lo(vidx), 1u);
+      if constexpr (F8 != 0) issue_pv_half_f8<D, 1>(o_t, p_lo, k_lo(vidx), 1u);
       else issue_pv_half<D, BF16, 1>(o_t, s_t, v_lo(vidx), 1u);
       mma_commit(bar(kBarKvEmpty + vidx % C::kStages));
       if (j == n - 1) {
         mma_commit(bar(kBarOFull + t));
       } else {
         if (!kv_full(knext)) { ok = false; break; }
-        if constexpr (F8) issue_qk_f8<D>(s_t, q_lo, k_lo(knext));
+        if constexpr (F8 != 0) issue_qk_f8<D>(s_t, q_lo, k_lo(knext));
         else issue_qk<D, BF16>(s_t, q_lo, k_lo(knext));
         mma_commit(bar(kBarSFull + t));
         mma_commit(bar(kBarKvEmpty + knext % C::kStages));
@@ -539,12 +562,24 @@ __device__ __forceinline__ void exp_tile_f8(const uint32_t (&r)[128], float sl2,
     for (int cc = 0; cc < 16; ++cc) {
       float pv[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int c = 64 * h + 4 * cc + e;
-        float pe = ex2_approx(fmaf(__uint_as_float(r[c]), sl2, nref));
-        if (MASKED) pe = (c < lim && c >= lim_lo) ? pe : 0.f;
-        sum[e] += pe;
-        pv[e] = pe;
+      for (int pr = 0; pr < 2; ++pr) {
+        const int c = 64 * h + 4 * cc + 2 * pr;
+        float p0, p1;
+        if (((2 * cc + pr) & 7) >= 8 - kF8PolyPairsPer8) {
+          f2_unpack(exp2_poly_x2(f2_pack(fmaf(__uint_as_float(r[c]), sl2, nref),
+                                         fmaf(__uint_as_float(r[c + 1]), sl2, nref))), p0, p1);
+        } else {
+          p0 = ex2_approx(fmaf(__uint_as_float(r[c]), sl2, nref));
+          p1 = ex2_approx(fmaf(__uint_as_float(r[c + 1]), sl2, nref));
+        }
+        if (MASKED) {
+          p0 = (c < lim && c >= lim_lo) ? p0 : 0.f;
+          p1 = (c + 1 < lim && c + 1 >= lim_lo) ? p1 : 0.f;
+        }
+        sum[2 * pr] += p0;
+        sum[2 * pr + 1] += p1;
+        pv[2 * pr] = p0;
+        pv[2 * pr + 1] = p1;
       }
       w[cc] = pack_e4m3x2(pv[0], pv[1]) | (pack_e4m3x2(pv[2], pv[3]) << 16);
     }
@@ -564,6 +599,18 @@ __device__ __forceinline__ void exp_tile_f8(const uint32_t (&r)[128], float sl2,
     __syncwarp();
     if (lane == 0) mbar_arrive(h == 0 ? bar_half : bar_full);
   }
+}
+
+// Four key scales of one 128-key tile (keys key .. key + 3 of a per-head
+// scale row; keys >= Lk read as 0: they are masked anyway).
+__device__ __forceinline__ float4 load_key_scales(const float* row, int key, int Lk) {
+  if (key + 3 < Lk) return __ldg(reinterpret_cast<const float4*>(row + key));
+  float4 v;
+  v.x = key < Lk ? __ldg(row + key) : 0.f;
+  v.y = key + 1 < Lk ? __ldg(row + key + 1) : 0.f;
+  v.z = key + 2 < Lk ? __ldg(row + key + 2) : 0.f;
+  v.w = 0.f;
+  return v;
 }
 
 template <bool BF16, bool MASKED>
@@ -609,7 +656,7 @@ __device__ __forceinline__ void exp_tile(const uint32_t (&r)[128], float sl2, fl
 // buffer to global memory with a TMA store (rows past Lq are clipped by the
 // tensor map), then hands the buffer to the other query tile. Order per unit:
 // tile 0, then tile 1, the same order the softmax warpgroups fill it in.
-template <int D, bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW, bool F8>
+template <int D, bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW, int F8>
 __device__ __forceinline__ void store_role(const CUtensorMap* tm_o, const FwdParams& p, uint32_t sStg,
                                            uint32_t bars, volatile int* abort_flag) {
   using C = Cfg<D, F8>;
@@ -632,12 +679,14 @@ __device__ __forceinline__ void store_role(const CUtensorMap* tm_o, const FwdPar
   bulk_wait_group0();  // every store complete before the CTA exits
 }
 
-template <int D, bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW, bool F8>
+template <int D, bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW, int F8>
 __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, uint32_t tmem,
-                                             uint32_t bars, uint32_t sstg, uint32_t sP,
+                                             uint32_t bars, uint32_t sstg, uint32_t sP, uint32_t sSk,
                                              volatile int* abort_flag) {
   using C = Cfg<D, F8>;
   const uint32_t prow = sP + t * C::kTileBytes + (threadIdx.x % kTileRows) * 128;  // e4m3 P row
+  // per-token scales: this warp's copy of the current KV tile's 128 key scales
+  const uint32_t skw = sSk + (threadIdx.x / 32) * 512;
   const int warp = threadIdx.x / 32;
   const int r_in = threadIdx.x % kTileRows;                      // row in tile = TMEM lane
   const uint32_t lane_bits = static_cast<uint32_t>((warp % 4) * 32) << 16;
@@ -672,8 +721,25 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
     }
     float ref = -INFINITY;  // scaled (log2) max the exponentials are taken against
     float l = 0.f;          // running row sum of exp2(s * sl2 - ref)
+    // per-token scales: the row's Q scale joins the log2 factor; each lane
+    // fetches 4 of the next KV tile's key scales one tile ahead
+    float sl2r = sl2;
+    const float* skrow = nullptr;
+    float4 skv = make_float4(0.f, 0.f, 0.f, 0.f);
+    if constexpr (F8 == 2) {
+      const size_t qs = (static_cast<size_t>(x.b) * p.Hq + x.hq) * p.sq_pitch + row;
+      sl2r = sl2 * (row < p.Lq ? __ldg(p.sq + qs) : 1.f);
+      skrow = p.sk + (static_cast<size_t>(x.b) * p.Hkv + x.hkv) * p.sk_pitch;
+      skv = load_key_scales(skrow, (x.j0 + s) * kTileRows + 4 * lane, p.Lk);
+    }
 
     for (int j = 0; j < n; ++j) {
+      if constexpr (F8 == 2) {
+        __syncwarp();  // every lane is done with the previous tile's scales
+        st_shared_v4f(skw + 16 * lane, skv);
+        __syncwarp();
+        if (j + 1 < n) skv = load_key_scales(skrow, (x.j0 + s + j + 1) * kTileRows + 4 * lane, p.Lk);
+      }
       bool ok = mbar_wait(bar_s, scnt & 1, abort_flag, kFaultSoftmaxSFull, p.timeout_ns);
       if (!__all_sync(0xffffffffu, ok)) return;
       ++scnt;
@@ -684,6 +750,28 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
       for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(tS + 32 * c, r + 32 * c);
       tmem_wait_ld_x128(r);
 
+      if constexpr (F8 == 2) {
+        // raw code product times the key's scale (before masking: an invisible
+        // key's -inf must not meet a scale)
+#pragma unroll
+        for (int c = 0; c < 128; c += 4) {
+          const float4 k4 = ld_shared_v4f(skw + 4 * c);
+#if F8_PACKED_KEY_SCALE
+          float a0, a1, a2, a3;
+          f2_unpack(f2_mul(f2_pack_bits(r[c], r[c + 1]), f2_pack(k4.x, k4.y)), a0, a1);
+          f2_unpack(f2_mul(f2_pack_bits(r[c + 2], r[c + 3]), f2_pack(k4.z, k4.w)), a2, a3);
+          r[c] = __float_as_uint(a0);
+          r[c + 1] = __float_as_uint(a1);
+          r[c + 2] = __float_as_uint(a2);
+          r[c + 3] = __float_as_uint(a3);
+#else
+          r[c] = __float_as_uint(__uint_as_float(r[c]) * k4.x);
+          r[c + 1] = __float_as_uint(__uint_as_float(r[c + 1]) * k4.y);
+          r[c + 2] = __float_as_uint(__uint_as_float(r[c + 2]) * k4.z);
+          r[c + 3] = __float_as_uint(__uint_as_float(r[c + 3]) * k4.w);
+#endif
+        }
+      }
       const int key0 = (x.j0 + s + j) * kTileRows;  // first key of this tile
       const int lim = row_lim - key0;                // keys c < lim of this tile are visible ...
       const int lim_lo = WINDOW ? row_lo - key0 : 0;  // ... and c >= lim_lo
@@ -710,7 +798,7 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
         for (int i = 0; i < 5; ++i) c5[i] = fmax3(b[3 * i], b[3 * i + 1], b[3 * i + 2]);
         m_tile = fmaxf(fmax3(c5[0], c5[1], c5[2]), fmaxf(c5[3], c5[4]));
       }
-      const float m_scaled = (m_tile == -INFINITY) ? -INFINITY : m_tile * sl2;
+      const float m_scaled = (m_tile == -INFINITY) ? -INFINITY : m_tile * sl2r;
 
       // lazy rescale: move the reference only when the max grew by > tau; after
       // the first tiles of a row this almost never fires, so the warp takes the
@@ -767,12 +855,12 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
       // (tcgen05.st, __syncwarp), so the choice must be the same for the whole
       // warp: rows of one warp can differ (causal), and a lane whose keys are
       // all visible is unaffected by the masked variant.
-      if constexpr (F8) {
+      if constexpr (F8 != 0) {
         if (__any_sync(0xffffffffu, partial)) {
-          exp_tile_f8<true>(r, sl2, nref, lim, lim_lo, sum, prow, r_in, bar_ph, bar_p, bar_turn_other,
+          exp_tile_f8<true>(r, sl2r, nref, lim, lim_lo, sum, prow, r_in, bar_ph, bar_p, bar_turn_other,
                             hand_over, lane);
         } else {
-          exp_tile_f8<false>(r, sl2, nref, lim, lim_lo, sum, prow, r_in, bar_ph, bar_p, bar_turn_other,
+          exp_tile_f8<false>(r, sl2r, nref, lim, lim_lo, sum, prow, r_in, bar_ph, bar_p, bar_turn_other,
                              hand_over, lane);
         }
       } else if (__any_sync(0xffffffffu, partial)) {
@@ -832,6 +920,20 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
       uint32_t ov[32];
       tmem_ld_32x32b_x32(tO + 32 * c, ov);
       tmem_wait_ld_x32(ov);
+      if constexpr (F8 == 2) {
+        if (p.sv != nullptr) {  // V's per-channel scales
+          const float4* sv4 =
+              reinterpret_cast<const float4*>(p.sv + (static_cast<size_t>(x.b) * p.Hkv + x.hkv) * D + 32 * c);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float4 f = __ldg(sv4 + e);
+            ov[4 * e] = __float_as_uint(__uint_as_float(ov[4 * e]) * f.x);
+            ov[4 * e + 1] = __float_as_uint(__uint_as_float(ov[4 * e + 1]) * f.y);
+            ov[4 * e + 2] = __float_as_uint(__uint_as_float(ov[4 * e + 2]) * f.z);
+            ov[4 * e + 3] = __float_as_uint(__uint_as_float(ov[4 * e + 3]) * f.w);
+          }
+        }
+      }
       uint32_t pk[16];
 #pragma unroll
       for (int e = 0; e < 16; ++e)
@@ -855,7 +957,7 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
   }
 }
 
-template <int D, bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW, bool F8>
+template <int D, bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW, int F8>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
@@ -922,7 +1024,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < 8) {
     regs_increase<kRegsSoftmax>();
-    softmax_role<D, BF16, CAUSAL, SPLIT, WINDOW, F8>(warp / 4, p, tmem, bars, sStg, sP, abort_flag);
+    softmax_role<D, BF16, CAUSAL, SPLIT, WINDOW, F8>(warp / 4, p, tmem, bars, sStg, sP, sbase + C::kOffSk,
+                                                     abort_flag);
   } else {
     regs_decrease<kRegsProducer>();
     if (warp == 8) {
@@ -1208,12 +1311,12 @@ bool encode_e4m3_vt(CUtensorMap* map, const void* ptr, int B, int Lk, int pitch,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, bool BF16, bool CAUSAL, bool SPLIT = false, bool WINDOW = false, bool F8 = false>
+template <int D, bool BF16, bool CAUSAL, bool SPLIT = false, bool WINDOW = false, int F8 = 0>
 int launch_fwd(const FwdParams& p, const void* q, const void* k, const void* v, int kv_rows, int grid,
                cudaStream_t stream) {
   using C = Cfg<D, F8>;
   CUtensorMap tq, tk, tv, to;
-  if constexpr (F8) {
+  if constexpr (F8 != 0) {
     // e4m3 Q / K (box: the 128-byte row of a head, 128 rows); V transposed,
     // [B, Hkv, d, kv_rows] bytes with kv_rows a multiple of 16 (box: 128 keys
     // x 128 d-rows); O bf16 as usual
@@ -1350,7 +1453,7 @@ int attn_fwd_impl(const void* q, const void* k, const void* v, void* o, float* l
   if (!di.ok) return ATTN_ERR_CUDA;
   if (!di.sm100) return ATTN_ERR_UNSUPPORTED;
 
-  FwdParams p;
+  FwdParams p{};
   p.o = o;
   p.lse = lse;
   p.B = B; p.Lq = Lq; p.Lk = Lk; p.Hq = Hq; p.Hkv = Hkv; p.group = Hq / Hkv;
@@ -1471,7 +1574,7 @@ int splitkv_run(const void* q, const void* k, const void* v, void* o, float* lse
     return ATTN_ERR_INVALID_ARG;
   if (base_units * ns > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
 
-  FwdParams p;
+  FwdParams p{};
   p.o = o;
   p.lse = lse;
   p.B = B; p.Lq = Lq; p.Lk = Lk; p.Hq = Hq; p.Hkv = Hkv; p.group = Hq / Hkv;
@@ -1529,9 +1632,15 @@ int attn_fwd_window(const void* q, const void* k, const void* v, void* o, float*
                        dtype, stream, true, window_left, window_right);
 }
 
-int attn_fwd_fp8(const void* q8, const void* k8, const void* vt8, void* o, float* lse, int B, int Lq,
-                 int Lk, int vt_pitch, int Hq, int Hkv, int d, float scale, int causal, int kv_offset,
-                 void* stream) {
+}  // extern "C"
+
+namespace hasb {
+
+// Both e4m3 entry points: unscaled (sq == sk == nullptr) and per-token scaled.
+int fp8_fwd(const void* q8, const void* k8, const void* vt8, const float* sq, const float* sk,
+            const float* sv, int sq_pitch, int sk_pitch, void* o, float* lse, int B, int Lq, int Lk,
+            int vt_pitch, int Hq, int Hkv, int d, float scale, int causal, int kv_offset, void* stream,
+            bool scaled) {
   // ---- argument contract (no CUDA call before it passes)
   if (q8 == nullptr || k8 == nullptr || vt8 == nullptr || o == nullptr) return ATTN_ERR_INVALID_ARG;
   if (B < 1 || Lq < 1 || Lk < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
@@ -1556,6 +1665,17 @@ int attn_fwd_fp8(const void* q8, const void* k8, const void* vt8, void* o, float
   if (ranges_overlap(o, q_elems * 2, q8, q_elems) || ranges_overlap(o, q_elems * 2, k8, k_elems) ||
       ranges_overlap(o, q_elems * 2, vt8, vt_bytes))
     return ATTN_ERR_INVALID_ARG;
+  if (scaled) {
+    if (sq == nullptr || sk == nullptr) return ATTN_ERR_INVALID_ARG;
+    if (sq_pitch < Lq || sk_pitch < Lk || sk_pitch % 4 != 0) return ATTN_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(sq) & 3u) != 0 || !a16(sk) || (sv != nullptr && !a16(sv)))
+      return ATTN_ERR_INVALID_ARG;
+    const unsigned long long sq_bytes = 4ull * B * Hq * sq_pitch, sk_bytes = 4ull * B * Hkv * sk_pitch;
+    if (sq_bytes >= (1ull << 40) || sk_bytes >= (1ull << 40)) return ATTN_ERR_INVALID_ARG;
+    if (ranges_overlap(o, q_elems * 2, sq, sq_bytes) || ranges_overlap(o, q_elems * 2, sk, sk_bytes) ||
+        (sv != nullptr && ranges_overlap(o, q_elems * 2, sv, 4ull * B * Hkv * d)))
+      return ATTN_ERR_INVALID_ARG;
+  }
   if (d != 128) return ATTN_ERR_UNSUPPORTED;
   // ---- device
   int dev = 0;
@@ -1563,7 +1683,7 @@ int attn_fwd_fp8(const void* q8, const void* k8, const void* vt8, void* o, float
   const DeviceInfo di = device_info(dev);
   if (!di.ok) return ATTN_ERR_CUDA;
   if (!di.sm100) return ATTN_ERR_UNSUPPORTED;
-  FwdParams p;
+  FwdParams p{};
   p.o = o;
   p.lse = lse;
   p.B = B; p.Lq = Lq; p.Lk = Lk; p.Hq = Hq; p.Hkv = Hkv; p.group = Hq / Hkv;
@@ -1578,11 +1698,38 @@ int attn_fwd_fp8(const void* q8, const void* k8, const void* vt8, void* o, float
   p.o_part = nullptr;
   p.lse_part = nullptr;
   p.win_left = p.win_right = -1;
+  p.sq = sq;
+  p.sk = sk;
+  p.sv = sv;
+  p.sq_pitch = sq_pitch;
+  p.sk_pitch = sk_pitch;
   const int grid = static_cast<int>(n_units < di.num_sms ? n_units : di.num_sms);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return causal == ATTN_MASK_CAUSAL
-             ? launch_fwd<128, true, true, false, false, true>(p, q8, k8, vt8, vt_pitch, grid, s)
-             : launch_fwd<128, true, false, false, false, true>(p, q8, k8, vt8, vt_pitch, grid, s);
+  const bool c = causal == ATTN_MASK_CAUSAL;
+  if (scaled)
+    return c ? launch_fwd<128, true, true, false, false, 2>(p, q8, k8, vt8, vt_pitch, grid, s)
+             : launch_fwd<128, true, false, false, false, 2>(p, q8, k8, vt8, vt_pitch, grid, s);
+  return c ? launch_fwd<128, true, true, false, false, 1>(p, q8, k8, vt8, vt_pitch, grid, s)
+           : launch_fwd<128, true, false, false, false, 1>(p, q8, k8, vt8, vt_pitch, grid, s);
+}
+
+}  // namespace hasb
+
+extern "C" {
+
+int attn_fwd_fp8(const void* q8, const void* k8, const void* vt8, void* o, float* lse, int B, int Lq,
+                 int Lk, int vt_pitch, int Hq, int Hkv, int d, float scale, int causal, int kv_offset,
+                 void* stream) {
+  return hasb::fp8_fwd(q8, k8, vt8, nullptr, nullptr, nullptr, 0, 0, o, lse, B, Lq, Lk, vt_pitch, Hq,
+                       Hkv, d, scale, causal, kv_offset, stream, false);
+}
+
+int attn_fwd_fp8_scaled(const void* q8, const void* k8, const void* vt8, const float* sq,
+                        const float* sk, const float* sv, void* o, float* lse, int B, int Lq, int Lk,
+                        int vt_pitch, int sq_pitch, int sk_pitch, int Hq, int Hkv, int d, float scale,
+                        int causal, int kv_offset, void* stream) {
+  return hasb::fp8_fwd(q8, k8, vt8, sq, sk, sv, sq_pitch, sk_pitch, o, lse, B, Lq, Lk, vt_pitch, Hq,
+                       Hkv, d, scale, causal, kv_offset, stream, true);
 }
 
 int attn_fwd_cache(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,

@@ -233,6 +233,21 @@ __device__ __forceinline__ void mma_f8_ss_lo_flag(uint32_t d_tmem, uint32_t a_lo
       : "memory");
 }
 
+__device__ __forceinline__ void st_shared_v4f(uint32_t addr, float4 v) {
+  asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x), "f"(v.y), "f"(v.z),
+               "f"(v.w)
+               : "memory");
+}
+
+__device__ __forceinline__ float4 ld_shared_v4f(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+
 // Two floats to two e4m3 bytes, round to nearest even, saturating at +-448:
 // lo in bits 0-7, hi in bits 8-15.
 __device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {

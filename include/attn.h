@@ -125,6 +125,39 @@ int attn_fwd_fp8(const void* q8, const void* k8, const void* vt8, void* o, float
                  void* stream);
 
 /*
+ * Per-token scaled FP8 attention (developer guide, "Quantization Toolkit":
+ * slice scales s = max(max |x| / 448, eps) in float32 with eps = 2^-126,
+ * codes e4m3(x / s) clipped to +-448; "Quantized GEMM", inner-dimension rule:
+ * the scales of each GEMM operand stay constant along its reduction axis).
+ *
+ * attn_fp8_quantize_tokens — one scale per (batch, token, head) of x
+ * [B, L, H, d] (16-bit, dtype): s[b, h, l] at s[(b H + h) s_pitch + l]
+ * (float32, s_pitch >= L), codes y [B, L, H, d] e4m3. d a power of two in
+ * 16..256; x 16-byte, y 8-byte, s 4-byte aligned; no overlap.
+ *
+ * attn_fp8_quantize_vt — one scale per (batch, head, channel) of V
+ * [B, Lk, Hkv, d] (the max runs over the keys): sv [B, Hkv, d] float32, codes
+ * written transposed like attn_fp8_cast_vt ([B, Hkv, d, pitch]). d a power of
+ * two in 64..256. Four launches on `stream` (zero sv, column maxima, codes,
+ * maxima to scales); sv holds the scales once they complete.
+ *
+ * attn_fwd_fp8_scaled — attn_fwd_fp8 on scaled codes: the score of row i and
+ * key j is scale * sq[b, hq, i] * sk[b, hkv, j] * (q8_i . k8_j) (sq
+ * [B, Hq, sq_pitch], sk [B, Hkv, sk_pitch] as attn_fp8_quantize_tokens writes
+ * them, sk_pitch a multiple of 4, sk 16-byte aligned), and column c of O is
+ * multiplied by sv[b, hkv, c] ([B, Hkv, d], 16-byte aligned; NULL: V cast
+ * without scales). P is rounded to e4m3 as in attn_fwd_fp8. d = 128.
+ */
+int attn_fp8_quantize_tokens(const void* x, void* y, float* s, int B, int L, int H, int d, int s_pitch,
+                             int dtype, void* stream);
+int attn_fp8_quantize_vt(const void* v, void* vt, float* sv, int B, int Lk, int Hkv, int d, int pitch,
+                         int dtype, void* stream);
+int attn_fwd_fp8_scaled(const void* q8, const void* k8, const void* vt8, const float* sq,
+                        const float* sk, const float* sv, void* o, float* lse, int B, int Lq, int Lk,
+                        int vt_pitch, int sq_pitch, int sk_pitch, int Hq, int Hkv, int d, float scale,
+                        int causal, int kv_offset, void* stream);
+
+/*
  * attn_fwd_cache — attn_fwd with K and V read from the first Lk tokens of a
  * [B, S, Hkv, d] cache (the rolling block cache of streaming self-attention,
  * whose valid tokens are a prefix of its S slots): batch b's keys start at

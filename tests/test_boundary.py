@@ -218,3 +218,36 @@ def test_fp8_binding_rejects_cpu_and_wrong_types():
         hasb.fp8_cast(q)
     with pytest.raises(ValueError):
         hasb.attn_fwd_fp8(q, q, q)
+
+
+def _fp8s_args(**kw):
+    a = dict(q=A, k=A + 0x100000, vt=A + 0x200000, sq=A + 0x500000, sk=A + 0x600000, sv=A + 0x700000,
+             o=A + 0x300000, lse=None, B=1, Lq=64, Lk=256, pitch=256, sqp=64, skp=256, Hq=2, Hkv=1,
+             d=128, scale=0.1, mask=0, off=0)
+    a.update(kw)
+    return [a[n] for n in ("q", "k", "vt", "sq", "sk", "sv", "o", "lse", "B", "Lq", "Lk", "pitch", "sqp",
+                           "skp", "Hq", "Hkv", "d", "scale", "mask", "off")] + [None]
+
+
+@pytest.mark.parametrize("kw", [dict(sq=None), dict(sk=None), dict(skp=255), dict(skp=250),
+                                dict(sqp=63), dict(sk=A + 0x600004), dict(sv=A + 0x700004),
+                                dict(sq=A + 0x500002), dict(o=A + 0x600000)])
+def test_fp8_scaled_attention_argument_contract(kw):
+    assert hasb.lib().attn_fwd_fp8_scaled(*_fp8s_args(**kw)) == hasb.ATTN_ERR_INVALID_ARG
+
+
+def test_fp8_scaled_attention_other_head_dims_are_unsupported():
+    assert hasb.lib().attn_fwd_fp8_scaled(*_fp8s_args(d=64)) == hasb.ATTN_ERR_UNSUPPORTED
+
+
+def test_fp8_quantize_argument_contract():
+    L = hasb.lib()
+    x, y, s = A, A + 0x100000, A + 0x200000
+    assert L.attn_fp8_quantize_tokens(x, y, s, 1, 10, 2, 24, 10, 0, None) == hasb.ATTN_ERR_INVALID_ARG  # d
+    assert L.attn_fp8_quantize_tokens(x, y, s, 1, 10, 2, 128, 9, 0, None) == hasb.ATTN_ERR_INVALID_ARG  # pitch
+    assert L.attn_fp8_quantize_tokens(x, y, None, 1, 10, 2, 128, 10, 0, None) == hasb.ATTN_ERR_INVALID_ARG
+    assert L.attn_fp8_quantize_tokens(x, x + 64, s, 1, 10, 2, 128, 10, 0, None) == hasb.ATTN_ERR_INVALID_ARG
+    assert L.attn_fp8_quantize_tokens(x, y, s, 1, 10, 2, 128, 10, 5, None) == hasb.ATTN_ERR_INVALID_ARG  # dtype
+    assert L.attn_fp8_quantize_vt(x, y, s, 1, 100, 1, 32, 112, 0, None) == hasb.ATTN_ERR_INVALID_ARG     # d
+    assert L.attn_fp8_quantize_vt(x, y, None, 1, 100, 1, 128, 112, 0, None) == hasb.ATTN_ERR_INVALID_ARG
+    assert L.attn_fp8_quantize_vt(x, y, s, 1, 100, 1, 128, 104, 0, None) == hasb.ATTN_ERR_INVALID_ARG    # pitch

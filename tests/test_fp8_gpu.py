@@ -123,3 +123,100 @@ def test_fp8_attention_is_deterministic_and_takes_the_caller_buffers():
     hasb.attn_fwd_fp8(q8, k8, vt8, out=o2, lse=l2)
     torch.cuda.synchronize()
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+# ---------------------------------------------------------------- per-token scaled FP8
+
+def _scaled_inputs(B, L, H, d, seed, mag=1.0):
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn(B, L, H, d, generator=g) * mag
+    return x.to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("d", [16, 64, 128, 256])
+def test_quantize_tokens_is_bit_exact(d):
+    from oracle import quantize as qz
+    x = _scaled_inputs(2, 37, 3, d, seed=d)
+    x[0, 5, 1] = 0.0                                   # an all-zero row takes the floor
+    x[1, 7] *= 1e4
+    x[1, 8] *= 1e-30
+    codes, s = hasb.fp8_quantize_tokens(x.cuda())
+    torch.cuda.synchronize()
+    c_ref, s_ref = qz.quantize(x.to(torch.float64).numpy(), "e4m3", qz.SLICE, axis=-1)
+    want = torch.from_numpy(c_ref).to(torch.float8_e4m3fn).view(torch.uint8)
+    assert torch.equal(codes.cpu().view(torch.uint8), want)
+    got_s = s.cpu()[:, :, :37].numpy()                              # [B, H, L]
+    np.testing.assert_array_equal(got_s, s_ref[..., 0].transpose(0, 2, 1))
+
+
+@pytest.mark.parametrize("B,Lk,Hkv,d", [(2, 700, 3, 128), (1, 5, 2, 64), (1, 1000, 1, 256)])
+def test_quantize_vt_is_bit_exact(B, Lk, Hkv, d):
+    from oracle import quantize as qz
+    v = _scaled_inputs(B, Lk, Hkv, d, seed=Lk)
+    v[:, :, 0, 3] = 0.0                                # an all-zero channel
+    v[:, :, -1, 5] *= 1e-6
+    codes, sv = hasb.fp8_quantize_vt(v.cuda())
+    torch.cuda.synchronize()
+    c_ref, s_ref = qz.quantize(v.to(torch.float64).numpy(), "e4m3", qz.SLICE, axis=1)
+    want = torch.from_numpy(c_ref).to(torch.float8_e4m3fn).view(torch.uint8).permute(0, 2, 3, 1)
+    assert torch.equal(codes.cpu().view(torch.uint8)[..., :Lk], want)
+    np.testing.assert_array_equal(sv.cpu().numpy(), s_ref[:, 0])
+
+
+def _fp8_scaled_case(B, Lq, Lk, Hq, Hkv, mask, off, seed, rows=None, mag=1.0, v_scaled=True):
+    d = 128
+    q, k, v = inputs.make_qkv(B, Lq, Lk, Hq, Hkv, d, torch.float32, seed=seed)
+    q, k, v = ((t * mag).to(torch.bfloat16) for t in (q, k, v))
+    scale = 1.0 / math.sqrt(d) / mag ** 2
+    q8, sq = hasb.fp8_quantize_tokens(q.cuda())
+    k8, sk = hasb.fp8_quantize_tokens(k.cuda())
+    if v_scaled:
+        vt8, sv = hasb.fp8_quantize_vt(v.cuda())
+    else:
+        vt8, sv = hasb.fp8_cast_vt(v.cuda()), None
+    o, lse = hasb.attn_fwd_fp8_scaled(q8, sq, k8, sk, vt8, sv, scale=scale, causal=mask, kv_offset=off)
+    torch.cuda.synchronize()
+    f64 = lambda t: t.to(torch.float64).numpy()
+    qd, kd, vd = fp8.dequantized_attention_inputs(f64(q), f64(k), f64(v), v_scaled)
+    o_ref, lse_ref = oracle.attention_fwd(qd, kd, vd, scale, mask, off, rows=rows)
+    bound = fp8.p_rounding_bound(qd, kd, vd, scale, mask, off, rows=rows, cast=False)
+    var = fp8.p_rounding_var(qd, kd, vd, scale, mask, off, rows=rows, cast=False)
+    o_c, l_c = f64(o.cpu()), f64(lse.cpu())
+    if rows is not None:
+        o_c, l_c = o_c[:, rows], l_c[:, :, rows]
+    err = np.abs(o_c - o_ref)
+    what = f"fp8 scaled {B}x{Lq}x{Lk} {Hq}/{Hkv} mask {mask} mag {mag}"
+    assert np.isfinite(o_c).all(), what
+    excess = err - (bound + 2.0 ** -8 * np.abs(o_ref) + 1e-3 * mag)
+    assert excess.max() <= 0, f"{what}: above the P-rounding bound by {excess.max():.3g}"
+    out_var = np.mean((2.0 ** -8 * o_ref) ** 2) / 3.0
+    ratio = np.mean(err ** 2) / (np.mean(var) + out_var)
+    assert ratio <= 1.5, f"{what}: mean squared error {ratio:.3g} x the variance bound"
+    assert np.abs(l_c - lse_ref).max() <= 1e-3, what
+    return err
+
+
+@pytest.mark.parametrize("B,Lq,Lk,Hq,Hkv,mask,off", [
+    (1, 300, 700, 4, 2, 0, 0),
+    (2, 257, 900, 4, 1, 1, 643),
+    (1, 256, 1000, 2, 2, 2, 300),
+    (3, 64, 64, 2, 2, 0, 0),
+    (1, 1, 3, 1, 1, 0, 0),
+])
+def test_fp8_scaled_attention(B, Lq, Lk, Hq, Hkv, mask, off):
+    _fp8_scaled_case(B, Lq, Lk, Hq, Hkv, mask, off, seed=31 + Lq)
+
+
+def test_fp8_scaled_attention_unscaled_v():
+    _fp8_scaled_case(1, 300, 700, 4, 2, 0, 0, seed=5, v_scaled=False)
+
+
+def test_fp8_scaled_attention_keeps_small_magnitudes():
+    """Inputs around 1e-3 (scale compensated): the scaled path stays within
+    its bars where a direct e4m3 cast would flush most values to subnormals."""
+    _fp8_scaled_case(1, 256, 512, 2, 2, 0, 0, seed=8, mag=1e-3)
+
+
+def test_fp8_scaled_attention_video_shape_sampled_rows():
+    rows = inputs.sample_rows(20480, 48, seed=6).numpy()
+    _fp8_scaled_case(1, 20480, 20480, 56, 56, 0, 0, seed=9, rows=rows)
