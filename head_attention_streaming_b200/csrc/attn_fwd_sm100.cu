@@ -200,6 +200,9 @@ struct FwdParams {
   const float* sk;
   const float* sv;
   int sq_pitch, sk_pitch;
+  // head dim of the tensors (<= D): d = 16 and 32 run the D = 64 kernel on
+  // 64-wide TMA boxes whose columns >= d load as zero and are not stored
+  int d;
 };
 
 // KV tiles of a work unit: the loader streams tiles j0 .. j0 + nu - 1 (the
@@ -1058,7 +1061,7 @@ template <int D, bool BF16>
 __global__ void __launch_bounds__(256) split_merge_kernel(const float* __restrict__ o_part,
                                                           const float* __restrict__ lse_part, void* o,
                                                           float* lse, int n_splits, int B, int Lq,
-                                                          int Hq) {
+                                                          int Hq, int d_out) {
   constexpr int kPer = D / 32;
   const long long w = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) / 32;
   const int lane = threadIdx.x % 32;
@@ -1084,11 +1087,14 @@ __global__ void __launch_bounds__(256) split_merge_kernel(const float* __restric
     for (int e = 0; e < kPer; ++e) acc[e] = fmaf(wg, src[e], acc[e]);
   }
   const float inv = 1.f / tot;
-  uint16_t* out = static_cast<uint16_t*>(o) + ((static_cast<size_t>(b) * Lq + i) * Hq + hq) * D + lane * kPer;
+  uint16_t* out = static_cast<uint16_t*>(o) + ((static_cast<size_t>(b) * Lq + i) * Hq + hq) * d_out + lane * kPer;
+  // d_out < D: the partials' columns >= d_out are zero and not stored
+  if (lane * kPer < d_out) {
 #pragma unroll
-  for (int e = 0; e < kPer; e += 2) {
-    const uint32_t pk = pack2<BF16>(acc[e] * inv, acc[e + 1] * inv);
-    *reinterpret_cast<uint32_t*>(out + e) = pk;
+    for (int e = 0; e < kPer; e += 2) {
+      const uint32_t pk = pack2<BF16>(acc[e] * inv, acc[e + 1] * inv);
+      *reinterpret_cast<uint32_t*>(out + e) = pk;
+    }
   }
   if (lse != nullptr && lane == 0) lse[w] = m + logf(tot);
 }
@@ -1326,10 +1332,11 @@ int launch_fwd(const FwdParams& p, const void* q, const void* k, const void* v, 
         !encode_bl_hd(&to, p.o, p.B, p.Lq, p.Hq, D, true))
       return ATTN_ERR_CUDA;
   } else {
-    if (!encode_bl_hd(&tq, q, p.B, p.Lq, p.Hq, D, BF16) ||
-        !encode_bl_hd(&tk, k, p.B, p.Lk, p.Hkv, D, BF16, kv_rows) ||
-        !encode_bl_hd(&tv, v, p.B, p.Lk, p.Hkv, D, BF16, kv_rows) ||
-        !encode_bl_hd(&to, p.o, p.B, p.Lq, p.Hq, D, BF16))
+    const int dt = p.d > 0 ? p.d : D;
+    if (dt > D || !encode_bl_hd(&tq, q, p.B, p.Lq, p.Hq, dt, BF16) ||
+        !encode_bl_hd(&tk, k, p.B, p.Lk, p.Hkv, dt, BF16, kv_rows) ||
+        !encode_bl_hd(&tv, v, p.B, p.Lk, p.Hkv, dt, BF16, kv_rows) ||
+        !encode_bl_hd(&to, p.o, p.B, p.Lq, p.Hq, dt, BF16))
       return ATTN_ERR_CUDA;
   }
   auto kern = attn_fwd_sm100_kernel<D, BF16, CAUSAL, SPLIT, WINDOW, F8>;
@@ -1428,7 +1435,7 @@ int attn_fwd_validate(const void* q, const void* k, const void* v, const void* o
   if (ranges_overlap(o, q_elems * 2, q, q_elems * 2) || ranges_overlap(o, q_elems * 2, k, kv_elems * 2) ||
       ranges_overlap(o, q_elems * 2, v, kv_elems * 2))
     return ATTN_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (d != 16 && d != 32 && d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
   return ATTN_OK;
 }
 
@@ -1454,6 +1461,7 @@ int attn_fwd_impl(const void* q, const void* k, const void* v, void* o, float* l
   if (!di.sm100) return ATTN_ERR_UNSUPPORTED;
 
   FwdParams p{};
+  p.d = d;
   p.o = o;
   p.lse = lse;
   p.B = B; p.Lq = Lq; p.Lk = Lk; p.Hq = Hq; p.Hkv = Hkv; p.group = Hq / Hkv;
@@ -1565,7 +1573,8 @@ int splitkv_run(const void* q, const void* k, const void* v, void* o, float* lse
     return attn_fwd(q, k, v, o, lse, B, Lq, Lk, Hq, Hkv, d, scale, causal, kv_offset, dtype, stream);
   const size_t need = attn_splitkv_workspace_bytes(B, Lq, Hq, d, ns);
   if (workspace == nullptr || workspace_bytes < need) return ATTN_ERR_INVALID_ARG;
-  const size_t o_elems = static_cast<size_t>(ns) * B * Hq * Lq * d;
+  // float32 partial rows of max(d, 64) columns (d = 16, 32 run the 64-wide kernel), then the LSEs
+  const size_t o_elems = static_cast<size_t>(ns) * B * Hq * Lq * (d < 64 ? 64 : d);
   if (ranges_overlap(workspace, need, q, 2ull * B * Lq * Hq * d) ||
       ranges_overlap(workspace, need, k, 2ull * B * Lk * Hkv * d) ||
       ranges_overlap(workspace, need, v, 2ull * B * Lk * Hkv * d) ||
@@ -1575,6 +1584,7 @@ int splitkv_run(const void* q, const void* k, const void* v, void* o, float* lse
   if (base_units * ns > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
 
   FwdParams p{};
+  p.d = d;
   p.o = o;
   p.lse = lse;
   p.B = B; p.Lq = Lq; p.Lk = Lk; p.Hq = Hq; p.Hkv = Hkv; p.group = Hq / Hkv;
@@ -1603,11 +1613,11 @@ int splitkv_run(const void* q, const void* k, const void* v, void* o, float* lse
   const long long rows = 1LL * B * Hq * Lq;
   const unsigned mgrid = static_cast<unsigned>((rows * 32 + 255) / 256);
   if (d == 128) {
-    if (bf16) split_merge_kernel<128, true><<<mgrid, 256, 0, s>>>(p.o_part, p.lse_part, o, lse, ns, B, Lq, Hq);
-    else split_merge_kernel<128, false><<<mgrid, 256, 0, s>>>(p.o_part, p.lse_part, o, lse, ns, B, Lq, Hq);
+    if (bf16) split_merge_kernel<128, true><<<mgrid, 256, 0, s>>>(p.o_part, p.lse_part, o, lse, ns, B, Lq, Hq, d);
+    else split_merge_kernel<128, false><<<mgrid, 256, 0, s>>>(p.o_part, p.lse_part, o, lse, ns, B, Lq, Hq, d);
   } else {
-    if (bf16) split_merge_kernel<64, true><<<mgrid, 256, 0, s>>>(p.o_part, p.lse_part, o, lse, ns, B, Lq, Hq);
-    else split_merge_kernel<64, false><<<mgrid, 256, 0, s>>>(p.o_part, p.lse_part, o, lse, ns, B, Lq, Hq);
+    if (bf16) split_merge_kernel<64, true><<<mgrid, 256, 0, s>>>(p.o_part, p.lse_part, o, lse, ns, B, Lq, Hq, d);
+    else split_merge_kernel<64, false><<<mgrid, 256, 0, s>>>(p.o_part, p.lse_part, o, lse, ns, B, Lq, Hq, d);
   }
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
@@ -1742,7 +1752,8 @@ int attn_fwd_cache(const void* q, const void* k_cache, const void* v_cache, void
 
 size_t attn_splitkv_workspace_bytes(int B, int Lq, int Hq, int d, int n_splits) {
   if (B < 1 || Lq < 1 || Hq < 1 || d < 1 || n_splits < 1) return 0;
-  return static_cast<size_t>(n_splits) * B * Hq * Lq * (static_cast<size_t>(d) + 1) * sizeof(float);
+  const size_t dp = d < 64 ? 64 : static_cast<size_t>(d);  // d = 16, 32 run with 64-column partials
+  return static_cast<size_t>(n_splits) * B * Hq * Lq * (dp + 1) * sizeof(float);
 }
 
 int attn_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse,

@@ -80,7 +80,7 @@ def test_invalid_arguments_are_rejected_before_any_launch(kw):
     assert _call(**kw) == hasb.ATTN_ERR_INVALID_ARG
 
 
-@pytest.mark.parametrize("d", [16, 32, 256])
+@pytest.mark.parametrize("d", [256])
 def test_head_dims_allowed_by_the_pages_but_not_built_are_unsupported(d):
     assert _call(d=d) == hasb.ATTN_ERR_UNSUPPORTED
 

@@ -1,0 +1,89 @@
+"""Head dims 16 and 32 on a B200 against the FP64 oracle: plain, masked,
+windowed, key-split and cache-prefix attention (the pages' contract allows
+powers of two 16..256; these two run the 64-wide kernel with the columns past
+d loaded as zero and not stored). Bars as in the attention parity tests."""
+
+from __future__ import annotations
+
+import math
+
+import pytest
+import torch
+
+import head_attention_streaming_b200 as hasb
+import oracle
+from head_attention_streaming_b200 import inputs
+from test_parity_gpu import _check
+
+pytestmark = pytest.mark.gpu
+
+f64 = lambda t: t.to(torch.float64).numpy()
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _device(cuda_ok):
+    torch.cuda.set_device(0)
+    yield
+    assert hasb.device_fault(clear=True) == 0
+
+
+def _qkv(B, Lq, Lk, Hq, Hkv, d, dtype, seed):
+    return inputs.make_qkv(B, Lq, Lk, Hq, Hkv, d, dtype, seed=seed)
+
+
+@pytest.mark.parametrize("d", [16, 32])
+@pytest.mark.parametrize("B,Lq,Lk,Hq,Hkv,dtype,mask,off", [
+    (1, 1, 1, 1, 1, torch.bfloat16, 0, 0),
+    (2, 257, 300, 4, 2, torch.bfloat16, 0, 0),
+    (1, 300, 300, 2, 1, torch.float16, 1, 0),
+    (1, 77, 500, 4, 4, torch.bfloat16, 1, 423),
+    (1, 200, 700, 8, 2, torch.float16, 2, 300),
+])
+def test_small_head_dims(d, B, Lq, Lk, Hq, Hkv, dtype, mask, off):
+    q, k, v = _qkv(B, Lq, Lk, Hq, Hkv, d, dtype, seed=7 * d + Lq)
+    scale = 1.0 / math.sqrt(d)
+    o, lse = hasb.attn_fwd(q.cuda(), k.cuda(), v.cuda(), scale=scale, causal=mask, kv_offset=off)
+    torch.cuda.synchronize()
+    o_ref, lse_ref = oracle.attention_fwd(f64(q), f64(k), f64(v), scale, mask, off)
+    _check(o.cpu(), lse.cpu(), o_ref, lse_ref, "bf16" if dtype == torch.bfloat16 else "fp16",
+           what=f"d={d}", output_ulp=True)
+
+
+@pytest.mark.parametrize("d", [16, 32])
+def test_small_head_dims_neighbours_untouched(d):
+    """The output's row stride is d: a store of 64 columns would overwrite the
+    next head's row. Surround O with sentinels and check they survive."""
+    q, k, v = _qkv(1, 130, 200, 3, 1, d, torch.bfloat16, seed=d)
+    buf = torch.full((1 * 130 * 3 * d + 2 * 4096,), 7.0, dtype=torch.bfloat16, device="cuda")
+    out = buf[4096:4096 + 130 * 3 * d].view(1, 130, 3, d)
+    hasb.attn_fwd(q.cuda(), k.cuda(), v.cuda(), out=out)
+    torch.cuda.synchronize()
+    assert bool((buf[:4096] == 7.0).all()) and bool((buf[-4096:] == 7.0).all())
+    o_ref, _ = oracle.attention_fwd(f64(q), f64(k), f64(v), 1.0 / math.sqrt(d), 0, 0)
+    assert abs(f64(out.cpu()) - o_ref).max() < 1e-2
+
+
+@pytest.mark.parametrize("d", [16, 32])
+def test_small_head_dims_window_split_and_cache(d):
+    q, k, v = _qkv(1, 300, 900, 4, 2, d, torch.bfloat16, seed=3 + d)
+    scale = 1.0 / math.sqrt(d)
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    o, lse = hasb.attn_fwd_window(qc, kc, vc, window=(100, 20), scale=scale, kv_offset=500)
+    torch.cuda.synchronize()
+    ref = oracle.attention_fwd(f64(q), f64(k), f64(v), scale, oracle.MASK_WINDOW, 500, window=(100, 20))
+    _check(o.cpu(), lse.cpu(), *ref, "bf16", what=f"window d={d}", output_ulp=True)
+    o, lse, used = hasb.attn_fwd_splitkv(qc, kc, vc, n_splits=3, scale=scale)
+    torch.cuda.synchronize()
+    assert used == 3
+    ref = oracle.attention_fwd(f64(q), f64(k), f64(v), scale, 0, 0)
+    _check(o.cpu(), lse.cpu(), *ref, "bf16", what=f"split d={d}", output_ulp=True)
+    # a cache of 1200 slots of which the first 900 are valid
+    S = 1200
+    kcache = torch.zeros(1, S, 2, d, dtype=torch.bfloat16, device="cuda")
+    vcache = torch.zeros_like(kcache)
+    kcache[:, :900] = kc
+    vcache[:, :900] = vc
+    o, lse = hasb.attn_fwd_cache(qc, kcache, vcache, 900, scale=scale, causal=hasb.MASK_CHUNK, kv_offset=600)
+    torch.cuda.synchronize()
+    ref = oracle.attention_fwd(f64(q), f64(k), f64(v), scale, 2, 600)
+    _check(o.cpu(), lse.cpu(), *ref, "bf16", what=f"cache d={d}", output_ulp=True)
