@@ -87,6 +87,30 @@ struct Cfg {
   static constexpr int kOffSk = 0;         // no key scales
 };
 
+// d = 256: one 128-row query tile per unit. Tensor memory holds two S buffers
+// (128 columns each, alternating over KV tiles, P aliased as for the other
+// head dims) and O (256 columns); shared memory holds the Q tile (64 KB) and a
+// two-stage K/V ring (64 KB a tile). O goes from registers straight to global
+// memory, so there is no staging buffer.
+template <>
+struct Cfg<256, 0> {
+  static constexpr int kChunks = 4;
+  static constexpr int kChunkBytes = kTileRows * 128;
+  static constexpr int kTileBytes = kTileRows * 256 * 2;
+  static constexpr int kStages = 2;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffKV = kTileBytes;
+  static constexpr int kOffStg = 0;
+  static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
+  static constexpr int kSmemBytes = kOffBar + 512 + 1024;
+  static __device__ __forceinline__ uint32_t col_s(int buf) { return buf ? 128u : 0u; }
+  static __device__ __forceinline__ uint32_t col_o(int) { return 256u; }
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr int kOChunks = 4;
+  static constexpr int kOffP = 0;
+  static constexpr int kOffSk = 0;
+};
+
 // e4m3 operands, d = 128: a Q / K row is one 128-byte swizzle chunk (16 KB per
 // 128-row tile), V arrives transposed (a tile is 128 d-rows of 128 keys) so
 // both P V operands are K-major, and P goes through shared memory (two 16 KB
@@ -219,6 +243,28 @@ __device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
 // Work unit u -> (b, hq, row pair). Query heads of one GQA group are adjacent
 // and the row pairs of one head are adjacent, so CTAs running together read
 // the same K/V head (L2 reuse). Causal units run longest first.
+// d = 256: unit u -> (b, hq, 128-row tile); p.n_pairs counts tiles here.
+// Same order as decode_unit (GQA group heads adjacent, causal longest first).
+template <bool CAUSAL>
+__device__ __forceinline__ Unit decode_single(const FwdParams& p, int u) {
+  Unit x;
+  x.split = 0;
+  int tile = u % p.n_pairs;
+  int t = u / p.n_pairs;
+  const int g = t % p.group;
+  t /= p.group;
+  x.hkv = t % p.Hkv;
+  x.b = t / p.Hkv;
+  x.hq = x.hkv * p.group + g;
+  if (CAUSAL) tile = p.n_pairs - 1 - tile;
+  x.r0 = tile * kTileRows;
+  x.j0 = 0;
+  x.s0 = x.s1 = 0;
+  const int lim = CAUSAL ? min(p.Lk, p.kv_offset + x.r0 + kTileRows) : p.kv_limit;
+  x.n0 = x.n1 = x.nu = (lim + kTileRows - 1) / kTileRows;
+  return x;
+}
+
 template <bool CAUSAL, bool SPLIT, bool WINDOW>
 __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
   Unit x;
@@ -380,8 +426,10 @@ __device__ __forceinline__ void load_role(const CUtensorMap* tm_q, const CUtenso
   int kv_it = 0, uit = 0;
   bool aborted = false;
   for (int u = blockIdx.x; u < p.n_units && !aborted; u += gridDim.x, ++uit) {
-    const Unit x = decode_unit<CAUSAL, SPLIT, WINDOW>(p, u);
-    for (int t = 0; t < 2; ++t) {
+    Unit x;
+    if constexpr (D == 256) x = decode_single<CAUSAL>(p, u);
+    else x = decode_unit<CAUSAL, SPLIT, WINDOW>(p, u);
+    for (int t = 0; t < (D == 256 ? 1 : 2); ++t) {
       const uint32_t bq = bars + 8 * (kBarQEmpty + t);
       if (!mbar_wait(bq, (uit & 1) ^ 1, abort_flag, kFaultLoadQEmpty, p.timeout_ns)) {
         aborted = true;
@@ -960,6 +1008,208 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
   }
 }
 
+// ----------------------------------------------------------------- d = 256
+// One query tile per unit and one MMA issuer: S alternates between two tensor
+// memory buffers over the KV tiles, so Q K_{j+1}^T runs on the tensor core
+// while the softmax works on tile j; O += P_j V_j follows once P_j is in. The
+// issuer commits kBarOFull after every P V, so the softmax knows when O may be
+// rescaled (and, after the last, read out).
+template <bool BF16, bool CAUSAL>
+__device__ __forceinline__ void mma_role_single(const FwdParams& p, uint32_t tmem, uint32_t sQ,
+                                                uint32_t sKV, uint32_t bars, volatile int* abort_flag) {
+  using C = Cfg<256, 0>;
+  auto bar = [&](int i) { return bars + 8 * i; };
+  const uint32_t q_lo = smem_desc_lo(sQ, 16);
+  auto k_lo = [&](int idx) { return smem_desc_lo(sKV + (idx % C::kStages) * C::kTileBytes, 16); };
+  auto v_lo = [&](int idx) {
+    return smem_desc_lo(sKV + (idx % C::kStages) * C::kTileBytes, C::kChunkBytes);
+  };
+  auto kv_full = [&](int idx) {
+    return mbar_wait(bar(kBarKvFull + idx % C::kStages), (idx / C::kStages) & 1, abort_flag,
+                     kFaultMmaKvFull, p.timeout_ns);
+  };
+  const uint32_t o_t = tmem + C::col_o(0);
+  int kv_it = 0, uit = 0, pcnt = 0, sc = 0;
+  bool ok = true;
+  for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++uit) {
+    const Unit x = decode_single<CAUSAL>(p, u);
+    const int n = x.n0;
+    ok = mbar_wait(bar(kBarQFull), uit & 1, abort_flag, kFaultMmaQFull, p.timeout_ns) && kv_full(kv_it);
+    if (!ok) break;
+    // S(0) = Q K_0^T
+    issue_qk<256, BF16>(tmem + C::col_s(sc & 1), q_lo, k_lo(kv_it));
+    mma_commit(bar(kBarSFull + (sc & 1)));
+    mma_commit(bar(kBarKvEmpty + kv_it % C::kStages));
+    if (n == 1) mma_commit(bar(kBarQEmpty));
+    ++sc;
+    for (int j = 0; j < n; ++j) {
+      const int vidx = kv_it + 2 * j + 1;
+      const uint32_t s_j = tmem + C::col_s((sc - 1) & 1);  // tile j's S / P buffer
+      if (j + 1 < n) {
+        // S(j+1) into the other buffer: its last P was read by a P V issued earlier
+        const int knext = vidx + 1;
+        if (!kv_full(knext)) { ok = false; break; }
+        issue_qk<256, BF16>(tmem + C::col_s(sc & 1), q_lo, k_lo(knext));
+        mma_commit(bar(kBarSFull + (sc & 1)));
+        mma_commit(bar(kBarKvEmpty + knext % C::kStages));
+        if (j + 1 == n - 1) mma_commit(bar(kBarQEmpty));
+      }
+      // O += P_j V_j in two halves of 64 keys
+      if (!kv_full(vidx) ||
+          !mbar_wait(bar(kBarPHalf), pcnt & 1, abort_flag, kFaultMmaPFull, p.timeout_ns)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after_sync();
+      issue_pv_half<256, BF16, 0>(o_t, s_j, v_lo(vidx), j > 0 ? 1u : 0u);
+      if (!mbar_wait(bar(kBarPFull), pcnt & 1, abort_flag, kFaultMmaPFull, p.timeout_ns)) {
+        ok = false;
+        break;
+      }
+      ++pcnt;
+      tc_fence_after_sync();
+      issue_pv_half<256, BF16, 1>(o_t, s_j, v_lo(vidx), 1u);
+      mma_commit(bar(kBarKvEmpty + vidx % C::kStages));
+      mma_commit(bar(kBarOFull));
+      if (j + 1 < n) ++sc;
+    }
+    kv_it += 2 * x.nu;
+  }
+  if (!ok) {
+    mma_commit(bar(kBarDrain));
+    mbar_drain(bar(kBarDrain), 0);
+  }
+}
+
+// The softmax of the one query tile (warps 0-3, one thread per row). Per KV
+// tile: wait for S_j; row max; wait until P_{j-1} V_{j-1} is done (O may then
+// be rescaled and S_j's buffer partner is free); exponentials into P_j. End of
+// a unit: wait for the last P V, O / l to 16 bits straight to global memory.
+template <bool BF16, bool CAUSAL>
+__device__ __forceinline__ void softmax_role_single(const FwdParams& p, uint32_t tmem, uint32_t bars,
+                                                    volatile int* abort_flag) {
+  using C = Cfg<256, 0>;
+  constexpr int D = 256;
+  const int warp = threadIdx.x / 32;
+  const int r_in = threadIdx.x % kTileRows;
+  const int lane = threadIdx.x % 32;
+  const uint32_t lane_bits = static_cast<uint32_t>((warp % 4) * 32) << 16;
+  const uint32_t tO = tmem + lane_bits + C::col_o(0);
+  const uint32_t bar_p = bars + 8 * kBarPFull;
+  const uint32_t bar_ph = bars + 8 * kBarPHalf;
+  const uint32_t bar_o = bars + 8 * kBarOFull;
+  const float sl2 = p.sl2;
+  int sc = 0, ocnt = 0;
+  for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
+    const Unit x = decode_single<CAUSAL>(p, u);
+    const int n = x.n0;
+    const int row = x.r0 + r_in;
+    const int row_lim = CAUSAL ? min(p.Lk, p.kv_offset + row + 1) : p.kv_limit;
+    float ref = -INFINITY;
+    float l = 0.f;
+    for (int j = 0; j < n; ++j) {
+      const int buf = sc & 1;
+      const uint32_t tS = tmem + lane_bits + C::col_s(buf);
+      bool ok = mbar_wait(bars + 8 * (kBarSFull + buf), (sc >> 1) & 1, abort_flag, kFaultSoftmaxSFull,
+                          p.timeout_ns);
+      if (!__all_sync(0xffffffffu, ok)) return;
+      ++sc;
+      tc_fence_after_sync();
+      uint32_t r[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(tS + 32 * c, r + 32 * c);
+      tmem_wait_ld_x128(r);
+      const int key0 = j * kTileRows;
+      const int lim = row_lim - key0;
+      const bool partial = lim < kTileRows;
+      if (partial) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (c >= lim) r[c] = __float_as_uint(-INFINITY);
+      }
+      float m_tile;
+      {  // three-input max tree
+        float a[43];
+#pragma unroll
+        for (int i = 0; i < 42; ++i)
+          a[i] = fmax3(__uint_as_float(r[3 * i]), __uint_as_float(r[3 * i + 1]), __uint_as_float(r[3 * i + 2]));
+        a[42] = fmaxf(__uint_as_float(r[126]), __uint_as_float(r[127]));
+        float b[15];
+#pragma unroll
+        for (int i = 0; i < 14; ++i) b[i] = fmax3(a[3 * i], a[3 * i + 1], a[3 * i + 2]);
+        b[14] = a[42];
+        float c5[5];
+#pragma unroll
+        for (int i = 0; i < 5; ++i) c5[i] = fmax3(b[3 * i], b[3 * i + 1], b[3 * i + 2]);
+        m_tile = fmaxf(fmax3(c5[0], c5[1], c5[2]), fmaxf(c5[3], c5[4]));
+      }
+      const float m_scaled = (m_tile == -INFINITY) ? -INFINITY : m_tile * sl2;
+      if (j > 0) {
+        // P_{j-1} V_{j-1} done: O may be rescaled
+        ok = mbar_wait(bar_o, ocnt & 1, abort_flag, kFaultSoftmaxOFull, p.timeout_ns);
+        if (!__all_sync(0xffffffffu, ok)) return;
+        ++ocnt;
+        tc_fence_after_sync();
+      }
+      const bool rescale = m_scaled > ref + kRescaleTau;
+      if (__any_sync(0xffffffffu, rescale)) {
+        float alpha = 1.f;
+        if (rescale) {
+          alpha = ex2_approx(ref - m_scaled);
+          ref = m_scaled;
+          l *= alpha;
+        }
+        if (j > 0) {
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t ov[32];
+            tmem_ld_32x32b_x32(tO + 32 * c, ov);
+            tmem_wait_ld_x32(ov);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+            tmem_st_32x32b_x32(tO + 32 * c, ov);
+          }
+          tmem_wait_st();
+        }
+      }
+      float sum[4] = {0.f, 0.f, 0.f, 0.f};
+      if (__any_sync(0xffffffffu, partial))
+        exp_tile<BF16, true>(r, sl2, -ref, lim, 0, sum, tS, bar_ph, bar_p, 0u, false, lane);
+      else
+        exp_tile<BF16, false>(r, sl2, -ref, lim, 0, sum, tS, bar_ph, bar_p, 0u, false, lane);
+      l += (sum[0] + sum[1]) + (sum[2] + sum[3]);
+    }
+    // the last P V, then O / l straight to global memory
+    bool ok = mbar_wait(bar_o, ocnt & 1, abort_flag, kFaultSoftmaxOFull, p.timeout_ns);
+    if (!__all_sync(0xffffffffu, ok)) return;
+    ++ocnt;
+    tc_fence_after_sync();
+    const float inv_l = 1.f / l;
+    const bool in_range = row < p.Lq;
+    uint16_t* dst = static_cast<uint16_t*>(p.o) + ((static_cast<size_t>(x.b) * p.Lq + row) * p.Hq + x.hq) * D;
+#pragma unroll 1
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t ov[32];
+      tmem_ld_32x32b_x32(tO + 32 * c, ov);
+      tmem_wait_ld_x32(ov);
+      if (in_range) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          pk[e] = pack2<BF16>(__uint_as_float(ov[2 * e]) * inv_l, __uint_as_float(ov[2 * e + 1]) * inv_l);
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          *reinterpret_cast<uint4*>(dst + 32 * c + 8 * e) =
+              make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+      }
+    }
+    if (p.lse != nullptr && in_range)
+      p.lse[(static_cast<size_t>(x.b) * p.Hq + x.hq) * p.Lq + row] = (ref + log2f(l)) * kLn2;
+    // every TMEM read of O is complete (wait::ld) before the next unit's first
+    // P V overwrites it: that MMA waits for this warpgroup's next P
+  }
+}
+
 template <int D, bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW, int F8>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -998,7 +1248,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bars + 8 * (kBarDrain + 1), 1);
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(bars + 8 * (kBarKvFull + s), 1);
-      mbar_init(bars + 8 * (kBarKvEmpty + s), 2);
+      mbar_init(bars + 8 * (kBarKvEmpty + s), D == 256 ? 1 : 2);  // one MMA issuer at d = 256
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -1025,7 +1275,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   griddep_wait();
   griddep_launch_dependents();
 
-  if (warp < 8) {
+  if constexpr (D == 256) {
+    // one query tile: warps 0-3 softmax, warp 8 loads, warp 9 issues the MMAs
+    if (warp < 8) {
+      regs_increase<kRegsSoftmax>();
+      if (warp < 4) softmax_role_single<BF16, CAUSAL>(p, tmem, bars, abort_flag);
+    } else {
+      regs_decrease<kRegsProducer>();
+      if (warp == 8 && lane == 0)
+        load_role<D, BF16, CAUSAL, SPLIT, WINDOW, F8>(&tm_q, &tm_k, &tm_v, p, sQ, sKV, bars, abort_flag);
+      else if (warp == 9 && lane == 0)
+        mma_role_single<BF16, CAUSAL>(p, tmem, sQ, sKV, bars, abort_flag);
+    }
+  } else if (warp < 8) {
     regs_increase<kRegsSoftmax>();
     softmax_role<D, BF16, CAUSAL, SPLIT, WINDOW, F8>(warp / 4, p, tmem, bars, sStg, sP, sbase + C::kOffSk,
                                                      abort_flag);
@@ -1435,7 +1697,7 @@ int attn_fwd_validate(const void* q, const void* k, const void* v, const void* o
   if (ranges_overlap(o, q_elems * 2, q, q_elems * 2) || ranges_overlap(o, q_elems * 2, k, kv_elems * 2) ||
       ranges_overlap(o, q_elems * 2, v, kv_elems * 2))
     return ATTN_ERR_INVALID_ARG;
-  if (d != 16 && d != 32 && d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (d != 16 && d != 32 && d != 64 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
   return ATTN_OK;
 }
 
@@ -1450,7 +1712,10 @@ int attn_fwd_impl(const void* q, const void* k, const void* v, void* o, float* l
                                       window ? ATTN_MASK_CHUNK : causal, kv_offset, dtype, kv_rows);
   if (valid != ATTN_OK) return valid;
   if (window && (win_left < -1 || win_right < -1)) return ATTN_ERR_INVALID_ARG;
-  const long long n_pairs = (Lq + 2LL * kTileRows - 1) / (2LL * kTileRows);
+  if (window && d == 256) return ATTN_ERR_UNSUPPORTED;
+  // units: pairs of 128-row query tiles; single tiles at d = 256
+  const long long rows_per_unit = d == 256 ? kTileRows : 2LL * kTileRows;
+  const long long n_pairs = (Lq + rows_per_unit - 1) / rows_per_unit;
   const long long n_units = n_pairs * B * Hq;
 
   // ---- device
@@ -1489,6 +1754,10 @@ int attn_fwd_impl(const void* q, const void* k, const void* v, void* o, float* l
                 : launch_fwd<64, false, false, false, true>(p, q, k, v, kv_rows, grid, s);
   }
   const bool cz = causal == ATTN_MASK_CAUSAL;
+  if (d == 256) {
+    if (bf16) return cz ? launch_fwd<256, true, true>(p, q, k, v, kv_rows, grid, s) : launch_fwd<256, true, false>(p, q, k, v, kv_rows, grid, s);
+    return cz ? launch_fwd<256, false, true>(p, q, k, v, kv_rows, grid, s) : launch_fwd<256, false, false>(p, q, k, v, kv_rows, grid, s);
+  }
   if (d == 128) {
     if (bf16) return cz ? launch_fwd<128, true, true>(p, q, k, v, kv_rows, grid, s) : launch_fwd<128, true, false>(p, q, k, v, kv_rows, grid, s);
     return cz ? launch_fwd<128, false, true>(p, q, k, v, kv_rows, grid, s) : launch_fwd<128, false, false>(p, q, k, v, kv_rows, grid, s);
@@ -1541,6 +1810,7 @@ int splitkv_validate(const void* q, const void* k, const void* v, const void* o,
                                       kv_offset, dtype, Lk);
   if (valid != ATTN_OK) return valid;
   if (causal == ATTN_MASK_CAUSAL || n_splits < 0) return ATTN_ERR_INVALID_ARG;
+  if (d == 256) return ATTN_ERR_UNSUPPORTED;  // the one-tile d = 256 kernel has no key split
   return ATTN_OK;
 }
 

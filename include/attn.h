@@ -63,10 +63,11 @@ typedef enum {
  *   lse  device, [B, Hq, Lq] float32, natural log of sum_j exp(scale * s_ij)
  *        over visible keys; may be NULL (then not written)
  *   B, Lq, Lk, Hq, Hkv  >= 1, Hq % Hkv == 0
- *   d    head_dim; the pages allow powers of two 16..256; this build runs 16, 32,
- *        64 and 128 (16 and 32 through the 64-wide kernel: its TMA boxes read
- *        the columns past d as zero and store only d columns; 256 returns
- *        ATTN_ERR_UNSUPPORTED)
+ *   d    head_dim, a power of two 16..256 (the pages' range): 16 and 32 run
+ *        through the 64-wide kernel (its TMA boxes read the columns past d as
+ *        zero and store only d columns); 256 runs one 128-row query tile per
+ *        work unit (its tensor memory holds S twice and O once); the key
+ *        split and the sliding window return ATTN_ERR_UNSUPPORTED at 256
  *   scale  finite, >= 0 (1/sqrt(d) in the pages)
  *   causal attn_mask_t: 0 none, 1 causal, 2 streaming chunk
  *   kv_offset  cache position of query row 0: 0 for mask 0; for masks 1 and 2,

@@ -87,3 +87,55 @@ def test_small_head_dims_window_split_and_cache(d):
     torch.cuda.synchronize()
     ref = oracle.attention_fwd(f64(q), f64(k), f64(v), scale, 2, 600)
     _check(o.cpu(), lse.cpu(), *ref, "bf16", what=f"cache d={d}", output_ulp=True)
+
+
+# ---------------------------------------------------------------- d = 256
+
+@pytest.mark.parametrize("B,Lq,Lk,Hq,Hkv,dtype,mask,off", [
+    (1, 1, 1, 1, 1, torch.bfloat16, 0, 0),
+    (2, 257, 300, 4, 2, torch.bfloat16, 0, 0),        # ragged query and key tails, GQA
+    (1, 300, 300, 2, 1, torch.float16, 1, 0),         # causal, MQA
+    (1, 77, 500, 4, 4, torch.bfloat16, 1, 423),       # causal with an offset
+    (1, 200, 700, 8, 2, torch.float16, 2, 300),       # streaming chunk
+    (1, 640, 640, 2, 2, torch.bfloat16, 0, 0),        # several units per CTA order
+])
+def test_d256(B, Lq, Lk, Hq, Hkv, dtype, mask, off):
+    d = 256
+    q, k, v = _qkv(B, Lq, Lk, Hq, Hkv, d, dtype, seed=11 + Lq + Lk)
+    scale = 1.0 / math.sqrt(d)
+    o, lse = hasb.attn_fwd(q.cuda(), k.cuda(), v.cuda(), scale=scale, causal=mask, kv_offset=off)
+    torch.cuda.synchronize()
+    o_ref, lse_ref = oracle.attention_fwd(f64(q), f64(k), f64(v), scale, mask, off)
+    _check(o.cpu(), lse.cpu(), o_ref, lse_ref, "bf16" if dtype == torch.bfloat16 else "fp16",
+           what="d=256", output_ulp=True)
+
+
+def test_d256_large_scores_rescale_and_cache_prefix():
+    """Scores that grow along the keys (each KV tile's max above the last by
+    more than the lazy-rescale threshold) and a cache prefix of 900 of 1024 slots."""
+    d = 256
+    q, k, v = _qkv(1, 256, 900, 2, 1, d, torch.bfloat16, seed=77)
+    ramp = torch.linspace(0.5, 6.0, 900).view(1, 900, 1, 1)
+    k = (k.float() * ramp).to(torch.bfloat16)
+    scale = 1.0 / math.sqrt(d)
+    kc = torch.zeros(1, 1024, 1, d, dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    kc[:, :900] = k.cuda()
+    vc[:, :900] = v.cuda()
+    o, lse = hasb.attn_fwd_cache(q.cuda(), kc, vc, 900, scale=scale, causal=hasb.MASK_CHUNK, kv_offset=644)
+    torch.cuda.synchronize()
+    o_ref, lse_ref = oracle.attention_fwd(f64(q), f64(k), f64(v), scale, 2, 644)
+    _check(o.cpu(), lse.cpu(), o_ref, lse_ref, "bf16", what="d=256 cache", output_ulp=True)
+
+
+def test_d256_deterministic_and_split_window_refused():
+    q, k, v = (t.cuda() for t in _qkv(1, 300, 500, 2, 2, 256, torch.bfloat16, seed=5))
+    a, la = hasb.attn_fwd(q, k, v)
+    b, lb = hasb.attn_fwd(q, k, v)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b) and torch.equal(la, lb)
+    for call in (lambda: hasb.attn_fwd_splitkv(q, k, v, n_splits=2),
+                 lambda: hasb.attn_fwd_window(q, k, v, window=(10, 10))):
+        with pytest.raises(hasb.AttnError) as e:
+            call()
+        assert e.value.status == hasb.ATTN_ERR_UNSUPPORTED
