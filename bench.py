@@ -58,6 +58,7 @@ METRIC = "attention fwd TFLOPS on 1 B200 and % of dense BF16 tensor-core peak"
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "attn_fwd_video_20480x56x128.md")
 PROLOGUE_SUMMARY = os.path.join(ROOT, "profiles", "qk_prologue_dit_1785x40x128.md")
+FP8_SUMMARY = os.path.join(ROOT, "profiles", "attn_fwd_fp8_video_20480x56x128.md")
 KERNEL_SOURCES = [os.path.join(ROOT, "head_attention_streaming_b200", "csrc", f)
                   for f in ("attn_fwd_sm100.cu", "sm100_ptx.cuh", "tmem_ldst.inc")]
 
@@ -668,6 +669,10 @@ def run_fp8(args):
               and ci["sm_mhz"] < 0.97 * ci.get("sm_max_mhz", ci["sm_mhz"]))
     peak = 2.0 * (peak16_sus if capped else peak16)   # e4m3 dense = 2 x bf16 dense (4.5 vs 2.25 PF)
     achieved = flops / (statistics.mean(attn_ms) * 1e-3) / 1e12
+    if args.scaled or w.name != "video_20480x56x128":
+        traffic, traffic_src = None, "no ncu summary of this variant / workload"
+    else:
+        traffic, traffic_src = profiled_traffic(FP8_SUMMARY)
     if rank == 0:
         line = {
             "metric": ("per-token scaled FP8 (e4m3) attention forward TFLOPS incl. the Q/K/V quantization"
@@ -682,8 +687,7 @@ def run_fp8(args):
                                  "attn_fwd_fp8_scaled: all timed") if args.scaled else
                                 "fp8_cast(Q), fp8_cast(K), fp8_cast_vt(V), attn_fwd_fp8: all timed"),
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                         "frac": achieved / peak, "traffic": None,
-                         "traffic_source": "no ncu summary of the FP8 kernel",
+                         "frac": achieved / peak, "traffic": traffic, "traffic_source": traffic_src,
                          "peak_source": ("2 x bf16_tflops_sustained" if capped else "2 x bf16_tflops (burst)")
                                         + f" of {peak_src} (nominal e4m3 / bf16 dense ratio)",
                          "kernel": "attn_fwd_sm100_kernel (e4m3" + (", per-token scales)" if args.scaled else ")"),
