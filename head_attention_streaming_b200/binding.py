@@ -296,7 +296,7 @@ def attn_fwd_splitkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, n_spl
                      workspace: torch.Tensor | None = None, out: torch.Tensor | None = None,
                      lse: torch.Tensor | None = None, return_lse: bool = True, stream=None):
     """Key-split attention forward through ``attn_fwd_splitkv`` of the C ABI
-    (masks 0 and 2). ``workspace`` (float32, CUDA) is allocated here when not
+    (masks 0, 1, 2). ``workspace`` (float32, CUDA) is allocated here when not
     given, sized for the split count the library chooses. Returns
     ``(out, lse, splits_used)``.
     """

@@ -304,9 +304,19 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
     return x;
   }
   if (CAUSAL) {
-    x.n0 = cdiv(min(p.Lk, p.kv_offset + x.r0 + kTileRows), kTileRows);
-    x.n1 = cdiv(min(p.Lk, p.kv_offset + x.r0 + 2 * kTileRows), kTileRows);
-    x.j0 = 0;
+    const int lim0 = cdiv(min(p.Lk, p.kv_offset + x.r0 + kTileRows), kTileRows);
+    const int lim1 = cdiv(min(p.Lk, p.kv_offset + x.r0 + 2 * kTileRows), kTileRows);
+    if constexpr (SPLIT) {
+      // this split's tiles a tile can see; 0 when the split starts past its
+      // last row's limit (its partial is then empty: O = 0, LSE = -inf)
+      x.j0 = x.split * p.split_tiles;
+      x.n0 = max(0, min(lim0, x.j0 + p.split_tiles) - x.j0);
+      x.n1 = max(0, min(lim1, x.j0 + p.split_tiles) - x.j0);
+    } else {
+      x.n0 = lim0;
+      x.n1 = lim1;
+      x.j0 = 0;
+    }
   } else if constexpr (SPLIT) {
     const int total = cdiv(p.kv_limit, kTileRows);
     x.j0 = x.split * p.split_tiles;
@@ -515,6 +525,24 @@ __device__ __forceinline__ void mma_role(const int t, const FwdParams& p, uint32
     const int n = t ? x.n1 : x.n0;  // KV tiles this query tile uses
     const int s = WINDOW ? (t ? x.s1 : x.s0) : 0;  // ... starting this many tiles into the stream
     ok = mbar_wait(bar(kBarQFull + t), uit & 1, abort_flag, kFaultMmaQFull, p.timeout_ns);
+    if (CAUSAL && SPLIT && n == 0) {
+      // no key of this split is visible to the tile: release Q and pass the
+      // unit's tiles through. O is neither written nor signalled: the softmax
+      // decodes the same empty tile and writes the empty partial itself (an
+      // O-full commit here, with no hand-shake from the softmax, could complete
+      // the barrier's phase twice before the softmax looked at it)
+      if (!ok) break;
+      mma_commit(bar(kBarQEmpty + t));
+      for (int j = 0; j < x.nu && ok; ++j) {
+        for (int kv = 0; kv < 2 && ok; ++kv) {
+          const int idx = kv_it + 2 * j + kv;
+          if (!kv_full(idx)) { ok = false; break; }
+          mbar_arrive(bar(kBarKvEmpty + idx % C::kStages));
+        }
+      }
+      kv_it += 2 * x.nu;
+      continue;
+    }
     if constexpr (WINDOW) {
       // tiles before this query tile's range pass through the ring; release
       // this thread's share once each has landed
@@ -927,11 +955,25 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
     if constexpr (SPLIT) {
       // key split: float32 O / l of this split's keys, each thread its own
       // row (d contiguous floats), straight from registers; LSE of the split
+      if (CAUSAL && n == 0) {
+        // the tile sees no key of this split (the MMA issuer left O alone)
+        const int row_e = x.r0 + t * kTileRows + r_in;
+        if (row_e < p.Lq) {
+          const size_t prow = ((static_cast<size_t>(x.split) * p.B + x.b) * p.Hq + x.hq) * p.Lq + row_e;
+          float* dst = p.o_part + prow * D;
+#pragma unroll 1
+          for (int c = 0; c < D; c += 4) *reinterpret_cast<float4*>(dst + c) = make_float4(0.f, 0.f, 0.f, 0.f);
+          p.lse_part[prow] = -INFINITY;
+        }
+        continue;
+      }
       bool ok = mbar_wait(bar_o, ocnt & 1, abort_flag, kFaultSoftmaxOFull, p.timeout_ns);
       if (!__all_sync(0xffffffffu, ok)) return;
       ++ocnt;
       tc_fence_after_sync();
-      const float inv_l = 1.f / l;
+      // a row that sees no key of this split (causal) leaves O = 0, LSE = -inf
+      const bool empty = !(l > 0.f);
+      const float inv_l = empty ? 0.f : 1.f / l;
       const bool in_range = row < p.Lq;
       const size_t prow = ((static_cast<size_t>(x.split) * p.B + x.b) * p.Hq + x.hq) * p.Lq + row;
       float* dst = p.o_part + prow * D;
@@ -948,7 +990,7 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
                             __uint_as_float(ov[e + 2]) * inv_l, __uint_as_float(ov[e + 3]) * inv_l);
         }
       }
-      if (in_range) p.lse_part[prow] = (ref + log2f(l)) * kLn2;
+      if (in_range) p.lse_part[prow] = empty ? -INFINITY : (ref + log2f(l)) * kLn2;
       // every TMEM read of O_t is complete (wait::ld) before the next unit's
       // P V overwrites it: that MMA waits for this warpgroup's next P
       continue;
@@ -1770,9 +1812,14 @@ int attn_fwd_impl(const void* q, const void* k, const void* v, void* o, float* l
 // KV tile count of the visible range, and the base unit count; returns the
 // split count actually used and the tiles per split (no split is empty).
 void choose_splits(int requested, int total_tiles, long long base_units, int num_sms, int* n_splits,
-                   int* split_tiles) {
+                   int* split_tiles, bool causal = false) {
   long long want = requested;
-  if (want <= 0) {
+  if (want <= 0 && causal) {
+    // causal units differ in length (the diagonal), so splitting only pays
+    // while the units do not fill the SMs on their own
+    want = base_units >= num_sms ? 1 : num_sms / base_units;
+    if (want > 32) want = 32;
+  } else if (want <= 0) {
     // fewest waves per unit of work: ceil(units * n / SMs) / n, with 2 % per
     // extra split for the partial outputs and the merge
     double best = 1e300;
@@ -1809,7 +1856,7 @@ int splitkv_validate(const void* q, const void* k, const void* v, const void* o,
   const int valid = attn_fwd_validate(q, k, v, o, lse, B, Lq, Lk, Hq, Hkv, d, scale, causal,
                                       kv_offset, dtype, Lk);
   if (valid != ATTN_OK) return valid;
-  if (causal == ATTN_MASK_CAUSAL || n_splits < 0) return ATTN_ERR_INVALID_ARG;
+  if (n_splits < 0) return ATTN_ERR_INVALID_ARG;
   if (d == 256) return ATTN_ERR_UNSUPPORTED;  // the one-tile d = 256 kernel has no key split
   return ATTN_OK;
 }
@@ -1823,7 +1870,8 @@ int splitkv_run(const void* q, const void* k, const void* v, void* o, float* lse
                 void* stream) {
   const long long n_pairs = (Lq + 2LL * kTileRows - 1) / (2LL * kTileRows);
   const long long base_units = n_pairs * B * Hq;
-  const int kv_limit = (causal == ATTN_MASK_CHUNK) ? kv_offset + Lq : Lk;
+  // keys past kv_offset + Lq are invisible to every row under masks 1 and 2
+  const int kv_limit = (causal == ATTN_MASK_NONE) ? Lk : kv_offset + Lq;
   const int total_tiles = (kv_limit + kTileRows - 1) / kTileRows;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
@@ -1831,7 +1879,7 @@ int splitkv_run(const void* q, const void* k, const void* v, void* o, float* lse
   if (!di.ok) return ATTN_ERR_CUDA;
   if (!di.sm100) return ATTN_ERR_UNSUPPORTED;
   int ns = 1, per = total_tiles;
-  choose_splits(n_splits, total_tiles, base_units, di.num_sms, &ns, &per);
+  choose_splits(n_splits, total_tiles, base_units, di.num_sms, &ns, &per, causal == ATTN_MASK_CAUSAL);
   if (fit) {
     while (ns > 1 && attn_splitkv_workspace_bytes(B, Lq, Hq, d, ns) > workspace_bytes) {
       per = (total_tiles + ns - 2) / (ns - 1);
@@ -1873,12 +1921,22 @@ int splitkv_run(const void* q, const void* k, const void* v, void* o, float* lse
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool bf16 = dtype == ATTN_DTYPE_BF16;
   int st;
-  if (d == 128)
-    st = bf16 ? launch_fwd<128, true, false, true>(p, q, k, v, Lk, grid, s)
+  const bool cz = causal == ATTN_MASK_CAUSAL;
+  if (d == 128) {
+    if (bf16)
+      st = cz ? launch_fwd<128, true, true, true>(p, q, k, v, Lk, grid, s)
+              : launch_fwd<128, true, false, true>(p, q, k, v, Lk, grid, s);
+    else
+      st = cz ? launch_fwd<128, false, true, true>(p, q, k, v, Lk, grid, s)
               : launch_fwd<128, false, false, true>(p, q, k, v, Lk, grid, s);
-  else
-    st = bf16 ? launch_fwd<64, true, false, true>(p, q, k, v, Lk, grid, s)
+  } else {
+    if (bf16)
+      st = cz ? launch_fwd<64, true, true, true>(p, q, k, v, Lk, grid, s)
+              : launch_fwd<64, true, false, true>(p, q, k, v, Lk, grid, s);
+    else
+      st = cz ? launch_fwd<64, false, true, true>(p, q, k, v, Lk, grid, s)
               : launch_fwd<64, false, false, true>(p, q, k, v, Lk, grid, s);
+  }
   if (st != ATTN_OK) return st;
   const long long rows = 1LL * B * Hq * Lq;
   const unsigned mgrid = static_cast<unsigned>((rows * 32 + 255) / 256);

@@ -180,12 +180,17 @@ int attn_fwd_cache(const void* q, const void* k_cache, const void* v_cache, void
  * Operation: attention over disjoint key ranges, combined exactly through the
  * per-range log-sum-exp: lse = ln sum_g exp(lse_g), O = sum_g exp(lse_g - lse)
  * O_g (the softmax of the developer guide's "Multi Head Attention Definition"
- * with its normaliser summed range by range). Masks 0 and 2 only (every row
- * sees the same key range); causal returns ATTN_ERR_INVALID_ARG.
+ * with its normaliser summed range by range). All three masks: under the
+ * causal mask a query tile takes only the tiles of a range it can see, and a
+ * row that sees no key of a range contributes an empty partial (O = 0,
+ * lse_g = -inf, weight 0); range 0 always holds key 0, which every row sees.
+ * Under masks 1 and 2 the ranges cover keys below kv_offset + Lq only.
  *
  * Arguments as attn_fwd, plus:
  *   n_splits   requested number of key ranges, >= 1, or 0 to choose one from
- *              the shape and the SM count. Ranges are whole 128-key tiles,
+ *              the shape and the SM count (causal: only while the unsplit
+ *              units are fewer than the SMs, since causal units differ in
+ *              length and a second wave of them costs more than it saves). Ranges are whole 128-key tiles,
  *              ceil(tiles / n_splits) each, so the count used can be lower than
  *              requested (4 tiles asked for 3 ranges give 2); never an empty range
  *   workspace  device float32 buffer of at least

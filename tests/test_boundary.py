@@ -160,9 +160,10 @@ def test_splitkv_argument_contract_before_any_cuda_call():
     L = hasb.lib()
     base = [A, A + 0x100000, A + 0x200000, A + 0x300000, None, A + 0x400000, 1 << 20]
     tail = [1, 64, 512, 2, 1, 128, 0.1]
-    # causal is refused; a negative split count is refused; a misaligned workspace is refused
-    assert L.attn_fwd_splitkv(*base, 0, *tail, 1, 0, 0, None, None) == hasb.ATTN_ERR_INVALID_ARG
+    # a negative split count is refused; a misaligned workspace is refused; a
+    # causal offset past Lk - Lq is refused like attn_fwd's
     assert L.attn_fwd_splitkv(*base, -1, *tail, 0, 0, 0, None, None) == hasb.ATTN_ERR_INVALID_ARG
+    assert L.attn_fwd_splitkv(*base, 2, *tail, 1, 500, 0, None, None) == hasb.ATTN_ERR_INVALID_ARG
     bad = list(base)
     bad[5] = A + 0x400000 + 4
     assert L.attn_fwd_splitkv(*bad, 2, *tail, 0, 0, 0, None, None) == hasb.ATTN_ERR_INVALID_ARG

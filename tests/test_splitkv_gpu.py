@@ -65,7 +65,31 @@ def test_one_split_is_attn_fwd_bitwise():
     assert used == 1 and torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
-def test_causal_is_refused():
-    q, k, v = (t.cuda() for t in inputs.make_qkv(1, 64, 64, 2, 2, 64, torch.bfloat16, seed=13))
-    with pytest.raises(hasb.AttnError):
-        hasb.attn_fwd_splitkv(q, k, v, causal=inputs.MASK_CAUSAL)
+@pytest.mark.parametrize("B,Lq,Lk,Hq,Hkv,d,dtype,off,n", [
+    (2, 2048, 2048, 8, 8, 64, torch.float16, 0, 2),       # the FP16 causal workload's shape
+    (1, 1000, 1000, 2, 2, 128, torch.bfloat16, 0, 5),     # many ranges empty for the first tiles
+    (1, 300, 1000, 4, 2, 128, torch.bfloat16, 700, 3),    # bottom-right causal with an offset
+    (1, 16, 4096, 8, 1, 128, torch.bfloat16, 4080, 0),    # a decode-sized causal chunk, automatic split
+    (1, 130, 700, 2, 2, 64, torch.bfloat16, 0, 6),        # rows whose whole range is invisible
+])
+def test_causal(B, Lq, Lk, Hq, Hkv, d, dtype, off, n):
+    """Causal key split: empty partials (tiles or rows that see no key of a
+    range) weigh nothing in the merge."""
+    _case(B, Lq, Lk, Hq, Hkv, d, dtype, inputs.MASK_CAUSAL, off, n, seed=13 + Lq)
+
+
+@pytest.mark.parametrize("n", [3, 4, 8, 16])
+def test_causal_many_units_per_cta(n):
+    """2 x 8 heads x 8 row pairs x n ranges: several units per CTA, many of
+    them empty (ranges past a pair's diagonal) next to full ones; a lost
+    barrier phase between them would stall the kernel until its wait limit."""
+    _case(2, 2048, 2048, 8, 8, 64, torch.float16, inputs.MASK_CAUSAL, 0, n, seed=15 + n)
+    assert hasb.device_fault(clear=True) == 0
+
+
+def test_causal_one_split_is_attn_fwd_bitwise():
+    q, k, v = (t.cuda() for t in inputs.make_qkv(1, 300, 900, 4, 2, 128, torch.bfloat16, seed=14))
+    o1, l1, used = hasb.attn_fwd_splitkv(q, k, v, n_splits=1, causal=inputs.MASK_CAUSAL, kv_offset=600)
+    o2, l2 = hasb.attn_fwd(q, k, v, causal=inputs.MASK_CAUSAL, kv_offset=600)
+    torch.cuda.synchronize()
+    assert used == 1 and torch.equal(o1, o2) and torch.equal(l1, l2)

@@ -19,10 +19,11 @@ def test_symbol_is_exported():
     assert hasattr(binding.lib(), "attn_fwd_splitkv_static")
 
 
-def test_causal_is_refused_before_any_cuda_call():
+def test_invalid_call_is_refused_before_any_cuda_call():
     A = 1 << 20
     used = binding.ctypes.c_int(-7)
-    st = binding.lib().attn_fwd_splitkv_static(A, A + 0x100000, A + 0x200000, A + 0x300000, None, 2, 1,
+    # a negative split count
+    st = binding.lib().attn_fwd_splitkv_static(A, A + 0x100000, A + 0x200000, A + 0x300000, None, -2, 1,
                                                64, 512, 2, 1, 128, 0.1, 1, 0, 0,
                                                binding.ctypes.byref(used), None)
     assert st == hasb.ATTN_ERR_INVALID_ARG and used.value == -7
@@ -49,6 +50,24 @@ def test_static_scratch_matches_oracle_and_workspace_path(cuda_ok):
     assert used2 == used and torch.equal(o1, o2) and torch.equal(l1, l2)
     f64 = lambda t: t.cpu().to(torch.float64).numpy()
     o_ref, lse_ref = oracle.attention_fwd(f64(q), f64(k), f64(v), w.scale, w.mask, w.kv_offset)
+    err = abs(f64(o1) - o_ref)
+    assert err.max() <= 8e-3 and err.mean() <= 2e-4
+    assert abs(f64(l1) - lse_ref).max() <= 1e-3
+    assert hasb.device_fault(clear=True) == 0
+
+
+@pytest.mark.gpu
+def test_static_scratch_causal(cuda_ok):
+    """The causal key split through the static scratch equals the workspace
+    path bitwise and the oracle within the bars."""
+    torch.cuda.set_device(0)
+    q, k, v = (t.cuda() for t in inputs.make_qkv(1, 600, 2000, 4, 2, 128, torch.bfloat16, seed=31))
+    o1, l1, used = hasb.attn_fwd_splitkv_static(q, k, v, n_splits=4, causal=hasb.MASK_CAUSAL, kv_offset=1400)
+    o2, l2, used2 = hasb.attn_fwd_splitkv(q, k, v, n_splits=4, causal=hasb.MASK_CAUSAL, kv_offset=1400)
+    torch.cuda.synchronize()
+    assert used == used2 == 4 and torch.equal(o1, o2) and torch.equal(l1, l2)
+    f64 = lambda t: t.cpu().to(torch.float64).numpy()
+    o_ref, lse_ref = oracle.attention_fwd(f64(q), f64(k), f64(v), 1.0 / math.sqrt(128), 1, 1400)
     err = abs(f64(o1) - o_ref)
     assert err.max() <= 8e-3 and err.mean() <= 2e-4
     assert abs(f64(l1) - lse_ref).max() <= 1e-3
