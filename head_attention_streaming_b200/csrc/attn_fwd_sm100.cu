@@ -245,10 +245,15 @@ __device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
 // the same K/V head (L2 reuse). Causal units run longest first.
 // d = 256: unit u -> (b, hq, 128-row tile); p.n_pairs counts tiles here.
 // Same order as decode_unit (GQA group heads adjacent, causal longest first).
-template <bool CAUSAL>
+template <bool CAUSAL, bool SPLIT, bool WINDOW>
 __device__ __forceinline__ Unit decode_single(const FwdParams& p, int u) {
   Unit x;
-  x.split = 0;
+  if constexpr (SPLIT) {
+    x.split = u % p.n_splits;
+    u /= p.n_splits;
+  } else {
+    x.split = 0;
+  }
   int tile = u % p.n_pairs;
   int t = u / p.n_pairs;
   const int g = t % p.group;
@@ -258,10 +263,26 @@ __device__ __forceinline__ Unit decode_single(const FwdParams& p, int u) {
   x.hq = x.hkv * p.group + g;
   if (CAUSAL) tile = p.n_pairs - 1 - tile;
   x.r0 = tile * kTileRows;
-  x.j0 = 0;
   x.s0 = x.s1 = 0;
-  const int lim = CAUSAL ? min(p.Lk, p.kv_offset + x.r0 + kTileRows) : p.kv_limit;
-  x.n0 = x.n1 = x.nu = (lim + kTileRows - 1) / kTileRows;
+  if constexpr (WINDOW) {
+    // key range of the tile from its first and last real rows
+    const int first = min(x.r0, p.Lq - 1), last = min(x.r0 + kTileRows - 1, p.Lq - 1);
+    const int lo = p.win_left < 0 ? 0 : max(0, p.kv_offset + first - p.win_left);
+    const int hi = p.win_right < 0 ? p.Lk : min(p.Lk, p.kv_offset + last + p.win_right + 1);
+    x.j0 = lo / kTileRows;
+    x.n0 = x.n1 = x.nu = cdiv(hi, kTileRows) - x.j0;
+    return x;
+  }
+  const int lim = cdiv(CAUSAL ? min(p.Lk, p.kv_offset + x.r0 + kTileRows) : p.kv_limit, kTileRows);
+  if constexpr (SPLIT) {
+    // this split's tiles the tile can see (0 under the causal mask when the
+    // split starts past its last row's limit)
+    x.j0 = x.split * p.split_tiles;
+    x.n0 = x.n1 = x.nu = max(0, min(lim, x.j0 + p.split_tiles) - x.j0);
+  } else {
+    x.j0 = 0;
+    x.n0 = x.n1 = x.nu = lim;
+  }
   return x;
 }
 
@@ -437,7 +458,7 @@ __device__ __forceinline__ void load_role(const CUtensorMap* tm_q, const CUtenso
   bool aborted = false;
   for (int u = blockIdx.x; u < p.n_units && !aborted; u += gridDim.x, ++uit) {
     Unit x;
-    if constexpr (D == 256) x = decode_single<CAUSAL>(p, u);
+    if constexpr (D == 256) x = decode_single<CAUSAL, SPLIT, WINDOW>(p, u);
     else x = decode_unit<CAUSAL, SPLIT, WINDOW>(p, u);
     for (int t = 0; t < (D == 256 ? 1 : 2); ++t) {
       const uint32_t bq = bars + 8 * (kBarQEmpty + t);
@@ -1056,7 +1077,7 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
 // while the softmax works on tile j; O += P_j V_j follows once P_j is in. The
 // issuer commits kBarOFull after every P V, so the softmax knows when O may be
 // rescaled (and, after the last, read out).
-template <bool BF16, bool CAUSAL>
+template <bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW>
 __device__ __forceinline__ void mma_role_single(const FwdParams& p, uint32_t tmem, uint32_t sQ,
                                                 uint32_t sKV, uint32_t bars, volatile int* abort_flag) {
   using C = Cfg<256, 0>;
@@ -1074,8 +1095,16 @@ __device__ __forceinline__ void mma_role_single(const FwdParams& p, uint32_t tme
   int kv_it = 0, uit = 0, pcnt = 0, sc = 0;
   bool ok = true;
   for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++uit) {
-    const Unit x = decode_single<CAUSAL>(p, u);
+    const Unit x = decode_single<CAUSAL, SPLIT, WINDOW>(p, u);
     const int n = x.n0;
+    if (SPLIT && n == 0) {
+      // (causal key split) no key of this range is visible: release Q; O is
+      // neither written nor signalled, the softmax writes the empty partial
+      ok = mbar_wait(bar(kBarQFull), uit & 1, abort_flag, kFaultMmaQFull, p.timeout_ns);
+      if (!ok) break;
+      mma_commit(bar(kBarQEmpty));
+      continue;
+    }
     ok = mbar_wait(bar(kBarQFull), uit & 1, abort_flag, kFaultMmaQFull, p.timeout_ns) && kv_full(kv_it);
     if (!ok) break;
     // S(0) = Q K_0^T
@@ -1127,7 +1156,7 @@ __device__ __forceinline__ void mma_role_single(const FwdParams& p, uint32_t tme
 // tile: wait for S_j; row max; wait until P_{j-1} V_{j-1} is done (O may then
 // be rescaled and S_j's buffer partner is free); exponentials into P_j. End of
 // a unit: wait for the last P V, O / l to 16 bits straight to global memory.
-template <bool BF16, bool CAUSAL>
+template <bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW>
 __device__ __forceinline__ void softmax_role_single(const FwdParams& p, uint32_t tmem, uint32_t bars,
                                                     volatile int* abort_flag) {
   using C = Cfg<256, 0>;
@@ -1143,10 +1172,16 @@ __device__ __forceinline__ void softmax_role_single(const FwdParams& p, uint32_t
   const float sl2 = p.sl2;
   int sc = 0, ocnt = 0;
   for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
-    const Unit x = decode_single<CAUSAL>(p, u);
+    const Unit x = decode_single<CAUSAL, SPLIT, WINDOW>(p, u);
     const int n = x.n0;
     const int row = x.r0 + r_in;
-    const int row_lim = CAUSAL ? min(p.Lk, p.kv_offset + row + 1) : p.kv_limit;
+    int row_lim = CAUSAL ? min(p.Lk, p.kv_offset + row + 1) : p.kv_limit;
+    int row_lo = 0;
+    if constexpr (WINDOW) {
+      const int pos = p.kv_offset + row;
+      row_lo = p.win_left < 0 ? 0 : max(0, pos - p.win_left);
+      row_lim = p.win_right < 0 ? p.Lk : min(p.Lk, pos + p.win_right + 1);
+    }
     float ref = -INFINITY;
     float l = 0.f;
     for (int j = 0; j < n; ++j) {
@@ -1161,13 +1196,14 @@ __device__ __forceinline__ void softmax_role_single(const FwdParams& p, uint32_t
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(tS + 32 * c, r + 32 * c);
       tmem_wait_ld_x128(r);
-      const int key0 = j * kTileRows;
+      const int key0 = (x.j0 + j) * kTileRows;
       const int lim = row_lim - key0;
-      const bool partial = lim < kTileRows;
+      const int lim_lo = WINDOW ? row_lo - key0 : 0;
+      const bool partial = lim < kTileRows || lim_lo > 0;
       if (partial) {
 #pragma unroll
         for (int c = 0; c < 128; ++c)
-          if (c >= lim) r[c] = __float_as_uint(-INFINITY);
+          if (c >= lim || c < lim_lo) r[c] = __float_as_uint(-INFINITY);
       }
       float m_tile;
       {  // three-input max tree
@@ -1216,10 +1252,46 @@ __device__ __forceinline__ void softmax_role_single(const FwdParams& p, uint32_t
       }
       float sum[4] = {0.f, 0.f, 0.f, 0.f};
       if (__any_sync(0xffffffffu, partial))
-        exp_tile<BF16, true>(r, sl2, -ref, lim, 0, sum, tS, bar_ph, bar_p, 0u, false, lane);
+        exp_tile<BF16, true>(r, sl2, -ref, lim, lim_lo, sum, tS, bar_ph, bar_p, 0u, false, lane);
       else
-        exp_tile<BF16, false>(r, sl2, -ref, lim, 0, sum, tS, bar_ph, bar_p, 0u, false, lane);
+        exp_tile<BF16, false>(r, sl2, -ref, lim, lim_lo, sum, tS, bar_ph, bar_p, 0u, false, lane);
       l += (sum[0] + sum[1]) + (sum[2] + sum[3]);
+    }
+    if constexpr (SPLIT) {
+      // float32 O / l and the LSE of this key range; a row (or the whole
+      // tile) that sees no key of the range writes O = 0, LSE = -inf
+      const bool in_range = row < p.Lq;
+      const size_t prow = ((static_cast<size_t>(x.split) * p.B + x.b) * p.Hq + x.hq) * p.Lq + row;
+      float* dst = p.o_part + prow * D;
+      if (n == 0) {
+        if (in_range) {
+#pragma unroll 1
+          for (int c = 0; c < D; c += 4) *reinterpret_cast<float4*>(dst + c) = make_float4(0.f, 0.f, 0.f, 0.f);
+          p.lse_part[prow] = -INFINITY;
+        }
+        continue;
+      }
+      bool ok = mbar_wait(bar_o, ocnt & 1, abort_flag, kFaultSoftmaxOFull, p.timeout_ns);
+      if (!__all_sync(0xffffffffu, ok)) return;
+      ++ocnt;
+      tc_fence_after_sync();
+      const bool empty = !(l > 0.f);
+      const float inv_l = empty ? 0.f : 1.f / l;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t ov[32];
+        tmem_ld_32x32b_x32(tO + 32 * c, ov);
+        tmem_wait_ld_x32(ov);
+        if (in_range) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(dst + 32 * c + e) =
+                make_float4(__uint_as_float(ov[e]) * inv_l, __uint_as_float(ov[e + 1]) * inv_l,
+                            __uint_as_float(ov[e + 2]) * inv_l, __uint_as_float(ov[e + 3]) * inv_l);
+        }
+      }
+      if (in_range) p.lse_part[prow] = empty ? -INFINITY : (ref + log2f(l)) * kLn2;
+      continue;
     }
     // the last P V, then O / l straight to global memory
     bool ok = mbar_wait(bar_o, ocnt & 1, abort_flag, kFaultSoftmaxOFull, p.timeout_ns);
@@ -1321,13 +1393,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     // one query tile: warps 0-3 softmax, warp 8 loads, warp 9 issues the MMAs
     if (warp < 8) {
       regs_increase<kRegsSoftmax>();
-      if (warp < 4) softmax_role_single<BF16, CAUSAL>(p, tmem, bars, abort_flag);
+      if (warp < 4) softmax_role_single<BF16, CAUSAL, SPLIT, WINDOW>(p, tmem, bars, abort_flag);
     } else {
       regs_decrease<kRegsProducer>();
       if (warp == 8 && lane == 0)
         load_role<D, BF16, CAUSAL, SPLIT, WINDOW, F8>(&tm_q, &tm_k, &tm_v, p, sQ, sKV, bars, abort_flag);
       else if (warp == 9 && lane == 0)
-        mma_role_single<BF16, CAUSAL>(p, tmem, sQ, sKV, bars, abort_flag);
+        mma_role_single<BF16, CAUSAL, SPLIT, WINDOW>(p, tmem, sQ, sKV, bars, abort_flag);
     }
   } else if (warp < 8) {
     regs_increase<kRegsSoftmax>();
@@ -1754,7 +1826,6 @@ int attn_fwd_impl(const void* q, const void* k, const void* v, void* o, float* l
                                       window ? ATTN_MASK_CHUNK : causal, kv_offset, dtype, kv_rows);
   if (valid != ATTN_OK) return valid;
   if (window && (win_left < -1 || win_right < -1)) return ATTN_ERR_INVALID_ARG;
-  if (window && d == 256) return ATTN_ERR_UNSUPPORTED;
   // units: pairs of 128-row query tiles; single tiles at d = 256
   const long long rows_per_unit = d == 256 ? kTileRows : 2LL * kTileRows;
   const long long n_pairs = (Lq + rows_per_unit - 1) / rows_per_unit;
@@ -1789,6 +1860,9 @@ int attn_fwd_impl(const void* q, const void* k, const void* v, void* o, float* l
   const bool bf16 = dtype == ATTN_DTYPE_BF16;
   if (window) {
     p.kv_limit = Lk;
+    if (d == 256)
+      return bf16 ? launch_fwd<256, true, false, false, true>(p, q, k, v, kv_rows, grid, s)
+                  : launch_fwd<256, false, false, false, true>(p, q, k, v, kv_rows, grid, s);
     if (d == 128)
       return bf16 ? launch_fwd<128, true, false, false, true>(p, q, k, v, kv_rows, grid, s)
                   : launch_fwd<128, false, false, false, true>(p, q, k, v, kv_rows, grid, s);
@@ -1857,7 +1931,6 @@ int splitkv_validate(const void* q, const void* k, const void* v, const void* o,
                                       kv_offset, dtype, Lk);
   if (valid != ATTN_OK) return valid;
   if (n_splits < 0) return ATTN_ERR_INVALID_ARG;
-  if (d == 256) return ATTN_ERR_UNSUPPORTED;  // the one-tile d = 256 kernel has no key split
   return ATTN_OK;
 }
 
@@ -1868,7 +1941,9 @@ int splitkv_run(const void* q, const void* k, const void* v, void* o, float* lse
                 size_t workspace_bytes, bool fit, int n_splits, int B, int Lq, int Lk, int Hq,
                 int Hkv, int d, float scale, int causal, int kv_offset, int dtype, int* splits_used,
                 void* stream) {
-  const long long n_pairs = (Lq + 2LL * kTileRows - 1) / (2LL * kTileRows);
+  // units: pairs of 128-row query tiles; single tiles at d = 256
+  const long long rows_per_unit = d == 256 ? kTileRows : 2LL * kTileRows;
+  const long long n_pairs = (Lq + rows_per_unit - 1) / rows_per_unit;
   const long long base_units = n_pairs * B * Hq;
   // keys past kv_offset + Lq are invisible to every row under masks 1 and 2
   const int kv_limit = (causal == ATTN_MASK_NONE) ? Lk : kv_offset + Lq;
@@ -1922,7 +1997,14 @@ int splitkv_run(const void* q, const void* k, const void* v, void* o, float* lse
   const bool bf16 = dtype == ATTN_DTYPE_BF16;
   int st;
   const bool cz = causal == ATTN_MASK_CAUSAL;
-  if (d == 128) {
+  if (d == 256) {
+    if (bf16)
+      st = cz ? launch_fwd<256, true, true, true>(p, q, k, v, Lk, grid, s)
+              : launch_fwd<256, true, false, true>(p, q, k, v, Lk, grid, s);
+    else
+      st = cz ? launch_fwd<256, false, true, true>(p, q, k, v, Lk, grid, s)
+              : launch_fwd<256, false, false, true>(p, q, k, v, Lk, grid, s);
+  } else if (d == 128) {
     if (bf16)
       st = cz ? launch_fwd<128, true, true, true>(p, q, k, v, Lk, grid, s)
               : launch_fwd<128, true, false, true>(p, q, k, v, Lk, grid, s);
@@ -1940,7 +2022,10 @@ int splitkv_run(const void* q, const void* k, const void* v, void* o, float* lse
   if (st != ATTN_OK) return st;
   const long long rows = 1LL * B * Hq * Lq;
   const unsigned mgrid = static_cast<unsigned>((rows * 32 + 255) / 256);
-  if (d == 128) {
+  if (d == 256) {
+    if (bf16) split_merge_kernel<256, true><<<mgrid, 256, 0, s>>>(p.o_part, p.lse_part, o, lse, ns, B, Lq, Hq, d);
+    else split_merge_kernel<256, false><<<mgrid, 256, 0, s>>>(p.o_part, p.lse_part, o, lse, ns, B, Lq, Hq, d);
+  } else if (d == 128) {
     if (bf16) split_merge_kernel<128, true><<<mgrid, 256, 0, s>>>(p.o_part, p.lse_part, o, lse, ns, B, Lq, Hq, d);
     else split_merge_kernel<128, false><<<mgrid, 256, 0, s>>>(p.o_part, p.lse_part, o, lse, ns, B, Lq, Hq, d);
   } else {

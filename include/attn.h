@@ -66,8 +66,7 @@ typedef enum {
  *   d    head_dim, a power of two 16..256 (the pages' range): 16 and 32 run
  *        through the 64-wide kernel (its TMA boxes read the columns past d as
  *        zero and store only d columns); 256 runs one 128-row query tile per
- *        work unit (its tensor memory holds S twice and O once); the key
- *        split and the sliding window return ATTN_ERR_UNSUPPORTED at 256
+ *        work unit (its tensor memory holds S twice and O once)
  *   scale  finite, >= 0 (1/sqrt(d) in the pages)
  *   causal attn_mask_t: 0 none, 1 causal, 2 streaming chunk
  *   kv_offset  cache position of query row 0: 0 for mask 0; for masks 1 and 2,

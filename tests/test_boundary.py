@@ -80,13 +80,9 @@ def test_invalid_arguments_are_rejected_before_any_launch(kw):
     assert _call(**kw) == hasb.ATTN_ERR_INVALID_ARG
 
 
-def test_d256_key_split_and_window_are_unsupported():
-    L = hasb.lib()
-    base = [A, A + 0x1000000, A + 0x2000000, A + 0x3000000, None, A + 0x4000000, 1 << 24]
-    assert L.attn_fwd_splitkv(*base, 2, 1, 64, 512, 2, 1, 256, 0.1, 0, 0, 0, None, None) == \
-        hasb.ATTN_ERR_UNSUPPORTED
-    assert L.attn_fwd_window(A, A + 0x1000000, A + 0x2000000, A + 0x3000000, None, 1, 64, 512, 2, 1, 256,
-                             0.1, 8, 8, 0, 0, None) == hasb.ATTN_ERR_UNSUPPORTED
+def test_head_dims_outside_the_pages_range_are_invalid():
+    for d in (8, 48, 512):
+        assert _call(d=d) == hasb.ATTN_ERR_INVALID_ARG
 
 
 def test_python_binding_rejects_cpu_tensors():

@@ -128,14 +128,37 @@ def test_d256_large_scores_rescale_and_cache_prefix():
     _check(o.cpu(), lse.cpu(), o_ref, lse_ref, "bf16", what="d=256 cache", output_ulp=True)
 
 
-def test_d256_deterministic_and_split_window_refused():
+def test_d256_deterministic():
     q, k, v = (t.cuda() for t in _qkv(1, 300, 500, 2, 2, 256, torch.bfloat16, seed=5))
     a, la = hasb.attn_fwd(q, k, v)
     b, lb = hasb.attn_fwd(q, k, v)
     torch.cuda.synchronize()
     assert torch.equal(a, b) and torch.equal(la, lb)
-    for call in (lambda: hasb.attn_fwd_splitkv(q, k, v, n_splits=2),
-                 lambda: hasb.attn_fwd_window(q, k, v, window=(10, 10))):
-        with pytest.raises(hasb.AttnError) as e:
-            call()
-        assert e.value.status == hasb.ATTN_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("window,off", [((100, 20), 500), ((0, 0), 0), ((-1, 64), 200)])
+def test_d256_window(window, off):
+    q, k, v = _qkv(1, 300, 900, 4, 2, 256, torch.bfloat16, seed=8)
+    scale = 1.0 / 16
+    o, lse = hasb.attn_fwd_window(q.cuda(), k.cuda(), v.cuda(), window=window, scale=scale, kv_offset=off)
+    torch.cuda.synchronize()
+    ref = oracle.attention_fwd(f64(q), f64(k), f64(v), scale, oracle.MASK_WINDOW, off, window=window)
+    _check(o.cpu(), lse.cpu(), *ref, "bf16", what=f"d=256 window {window}", output_ulp=True)
+
+
+@pytest.mark.parametrize("B,Lq,Lk,Hq,Hkv,dtype,mask,off,n", [
+    (1, 64, 3000, 4, 1, torch.bfloat16, 0, 0, 5),        # short chunk, long keys
+    (1, 200, 1500, 2, 2, torch.float16, 2, 1300, 0),     # chunk mask, automatic split
+    (2, 640, 640, 2, 2, torch.bfloat16, 1, 0, 3),        # causal: empty tiles and rows
+    (1, 700, 700, 8, 8, torch.bfloat16, 1, 0, 6),        # causal, several units per CTA
+])
+def test_d256_split(B, Lq, Lk, Hq, Hkv, dtype, mask, off, n):
+    q, k, v = _qkv(B, Lq, Lk, Hq, Hkv, 256, dtype, seed=21 + Lq)
+    scale = 1.0 / 16
+    o, lse, used = hasb.attn_fwd_splitkv(q.cuda(), k.cuda(), v.cuda(), n_splits=n, scale=scale,
+                                         causal=mask, kv_offset=off)
+    torch.cuda.synchronize()
+    ref = oracle.attention_fwd(f64(q), f64(k), f64(v), scale, mask, off)
+    _check(o.cpu(), lse.cpu(), *ref, "bf16" if dtype == torch.bfloat16 else "fp16",
+           what=f"d=256 split {used}", output_ulp=True)
+    assert hasb.device_fault(clear=True) == 0
