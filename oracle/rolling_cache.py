@@ -27,6 +27,8 @@ Readings where the pages are silent (each is listed in the design doc):
 * Every query of the chunk sees every visible key (the chunk's own K/V are in
   the cache before it is queried, and the self-attention SDPA is non-causal),
   so the result does not depend on where the keys sit in storage.
+* After-cache RoPE (``stream_attention_after_rope``): positions are
+  cache-relative, the index of a key in the visible set in stream order.
 """
 
 from __future__ import annotations
@@ -60,4 +62,37 @@ def stream_attention(q_chunks, k_all, v_all, chunk: int, sink: int, window: int,
         k = np.asarray(k_all)[:, idx]
         v = np.asarray(v_all)[:, idx]
         out.append(attention_fwd(q, k, v, scale, MASK_NONE, 0))
+    return out
+
+
+def stream_attention_after_rope(q_chunks, k_all, v_all, chunk: int, sink: int, window: int,
+                                scale: float, angles, style: int):
+    """Per-chunk outputs with RoPE applied after the cache update.
+
+    developer guide, "Multi Head Attention Definition" (RoPE after the K/V
+    cache update: the cache keeps unrotated keys; right before attention the
+    current queries and every visible cached key are rotated with the angles of
+    their current positions) and "Generic Multi Head Attention Interface" (for
+    after-cache RoPE the angle table covers the query and every visible cache
+    position; cached keys take cache-relative frequencies).
+
+    Reading (listed in the design doc): a visible key's current position is its
+    index in the visible set in stream order (sinks first, then the window
+    oldest first, the current chunk last); the chunk's queries take the
+    positions of the chunk's own keys, the last ``chunk`` of them.
+
+    q_chunks: list of [B, C, Hq, d] (already normalised, unrotated); k_all,
+    v_all: [B, T, Hkv, d] as written into the cache (normalised, unrotated);
+    angles: [R, d] expanded per-feature angle table of positions 0 .. R - 1.
+    Returns a list of (o, lse) as ``stream_attention``.
+    """
+    from .prologue import rope
+    out = []
+    ang = np.asarray(angles, dtype=np.float64)
+    for c, q in enumerate(q_chunks):
+        idx = visible_tokens(c, chunk, sink, window)
+        R = len(idx)
+        k = rope(np.asarray(k_all)[:, idx], ang[:R], style)
+        qr = rope(np.asarray(q), ang[R - chunk:R], style)
+        out.append(attention_fwd(qr, k, np.asarray(v_all)[:, idx], scale, MASK_NONE, 0))
     return out

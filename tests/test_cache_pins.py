@@ -105,3 +105,81 @@ def test_sizes_must_be_whole_chunks(bad):
     kw.update(bad)
     with pytest.raises(ValueError):
         rc.visible_tokens(2, kw["chunk"], kw["sink"], kw["window"])
+
+
+# ------------------------------------------------------------ after-cache RoPE
+
+def _linear_angles(R, d, base=10000.0):
+    """Expanded interleaved table: feature pair r of position p at angle p * base^(-2r/d)."""
+    inv = base ** (-np.arange(0, d, 2) / d)
+    ang = np.repeat(np.arange(R)[:, None] * inv[None, :], 2, axis=1)
+    return ang
+
+
+def _rot_pairs(x, theta):
+    """Interleaved rotation written as complex multiplication (x [.., d], theta [d/2])."""
+    z = x[..., 0::2] + 1j * x[..., 1::2]
+    z = z * np.exp(1j * theta)
+    y = np.empty_like(x)
+    y[..., 0::2], y[..., 1::2] = z.real, z.imag
+    return y
+
+
+def _before(q_chunks, k, v, C, sink, W, scale, ang):
+    """Before-cache reference: every token rotated once at its absolute position."""
+    from oracle.prologue import ROPE_INTERLEAVED, rope
+    T = k.shape[1]
+    kr = rope(k, ang[:T], ROPE_INTERLEAVED)
+    qr = [rope(q, ang[c * C:(c + 1) * C], ROPE_INTERLEAVED) for c, q in enumerate(q_chunks)]
+    return rc.stream_attention(qr, kr, v, C, sink, W, scale)
+
+
+def test_after_cache_rope_without_eviction_equals_before_cache():
+    """No key evicted: cache-relative positions are the absolute ones."""
+    q, k, v = _stream(24, 4, 2, 16, seed=41)
+    C = 8
+    qc = [q[:, c * C:(c + 1) * C] for c in range(3)]
+    ang = _linear_angles(24, 16)
+    a = rc.stream_attention_after_rope(qc, k, v, C, 0, 24, 0.3, ang, 1)
+    b = _before(qc, k, v, C, 0, 24, 0.3, ang)
+    for (oa, la), (ob, lb) in zip(a, b):
+        np.testing.assert_allclose(oa, ob, rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(la, lb, rtol=1e-12, atol=1e-12)
+
+
+def test_after_cache_rope_window_only_matches_before_cache_after_eviction():
+    """RoPE scores depend on position differences only, so a sink-free window
+    (cache-relative positions = absolute ones minus a constant) gives the
+    before-cache result even after evictions."""
+    q, k, v = _stream(40, 2, 2, 16, seed=42)
+    C = 8
+    qc = [q[:, c * C:(c + 1) * C] for c in range(5)]
+    a = rc.stream_attention_after_rope(qc, k, v, C, 0, 16, 0.3, _linear_angles(16, 16), 1)
+    b = _before(qc, k, v, C, 0, 16, 0.3, _linear_angles(40, 16))
+    for (oa, la), (ob, lb) in zip(a, b):
+        np.testing.assert_allclose(oa, ob, rtol=1e-9, atol=1e-9)
+        np.testing.assert_allclose(la, lb, rtol=1e-9, atol=1e-9)
+
+
+def test_after_cache_rope_with_sinks_brute_force():
+    """With a sink the cache-relative positions close the gap between the sink
+    and the window (unlike before-cache RoPE); checked against a direct loop
+    over the visible keys with complex-number rotations."""
+    q, k, v = _stream(32, 2, 1, 8, seed=43)
+    C, sink, W = 4, 4, 8
+    qc = [q[:, c * C:(c + 1) * C] for c in range(8)]
+    ang = _linear_angles(12, 8)
+    got = rc.stream_attention_after_rope(qc, k, v, C, sink, W, 0.4, ang, 1)
+    for c in (2, 5, 7):
+        vis = [t for t in range(min(sink, max(0, (c + 1) * C - W)))] + \
+              list(range(max(0, (c + 1) * C - W), (c + 1) * C))
+        R = len(vis)
+        for h in range(2):
+            for i in range(C):
+                qi = _rot_pairs(qc[c][0, i, h], ang[R - C + i, 0::2])
+                s = np.array([0.4 * qi @ _rot_pairs(k[0, t, 0], ang[j, 0::2]) for j, t in enumerate(vis)])
+                w = np.exp(s - s.max())
+                o = (w[:, None] * v[0, vis, 0]).sum(0) / w.sum()
+                np.testing.assert_allclose(got[c][0][0, i, h], o, rtol=1e-10, atol=1e-12)
+    before = _before(qc, k, v, C, sink, W, 0.4, _linear_angles(32, 8))
+    assert np.abs(got[7][0] - before[7][0]).max() > 1e-3   # the sink's distance changed
