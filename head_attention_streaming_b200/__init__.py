@@ -10,7 +10,7 @@ from .binding import (ATTN_ERR_CUDA, ATTN_ERR_INVALID_ARG, ATTN_ERR_TIMEOUT, ATT
                       NORM_NONE, ROPE_INTERLEAVED, ROPE_NONE, ROPE_SPLIT, AttnError, attn_fwd,
                       attn_fwd_cache, attn_fwd_host, attn_fwd_splitkv, attn_fwd_splitkv_static,
                       attn_fwd_window, attn_fwd_fp8, attn_fwd_fp8_scaled, fp8_cast, fp8_cast_vt,
-                      fp8_quantize_tokens, fp8_quantize_vt, qk_prologue,
+                      fp8_quantize_tokens, fp8_quantize_vt, qk_prologue, rope_after_cache,
                       splitkv_workspace_bytes, stream_update,
                       device_fault, lib, library_path, selftest_exp2, selftest_mma,
                       selftest_wait_timeout,
@@ -23,6 +23,6 @@ __all__ = ["attn_fwd", "attn_fwd_host", "AttnError", "lib", "library_path", "sta
            "NORM_INNER", "ROPE_NONE", "ROPE_INTERLEAVED", "ROPE_SPLIT", "attn_fwd_cache", "stream_update",
            "attn_fwd_splitkv", "splitkv_workspace_bytes", "attn_fwd_splitkv_static", "attn_fwd_window",
            "attn_fwd_fp8", "fp8_cast", "fp8_cast_vt", "attn_fwd_fp8_scaled", "fp8_quantize_tokens",
-           "fp8_quantize_vt", "BlockKVCache"]
+           "fp8_quantize_vt", "rope_after_cache", "BlockKVCache"]
 
 from .cache import BlockKVCache  # noqa: E402

@@ -67,6 +67,8 @@ _SIGNATURES = {
     "attn_fp8_quantize_vt": (ctypes.c_int, [ctypes.c_void_p] * 3 + [ctypes.c_int] * 6 + [ctypes.c_void_p]),
     "attn_fwd_fp8_scaled": (ctypes.c_int, [ctypes.c_void_p] * 8 + [ctypes.c_int] * 9 +
                             [ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
+    "attn_rope_after_cache": (ctypes.c_int, [ctypes.c_void_p] * 5 + [ctypes.c_int] * 2 + [ctypes.c_void_p] +
+                              [ctypes.c_int] * 9 + [ctypes.c_void_p]),
     "attn_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "attn_device_fault": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint), ctypes.c_int]),
     "attn_set_wait_timeout_ns": (ctypes.c_int, [ctypes.c_ulonglong]),
@@ -561,6 +563,40 @@ def attn_fwd_fp8_scaled(q8: torch.Tensor, sq: torch.Tensor, k8: torch.Tensor, sk
     if st != ATTN_OK:
         raise AttnError(st, "attn_fwd_fp8_scaled")
     return out, lse
+
+
+def rope_after_cache(q: torch.Tensor, k_cache: torch.Tensor, Lk: int, angles: torch.Tensor, *,
+                     rope_style: int, q_row0: int = 0, k_rows: torch.Tensor | None = None,
+                     q_out: torch.Tensor | None = None, k_rot: torch.Tensor | None = None, stream=None):
+    """After-cache RoPE through ``attn_rope_after_cache``: q [B, Lq, Hq, d]
+    rotated with angle rows q_row0.., and the first ``Lk`` slots of k_cache
+    [B, S, Hkv, d] rotated into the same slots of k_rot with angle rows
+    ``k_rows`` (int32 [Lk] on the device; None: the slot index). Returns
+    ``(q_out, k_rot)``."""
+    _check_cuda("q", q, 4)
+    _check_cuda("k_cache", k_cache, 4)
+    if q.dtype not in DTYPE_CODES or k_cache.dtype != q.dtype:
+        raise ValueError("q and k_cache must share one dtype, bf16 or fp16")
+    if not angles.is_cuda or angles.dtype != torch.float32 or not angles.is_contiguous() or angles.dim() != 2:
+        raise ValueError("angles must be a contiguous float32 CUDA tensor [rows, d]")
+    B, Lq, Hq, d = q.shape
+    S, Hkv = k_cache.shape[1], k_cache.shape[2]
+    if k_rows is not None and (not k_rows.is_cuda or k_rows.dtype != torch.int32
+                               or not k_rows.is_contiguous() or k_rows.numel() < Lk):
+        raise ValueError("k_rows must be a contiguous int32 CUDA tensor of at least Lk entries")
+    if q_out is None:
+        q_out = torch.empty_like(q)
+    if k_rot is None:
+        k_rot = torch.empty_like(k_cache)
+    elif k_rot.shape != k_cache.shape or k_rot.dtype != k_cache.dtype or not k_rot.is_contiguous():
+        raise ValueError("k_rot must be a contiguous tensor shaped and typed like k_cache")
+    st = lib().attn_rope_after_cache(_ptr(q), _ptr(q_out), _ptr(k_cache), _ptr(k_rot), _ptr(angles),
+                                     angles.shape[0], int(q_row0), _ptr(k_rows), B, Lq, int(Lk), S, Hq,
+                                     Hkv, d, int(rope_style), DTYPE_CODES[q.dtype],
+                                     _stream_handle(stream, q.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_rope_after_cache")
+    return q_out, k_rot
 
 
 def attn_fwd_host(q_host, k_host, v_host, o_host, lse_host, q_dev, k_dev, v_dev, o_dev, lse_dev, *,

@@ -103,17 +103,42 @@ class BlockKVCache:
 
     # ----------------------------------------------------------- one chunk step
 
+    def cache_positions(self, chunk_idx: int) -> list[int]:
+        """Cache-relative position of every valid slot once chunk ``chunk_idx``
+        is written: the slot's index among the visible keys in stream order
+        (sinks, then the window oldest first; the current chunk last)."""
+        valid = self.valid_length(chunk_idx)
+        rows = list(range(valid))
+        if chunk_idx >= self.sink_chunks + self.window_chunks:
+            # ring full: ring position r holds the window's ((r - r_oldest) mod W)-th chunk
+            r_oldest = (chunk_idx + 1 - self.sink_chunks) % self.window_chunks
+            C, W = self.chunk_size, self.window_size
+            for s in range(self.sink_size, valid):
+                rows[s] = self.sink_size + (s - self.sink_size - r_oldest * C) % W
+        return rows
+
     def attend(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, scale: float | None = None,
                norm_scope: int = binding.NORM_NONE, eps: float = 1e-6, gamma_q=None, gamma_k=None,
                rope_style: int = binding.ROPE_NONE, angles_q=None, angles_k=None,
+               rope_after_cache: bool = False, angles_cache=None,
                out: torch.Tensor | None = None, lse: torch.Tensor | None = None, stream=None):
         """The attention call of one streaming step, between before_update and
-        after_update: Q/K normalisation and before-cache RoPE of the chunk, its
-        K/V written into the reserved slots (one launch), then attention of the
-        chunk's queries over every valid cached key (one launch).
+        after_update.
 
-        q: [B, C, Hq, d]; k, v: [B, C, H, d] (C = chunk_size). ``angles_*`` are
-        the chunk's [C, d] angle tables (its absolute positions). Returns
+        Before-cache RoPE (default): Q/K normalisation and RoPE of the chunk,
+        its K/V written into the reserved slots (one launch), then attention of
+        the chunk's queries over every valid cached key (one launch);
+        ``angles_q`` / ``angles_k`` are the chunk's [C, d] angle tables (its
+        absolute positions).
+
+        After-cache RoPE (``rope_after_cache=True``): the chunk's K is written
+        normalised but unrotated; then the queries and every valid cached key
+        are rotated with their cache-relative positions into a scratch copy of
+        the K cache (one launch) and the attention runs on that copy.
+        ``angles_cache`` is the [R, d] angle table of cache positions 0 .. R - 1
+        (R at least the valid length); ``angles_q`` / ``angles_k`` are unused.
+
+        q: [B, C, Hq, d]; k, v: [B, C, H, d] (C = chunk_size). Returns
         ``(out, lse)``.
         """
         if self._pending is None:
@@ -121,9 +146,29 @@ class BlockKVCache:
         chunk_idx, slot = self._pending
         if k.shape != (self.batch, self.chunk_size, self.heads, self.head_dim):
             raise ValueError("k must be [batch, chunk_size, heads, head_dim]")
-        q_rot = binding.stream_update(k, v, self.k, self.v, slot, q=q, norm_scope=norm_scope, eps=eps,
-                                      gamma_q=gamma_q, gamma_k=gamma_k, rope_style=rope_style,
-                                      angles_q=angles_q, angles_k=angles_k, stream=stream)
+        valid = self.valid_length(chunk_idx)
+        if not rope_after_cache:
+            q_rot = binding.stream_update(k, v, self.k, self.v, slot, q=q, norm_scope=norm_scope, eps=eps,
+                                          gamma_q=gamma_q, gamma_k=gamma_k, rope_style=rope_style,
+                                          angles_q=angles_q, angles_k=angles_k, stream=stream)
+            self._written = True
+            return binding.attn_fwd_cache(q_rot, self.k, self.v, valid, scale=scale,
+                                          causal=binding.MASK_NONE, out=out, lse=lse, stream=stream)
+        if rope_style == binding.ROPE_NONE or angles_cache is None:
+            raise ValueError("after-cache RoPE needs a rope_style and angles_cache")
+        if angles_cache.dim() != 2 or angles_cache.shape[0] < valid:
+            raise ValueError("angles_cache must be [R, d] with R >= the valid cache length")
+        q_norm = binding.stream_update(k, v, self.k, self.v, slot, q=q, norm_scope=norm_scope, eps=eps,
+                                       gamma_q=gamma_q, gamma_k=gamma_k, rope_style=binding.ROPE_NONE,
+                                       stream=stream)
         self._written = True
-        return binding.attn_fwd_cache(q_rot, self.k, self.v, self.valid_length(chunk_idx), scale=scale,
+        if getattr(self, "_k_rot", None) is None:
+            self._k_rot = torch.empty_like(self.k)
+            self._rows = torch.empty(self.capacity, dtype=torch.int32, device=self.k.device)
+        host_rows = torch.tensor(self.cache_positions(chunk_idx), dtype=torch.int32).pin_memory()
+        self._rows[:valid].copy_(host_rows, non_blocking=True)
+        q_rot, _ = binding.rope_after_cache(q_norm, self.k, valid, angles_cache, rope_style=rope_style,
+                                            q_row0=valid - self.chunk_size, k_rows=self._rows,
+                                            q_out=q_norm, k_rot=self._k_rot, stream=stream)
+        return binding.attn_fwd_cache(q_rot, self._k_rot, self.v, valid, scale=scale,
                                       causal=binding.MASK_NONE, out=out, lse=lse, stream=stream)

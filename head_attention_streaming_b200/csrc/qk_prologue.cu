@@ -46,6 +46,12 @@ struct ProTensor {
   int L, H;
   int ystride, yoff;
   int raw;              // copy only: neither normalised nor rotated (V)
+  // angle row of token position l: rows[l] when rows is set (a per-token
+  // position map, e.g. cache slot -> cache-relative position), else l + row_off;
+  // clamped to the table's n_rows rows
+  const int* rows;
+  int row_off, n_rows;
+  int xstride;  // tokens per batch of the input (L, or a cache's S)
 };
 
 struct ProParams {
@@ -110,7 +116,8 @@ __global__ void __launch_bounds__(kThreads) qk_prologue_kernel(const ProParams p
   const int per_head = d / 16;                  // items per head
   const int sh = __ffs(per_head) - 1;           // log2(per_head)
   const int items = T.H * per_head;             // items of the token
-  const uint16_t* x = static_cast<const uint16_t*>(T.x) + static_cast<size_t>(token) * T.H * d;
+  const uint16_t* x = static_cast<const uint16_t*>(T.x) +
+                      (static_cast<size_t>(bat) * T.xstride + pos) * T.H * d;
   uint16_t* y = static_cast<uint16_t*>(T.y) +
                 (static_cast<size_t>(bat) * T.ystride + T.yoff + pos) * T.H * d;
   // intra-head item index is the same for every item this thread handles
@@ -122,7 +129,9 @@ __global__ void __launch_bounds__(kThreads) qk_prologue_kernel(const ProParams p
     // pair r: first feature a_r = 2r (interleaved) or r (split-half)
     if (!raw && threadIdx.x < d / 2) {
       const int a = split ? threadIdx.x : 2 * threadIdx.x;
-      sincosf(T.angles[static_cast<size_t>(pos) * d + a], &sn_s[threadIdx.x], &cs_s[threadIdx.x]);
+      int arow = T.rows != nullptr ? __ldg(T.rows + pos) : pos + T.row_off;
+      arow = arow < 0 ? 0 : (arow >= T.n_rows ? T.n_rows - 1 : arow);
+      sincosf(T.angles[static_cast<size_t>(arow) * d + a], &sn_s[threadIdx.x], &cs_s[threadIdx.x]);
     }
   }
   float ghead[16];
@@ -311,8 +320,8 @@ extern "C" int attn_qk_prologue(const void* q, void* q_out, const void* k, void*
   }
 
   ProParams p{};
-  p.t[0] = ProTensor{q, q_out, norm_scope ? gamma_q : nullptr, angles_q, Lq, Hq, Lq, 0, 0};
-  p.t[1] = ProTensor{k, k_out, norm_scope ? gamma_k : nullptr, angles_k, Lk, Hkv, Lk, 0, 0};
+  p.t[0] = ProTensor{q, q_out, norm_scope ? gamma_q : nullptr, angles_q, Lq, Hq, Lq, 0, 0, nullptr, 0, Lq, Lq};
+  p.t[1] = ProTensor{k, k_out, norm_scope ? gamma_k : nullptr, angles_k, Lk, Hkv, Lk, 0, 0, nullptr, 0, Lk, Lk};
   p.tok_end[0] = B * Lq;
   p.tok_end[1] = p.tok_end[2] = static_cast<int>(tokens);
   p.d = d;
@@ -365,9 +374,9 @@ extern "C" int attn_stream_update(const void* q, void* q_out, const void* k, con
   }
 
   ProParams p{};
-  p.t[0] = ProTensor{q, q_out, norm_scope ? gamma_q : nullptr, angles_q, L, Hq, L, 0, 0};
-  p.t[1] = ProTensor{k, k_cache, norm_scope ? gamma_k : nullptr, angles_k, L, Hkv, S, slot, 0};
-  p.t[2] = ProTensor{v, v_cache, nullptr, nullptr, L, Hkv, S, slot, 1};
+  p.t[0] = ProTensor{q, q_out, norm_scope ? gamma_q : nullptr, angles_q, L, Hq, L, 0, 0, nullptr, 0, L, L};
+  p.t[1] = ProTensor{k, k_cache, norm_scope ? gamma_k : nullptr, angles_k, L, Hkv, S, slot, 0, nullptr, 0, L, L};
+  p.t[2] = ProTensor{v, v_cache, nullptr, nullptr, L, Hkv, S, slot, 1, nullptr, 0, 0, L};
   p.tok_end[0] = static_cast<int>(tok_q);
   p.tok_end[1] = static_cast<int>(tok_q + tok_kv);
   p.tok_end[2] = static_cast<int>(tok_q + 2 * tok_kv);
@@ -377,5 +386,44 @@ extern "C" int attn_stream_update(const void* q, void* q_out, const void* k, con
   (void)cudaGetLastError();
   launch_prologue(p, dtype == ATTN_DTYPE_BF16, norm_scope, rope_style,
                   static_cast<unsigned>(p.tok_end[2]), s);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+extern "C" int attn_rope_after_cache(const void* q, void* q_out, const void* k_cache, void* k_rot,
+                                     const float* angles, int n_angle_rows, int q_row0,
+                                     const int* k_rows, int B, int Lq, int Lk, int S, int Hq, int Hkv,
+                                     int d, int rope_style, int dtype, void* stream) {
+  // ---- arguments (all checked before any CUDA call)
+  if (q == nullptr || q_out == nullptr || k_cache == nullptr || k_rot == nullptr || angles == nullptr)
+    return ATTN_ERR_INVALID_ARG;
+  if (dtype != ATTN_DTYPE_BF16 && dtype != ATTN_DTYPE_FP16) return ATTN_ERR_INVALID_ARG;
+  if (rope_style != ATTN_ROPE_INTERLEAVED && rope_style != ATTN_ROPE_SPLIT) return ATTN_ERR_INVALID_ARG;
+  if (B < 1 || Lq < 1 || Lk < 1 || S < Lk || Hq < 1 || Hkv < 1 || n_angle_rows < 1) return ATTN_ERR_INVALID_ARG;
+  if (q_row0 < 0 || static_cast<long long>(q_row0) + Lq > n_angle_rows) return ATTN_ERR_INVALID_ARG;
+  if (k_rows == nullptr && Lk > n_angle_rows) return ATTN_ERR_INVALID_ARG;
+  if (d < 16 || d > 256 || (d & (d - 1)) != 0) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(q_out, 16) || !aligned(k_cache, 16) || !aligned(k_rot, 16) ||
+      !aligned(angles, 4) || (k_rows != nullptr && !aligned(k_rows, 4)))
+    return ATTN_ERR_INVALID_ARG;
+  const long long nq = 1LL * B * Lq * Hq * d, nk = 1LL * B * S * Hkv * d;
+  if (1LL * B * (Lq + Lk) > 0x7fffffffLL || 1LL * Hq * d > (1 << 20) || 1LL * Hkv * d > (1 << 20))
+    return ATTN_ERR_INVALID_ARG;
+  if (q_out != q && overlap(q_out, nq * 2, q, nq * 2)) return ATTN_ERR_INVALID_ARG;
+  if (overlap(k_rot, nk * 2, k_cache, nk * 2) || overlap(q_out, nq * 2, k_rot, nk * 2) ||
+      overlap(q_out, nq * 2, k_cache, nk * 2) || overlap(k_rot, nk * 2, q, nq * 2))
+    return ATTN_ERR_INVALID_ARG;
+
+  ProParams p{};
+  p.t[0] = ProTensor{q, q_out, nullptr, angles, Lq, Hq, Lq, 0, 0, nullptr, q_row0, n_angle_rows, Lq};
+  // the first Lk slots of each batch's cache, in storage order, to the same slots of k_rot
+  p.t[1] = ProTensor{k_cache, k_rot, nullptr, angles, Lk, Hkv, S, 0, 0, k_rows, 0, n_angle_rows, S};
+  p.tok_end[0] = B * Lq;
+  p.tok_end[1] = p.tok_end[2] = B * (Lq + Lk);
+  p.d = d;
+  p.eps = 0.f;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  (void)cudaGetLastError();
+  launch_prologue(p, dtype == ATTN_DTYPE_BF16, ATTN_NORM_NONE, rope_style, static_cast<unsigned>(p.tok_end[2]),
+                  st);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }

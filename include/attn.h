@@ -322,6 +322,33 @@ int attn_stream_update(const void* q, void* q_out, const void* k, const void* v,
                        int Hq, int Hkv, int d, int norm_scope, float eps, int rope_style, int dtype,
                        void* stream);
 
+/*
+ * attn_rope_after_cache — RoPE after the K/V cache update (developer guide,
+ * "Multi Head Attention Definition": the cache keeps unrotated keys, and right
+ * before attention the current queries and every visible cached key are
+ * rotated with the angles of their current positions, again at every step).
+ *
+ *   q, q_out   device [B, Lq, Hq, d] (16-bit, dtype): queries, rotated with
+ *              angle rows q_row0 .. q_row0 + Lq - 1; q_out may be q (in place)
+ *   k_cache    device [B, S, Hkv, d]: its first Lk slots are read
+ *   k_rot      device [B, S, Hkv, d]: slot s < Lk receives k_cache slot s
+ *              rotated with angle row k_rows[s] (device int32 [Lk]; NULL: row
+ *              s); other slots are not written
+ *   angles     device float32 [n_angle_rows, d], the expanded per-feature
+ *              angle table of positions 0 .. n_angle_rows - 1 (the pages'
+ *              cache-relative rope_freqs); rows read from k_rows are clamped
+ *              to the table
+ *   rope_style ATTN_ROPE_INTERLEAVED or ATTN_ROPE_SPLIT; no normalisation
+ *              (the cache holds keys already normalised)
+ * One launch, asynchronous on `stream`. Errors: arguments checked before any
+ * CUDA call (ATTN_ERR_INVALID_ARG; ATTN_ERR_UNSUPPORTED for d outside the
+ * powers of two 16..256); k_rot may overlap nothing else.
+ */
+int attn_rope_after_cache(const void* q, void* q_out, const void* k_cache, void* k_rot,
+                          const float* angles, int n_angle_rows, int q_row0, const int* k_rows, int B,
+                          int Lq, int Lk, int S, int Hq, int Hkv, int d, int rope_style, int dtype,
+                          void* stream);
+
 /* Short English text of a status code (static storage). */
 const char* attn_status_string(int status);
 

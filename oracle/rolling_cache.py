@@ -66,7 +66,7 @@ def stream_attention(q_chunks, k_all, v_all, chunk: int, sink: int, window: int,
 
 
 def stream_attention_after_rope(q_chunks, k_all, v_all, chunk: int, sink: int, window: int,
-                                scale: float, angles, style: int):
+                                scale: float, angles, style: int, round_rotated=None):
     """Per-chunk outputs with RoPE applied after the cache update.
 
     developer guide, "Multi Head Attention Definition" (RoPE after the K/V
@@ -84,7 +84,9 @@ def stream_attention_after_rope(q_chunks, k_all, v_all, chunk: int, sink: int, w
     q_chunks: list of [B, C, Hq, d] (already normalised, unrotated); k_all,
     v_all: [B, T, Hkv, d] as written into the cache (normalised, unrotated);
     angles: [R, d] expanded per-feature angle table of positions 0 .. R - 1.
-    Returns a list of (o, lse) as ``stream_attention``.
+    ``round_rotated``, if given, is applied to the rotated queries and keys
+    (a path that stores them in a 16-bit type rounds there; the default keeps
+    them exact). Returns a list of (o, lse) as ``stream_attention``.
     """
     from .prologue import rope
     out = []
@@ -94,5 +96,7 @@ def stream_attention_after_rope(q_chunks, k_all, v_all, chunk: int, sink: int, w
         R = len(idx)
         k = rope(np.asarray(k_all)[:, idx], ang[:R], style)
         qr = rope(np.asarray(q), ang[R - chunk:R], style)
+        if round_rotated is not None:
+            k, qr = round_rotated(k), round_rotated(qr)
         out.append(attention_fwd(qr, k, np.asarray(v_all)[:, idx], scale, MASK_NONE, 0))
     return out

@@ -252,3 +252,23 @@ def test_fp8_quantize_argument_contract():
     assert L.attn_fp8_quantize_vt(x, y, s, 1, 100, 1, 32, 112, 0, None) == hasb.ATTN_ERR_INVALID_ARG     # d
     assert L.attn_fp8_quantize_vt(x, y, None, 1, 100, 1, 128, 112, 0, None) == hasb.ATTN_ERR_INVALID_ARG
     assert L.attn_fp8_quantize_vt(x, y, s, 1, 100, 1, 128, 104, 0, None) == hasb.ATTN_ERR_INVALID_ARG    # pitch
+
+
+def test_rope_after_cache_argument_contract():
+    L = hasb.lib()
+    args = dict(q=A, qo=A + 0x100000, kc=A + 0x200000, kr=A + 0x300000, ang=A + 0x400000, R=300, q0=260,
+                rows=None, B=1, Lq=40, Lk=250, S=300, Hq=2, Hkv=1, d=64, style=2, dtype=0)
+
+    def call(**kw):
+        a = dict(args)
+        a.update(kw)
+        return L.attn_rope_after_cache(*[a[n] for n in ("q", "qo", "kc", "kr", "ang", "R", "q0", "rows", "B",
+                                                        "Lq", "Lk", "S", "Hq", "Hkv", "d", "style",
+                                                        "dtype")], None)
+    assert call(style=0) == hasb.ATTN_ERR_INVALID_ARG          # RoPE is the point
+    assert call(q0=261) == hasb.ATTN_ERR_INVALID_ARG           # query rows past the table
+    assert call(S=200) == hasb.ATTN_ERR_INVALID_ARG            # Lk > S
+    assert call(R=200) == hasb.ATTN_ERR_INVALID_ARG            # identity rows past the table
+    assert call(kr=A + 0x200000 + 64) == hasb.ATTN_ERR_INVALID_ARG  # k_rot overlaps the cache
+    assert call(ang=None) == hasb.ATTN_ERR_INVALID_ARG
+    assert call(d=512) == hasb.ATTN_ERR_UNSUPPORTED

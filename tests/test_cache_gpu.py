@@ -101,3 +101,71 @@ def test_dit_stream_full_size_through_eviction():
     rows = np.sort(np.random.default_rng(7).choice(1785, size=64, replace=False))
     _stream(1, 1785, 0, 7140, 40, 8, 128, 5, torch.bfloat16, qp.NORM_HEAD, qp.ROPE_SPLIT, seed=4,
             sample_rows=rows)
+
+
+@pytest.mark.parametrize("style,sink,window,n_chunks,dtype", [
+    (qp.ROPE_SPLIT, 128, 256, 6, torch.bfloat16),        # sink + ring, evictions from chunk 3 on
+    (qp.ROPE_INTERLEAVED, 0, 384, 5, torch.float16),     # window only, evictions from chunk 3 on
+])
+def test_after_cache_rope_stream(style, sink, window, n_chunks, dtype):
+    """RoPE after the cache update: the cache keeps normalised, unrotated K;
+    each step rotates the queries and every valid cached key with their
+    cache-relative positions (the oracle's reading) before attending."""
+    B, C, Hq, Hkv, d = 2, 128, 4, 2, 128
+    g = torch.Generator().manual_seed(50 + n_chunks)
+    T = n_chunks * C
+    q = torch.randn(B, T, Hq, d, generator=g).to(dtype)
+    k = torch.randn(B, T, Hkv, d, generator=g).to(dtype)
+    v = torch.randn(B, T, Hkv, d, generator=g).to(dtype)
+    gq = 1.0 + 0.1 * torch.randn(d, generator=g)
+    gk = 1.0 + 0.1 * torch.randn(d, generator=g)
+    ang = rope_angle_table(sink + window, d, style, 0)       # cache positions 0 .. sink + window - 1
+    scale, eps = 1.0 / math.sqrt(d), 1e-6
+    f64 = lambda t: t.to(torch.float64).numpy()
+    qn = _round16(qp.rms_norm(f64(q), f64(gq), eps, qp.NORM_HEAD), dtype)
+    kn = _round16(qp.rms_norm(f64(k), f64(gk), eps, qp.NORM_HEAD), dtype)
+    ref = rc.stream_attention_after_rope([qn[:, c * C:(c + 1) * C] for c in range(n_chunks)], kn, f64(v),
+                                         C, sink, window, scale, f64(ang), style,
+                                         round_rotated=lambda x: _round16(x, dtype))
+    cache = hasb.BlockKVCache(B, Hkv, d, C, window, sink, dtype=dtype)
+    tag = "bf16" if dtype == torch.bfloat16 else "fp16"
+    for c in range(n_chunks):
+        sl = slice(c * C, (c + 1) * C)
+        cache.before_update(c)
+        o, lse = cache.attend(q[:, sl].contiguous().cuda(), k[:, sl].contiguous().cuda(),
+                              v[:, sl].contiguous().cuda(), scale=scale, norm_scope=hasb.NORM_HEAD, eps=eps,
+                              gamma_q=gq.cuda(), gamma_k=gk.cuda(), rope_style=style,
+                              rope_after_cache=True, angles_cache=ang.cuda())
+        torch.cuda.synchronize()
+        cache.after_update(c)
+        _check(o.cpu(), lse.cpu(), *ref[c], tag, what=f"after-cache chunk {c}", output_ulp=True)
+    # the cache itself keeps the normalised, unrotated keys of the visible chunks
+    stored = cache.k.cpu().to(torch.float64).numpy()
+    last = n_chunks - 1
+    for c2 in sorted(set(int(t) // C for t in rc.visible_tokens(last, C, sink, window))):
+        s0 = cache.slot_of(c2)
+        want = kn[:, c2 * C:(c2 + 1) * C]
+        assert np.abs(stored[:, s0:s0 + C] - want).max() <= 2 ** -7 * np.abs(want).max(), c2
+
+
+def test_rope_after_cache_rows_and_batch_stride():
+    """attn_rope_after_cache on its own: a B = 2 cache with S > Lk (batch
+    stride S), a row map that permutes the slots, slots past Lk untouched."""
+    B, S, Lk, Lq, H, d = 2, 300, 250, 40, 2, 64
+    g = torch.Generator().manual_seed(61)
+    kc = torch.randn(B, S, H, d, generator=g).to(torch.bfloat16)
+    q = torch.randn(B, Lq, 4, d, generator=g).to(torch.bfloat16)
+    ang = rope_angle_table(Lk, d, qp.ROPE_SPLIT, 0)
+    perm = torch.randperm(Lk, generator=g).to(torch.int32)
+    k_rot = torch.full((B, S, H, d), 3.0, dtype=torch.bfloat16, device="cuda")
+    q_out, _ = hasb.rope_after_cache(q.cuda(), kc.cuda(), Lk, ang.cuda(), rope_style=hasb.ROPE_SPLIT,
+                                     q_row0=Lk - Lq, k_rows=perm.cuda(), k_rot=k_rot)
+    torch.cuda.synchronize()
+    f64 = lambda t: t.to(torch.float64).numpy()
+    a = f64(ang)
+    want_k = _round16(qp.rope(f64(kc[:, :Lk]), a[perm.long().numpy()], qp.ROPE_SPLIT), torch.bfloat16)
+    want_q = _round16(qp.rope(f64(q), a[Lk - Lq:], qp.ROPE_SPLIT), torch.bfloat16)
+    got_k = f64(k_rot.cpu())
+    assert np.abs(got_k[:, :Lk] - want_k).max() <= 2 ** -7 * np.abs(want_k).max()
+    assert np.all(got_k[:, Lk:] == 3.0)
+    assert np.abs(f64(q_out.cpu()) - want_q).max() <= 2 ** -7 * np.abs(want_q).max()
