@@ -768,9 +768,10 @@ __device__ __forceinline__ void store_role(const CUtensorMap* tm_o, const FwdPar
       ok = mbar_wait(bars + 8 * kBarStgFull, scnt & 1, abort_flag, kFaultStore, p.timeout_ns);
       if (!ok) break;
       ++scnt;
+      const int dt = p.d > 0 ? p.d : D;  // a chunk wholly past the tensor's head dim is not stored
 #pragma unroll
       for (int c = 0; c < C::kOChunks; ++c)
-        tma_store_4d(tm_o, sStg + c * C::kChunkBytes, c * 64, x.hq, x.r0 + t * kTileRows, x.b);
+        if (c * 64 < dt) tma_store_4d(tm_o, sStg + c * C::kChunkBytes, c * 64, x.hq, x.r0 + t * kTileRows, x.b);
       bulk_commit_group();
       bulk_wait_group_read0();
       mbar_arrive(bars + 8 * (kBarStgFree + (1 - t)));
@@ -1035,9 +1036,9 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
       tmem_ld_32x32b_x32(tO + 32 * c, ov);
       tmem_wait_ld_x32(ov);
       if constexpr (F8 == 2) {
-        if (p.sv != nullptr) {  // V's per-channel scales
+        if (p.sv != nullptr && 32 * c < p.d) {  // V's per-channel scales (columns past d stay 0)
           const float4* sv4 =
-              reinterpret_cast<const float4*>(p.sv + (static_cast<size_t>(x.b) * p.Hkv + x.hkv) * D + 32 * c);
+              reinterpret_cast<const float4*>(p.sv + (static_cast<size_t>(x.b) * p.Hkv + x.hkv) * p.d + 32 * c);
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             const float4 f = __ldg(sv4 + e);
@@ -1702,10 +1703,13 @@ int launch_fwd(const FwdParams& p, const void* q, const void* k, const void* v, 
     // e4m3 Q / K (box: the 128-byte row of a head, 128 rows); V transposed,
     // [B, Hkv, d, kv_rows] bytes with kv_rows a multiple of 16 (box: 128 keys
     // x 128 d-rows); O bf16 as usual
-    if (!encode_e4m3_bl_hd(&tq, q, p.B, p.Lq, p.Hq, D) ||
-        !encode_e4m3_bl_hd(&tk, k, p.B, p.Lk, p.Hkv, D) ||
-        !encode_e4m3_vt(&tv, v, p.B, p.Lk, kv_rows, p.Hkv, D) ||
-        !encode_bl_hd(&to, p.o, p.B, p.Lq, p.Hq, D, true))
+    // d < 128: the 128-byte boxes read the columns (V^T: the rows) past d as
+    // zero, and the O chunks past d are clipped or skipped
+    const int dt = p.d > 0 ? p.d : D;
+    if (dt > D || !encode_e4m3_bl_hd(&tq, q, p.B, p.Lq, p.Hq, dt) ||
+        !encode_e4m3_bl_hd(&tk, k, p.B, p.Lk, p.Hkv, dt) ||
+        !encode_e4m3_vt(&tv, v, p.B, p.Lk, kv_rows, p.Hkv, dt) ||
+        !encode_bl_hd(&to, p.o, p.B, p.Lq, p.Hq, dt, true))
       return ATTN_ERR_CUDA;
   } else {
     const int dt = p.d > 0 ? p.d : D;
@@ -2099,7 +2103,7 @@ int fp8_fwd(const void* q8, const void* k8, const void* vt8, const float* sq, co
         (sv != nullptr && ranges_overlap(o, q_elems * 2, sv, 4ull * B * Hkv * d)))
       return ATTN_ERR_INVALID_ARG;
   }
-  if (d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (d > 128) return ATTN_ERR_UNSUPPORTED;  // d < 128 runs the 128-wide kernel on zero-filled columns
   // ---- device
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
@@ -2107,6 +2111,7 @@ int fp8_fwd(const void* q8, const void* k8, const void* vt8, const float* sq, co
   if (!di.ok) return ATTN_ERR_CUDA;
   if (!di.sm100) return ATTN_ERR_UNSUPPORTED;
   FwdParams p{};
+  p.d = d;
   p.o = o;
   p.lse = lse;
   p.B = B; p.Lq = Lq; p.Lk = Lk; p.Hq = Hq; p.Hkv = Hkv; p.group = Hq / Hkv;

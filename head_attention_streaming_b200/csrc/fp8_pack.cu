@@ -60,14 +60,16 @@ __global__ void __launch_bounds__(256) cast_vt_kernel(const uint16_t* __restrict
   const int tx = threadIdx.x % 64, ty = threadIdx.x / 64;  // 64 x 4
   for (int r = ty; r < 64; r += 4) {
     const int j = j0 + r;
-    tile[r][tx] = j < Lk ? to_f32<BF16>(v[((static_cast<size_t>(b) * Lk + j) * H + h) * d + c0 + tx]) : 0.f;
+    tile[r][tx] = (j < Lk && c0 + tx < d)
+                      ? to_f32<BF16>(v[((static_cast<size_t>(b) * Lk + j) * H + h) * d + c0 + tx])
+                      : 0.f;
   }
   __syncthreads();
   // each thread writes 4 consecutive keys of one feature row
   const int c = threadIdx.x / 16, jj = (threadIdx.x % 16) * 4;
   for (int cc = c; cc < 64; cc += 16) {
     const int j = j0 + jj;
-    if (j >= Lk) continue;
+    if (j >= Lk || c0 + cc >= d) continue;
     uint8_t* dst = vt + ((static_cast<size_t>(b) * H + h) * d + c0 + cc) * pitch + j;
     const uint32_t w = e4m3x2(tile[jj][cc], tile[jj + 1][cc]) | (e4m3x2(tile[jj + 2][cc], tile[jj + 3][cc]) << 16);
     if (j + 4 <= Lk) {
@@ -175,13 +177,15 @@ __global__ void __launch_bounds__(256) quantize_vt_kernel(const uint16_t* __rest
   const int tx = threadIdx.x % 64, ty = threadIdx.x / 64;
   for (int r = ty; r < 64; r += 4) {
     const int j = j0 + r;
-    tile[r][tx] = j < Lk ? to_f32<BF16>(v[((static_cast<size_t>(b) * Lk + j) * H + h) * d + c0 + tx]) : 0.f;
+    tile[r][tx] = (j < Lk && c0 + tx < d)
+                      ? to_f32<BF16>(v[((static_cast<size_t>(b) * Lk + j) * H + h) * d + c0 + tx])
+                      : 0.f;
   }
   __syncthreads();
   const int c = threadIdx.x / 16, jj = (threadIdx.x % 16) * 4;
   for (int cc = c; cc < 64; cc += 16) {
     const int j = j0 + jj;
-    if (j >= Lk) continue;
+    if (j >= Lk || c0 + cc >= d) continue;
     const float sc = slice_scale(__uint_as_float(amax_bits[static_cast<size_t>(bh) * d + c0 + cc]));
     uint8_t* dst = vt + ((static_cast<size_t>(b) * H + h) * d + c0 + cc) * pitch + j;
     const uint32_t w = e4m3x2(__fdiv_rn(tile[jj][cc], sc), __fdiv_rn(tile[jj + 1][cc], sc)) |
@@ -233,13 +237,13 @@ extern "C" int attn_fp8_cast_vt(const void* v, void* vt, int B, int Lk, int Hkv,
                                 int dtype, void* stream) {
   if (v == nullptr || vt == nullptr) return ATTN_ERR_INVALID_ARG;
   if (dtype != ATTN_DTYPE_BF16 && dtype != ATTN_DTYPE_FP16) return ATTN_ERR_INVALID_ARG;
-  if (B < 1 || Lk < 1 || Hkv < 1 || d < 64 || d % 64 != 0 || pitch < Lk || pitch % 16 != 0)
+  if (B < 1 || Lk < 1 || Hkv < 1 || d < 16 || d > 256 || (d & (d - 1)) != 0 || pitch < Lk || pitch % 16 != 0)
     return ATTN_ERR_INVALID_ARG;
   if (!aligned(v, 16) || !aligned(vt, 16)) return ATTN_ERR_INVALID_ARG;
   const size_t nv = 2ull * B * Lk * Hkv * d, nvt = 1ull * B * Hkv * d * pitch;
   if (overlap(v, nv, vt, nvt)) return ATTN_ERR_INVALID_ARG;
   if (static_cast<long long>(B) * Hkv > 65535) return ATTN_ERR_INVALID_ARG;
-  dim3 grid((Lk + 63) / 64, d / 64, B * Hkv);
+  dim3 grid((Lk + 63) / 64, (d + 63) / 64, B * Hkv);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   (void)cudaGetLastError();
   if (dtype == ATTN_DTYPE_BF16)
@@ -279,7 +283,7 @@ extern "C" int attn_fp8_quantize_vt(const void* v, void* vt, float* sv, int B, i
                                     int pitch, int dtype, void* stream) {
   if (v == nullptr || vt == nullptr || sv == nullptr) return ATTN_ERR_INVALID_ARG;
   if (dtype != ATTN_DTYPE_BF16 && dtype != ATTN_DTYPE_FP16) return ATTN_ERR_INVALID_ARG;
-  if (B < 1 || Lk < 1 || Hkv < 1 || d < 64 || d > 256 || (d & (d - 1)) != 0 || pitch < Lk || pitch % 16 != 0)
+  if (B < 1 || Lk < 1 || Hkv < 1 || d < 16 || d > 256 || (d & (d - 1)) != 0 || pitch < Lk || pitch % 16 != 0)
     return ATTN_ERR_INVALID_ARG;
   if (!aligned(v, 16) || !aligned(vt, 16) || !aligned(sv, 4)) return ATTN_ERR_INVALID_ARG;
   if (static_cast<long long>(B) * Hkv > 65535) return ATTN_ERR_INVALID_ARG;
@@ -290,7 +294,7 @@ extern "C" int attn_fp8_quantize_vt(const void* v, void* vt, float* sv, int B, i
   if (cudaMemsetAsync(sv, 0, ns, st) != cudaSuccess) return ATTN_ERR_CUDA;
   const int G = d / 8, kpb = 256;
   const dim3 agrid((Lk + kpb - 1) / kpb, B * Hkv);
-  const dim3 qgrid((Lk + 63) / 64, d / 64, B * Hkv);
+  const dim3 qgrid((Lk + 63) / 64, (d + 63) / 64, B * Hkv);
   unsigned* bits = reinterpret_cast<unsigned*>(sv);
   const int n = B * Hkv * d;
   if (dtype == ATTN_DTYPE_BF16) {

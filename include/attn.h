@@ -110,15 +110,17 @@ int attn_fwd_window(const void* q, const void* k, const void* v, void* o, float*
  *
  * attn_fp8_cast_vt — V [B, Lk, Hkv, d] (16-bit, dtype) to e4m3 transposed:
  * vt[b, h, c, j] = e4m3(v[b, j, h, c]) in [B, Hkv, d, pitch] bytes, pitch >= Lk
- * and a multiple of 16 (bytes j >= Lk of a row are not written); d a multiple
- * of 64. The transposed layout makes V's tiles the K-major operand of P V.
+ * and a multiple of 16 (bytes j >= Lk of a row are not written); d a power of
+ * two 16..256. The transposed layout makes V's tiles the K-major operand of P V.
  *
  * attn_fwd_fp8 — attention forward on e4m3 operands: q8 [B, Lq, Hq, d] and
  * k8 [B, Lk, Hkv, d] e4m3, vt8 as written by attn_fp8_cast_vt (pitch
  * vt_pitch); S = scale q8 k8^T and the softmax in float32; P rounded to e4m3
  * for the P V product (the row sum uses the unrounded P); o [B, Lq, Hq, d]
  * bfloat16 and lse as attn_fwd. Masks, GQA, kv_offset and errors as attn_fwd;
- * this build runs d = 128 (other head dims: ATTN_ERR_UNSUPPORTED).
+ * this build runs d = 16, 32, 64, 128 (below 128 through the 128-wide kernel,
+ * whose 128-byte TMA boxes read the columns of Q, K and the rows of V^T past d
+ * as zero; O chunks past d are not stored); d = 256: ATTN_ERR_UNSUPPORTED.
  */
 int attn_fp8_cast(const void* x, void* y, long long n, int dtype, void* stream);
 int attn_fp8_cast_vt(const void* v, void* vt, int B, int Lk, int Hkv, int d, int pitch, int dtype,
@@ -141,7 +143,7 @@ int attn_fwd_fp8(const void* q8, const void* k8, const void* vt8, void* o, float
  * attn_fp8_quantize_vt — one scale per (batch, head, channel) of V
  * [B, Lk, Hkv, d] (the max runs over the keys): sv [B, Hkv, d] float32, codes
  * written transposed like attn_fp8_cast_vt ([B, Hkv, d, pitch]). d a power of
- * two in 64..256. Four launches on `stream` (zero sv, column maxima, codes,
+ * two in 16..256. Four launches on `stream` (zero sv, column maxima, codes,
  * maxima to scales); sv holds the scales once they complete.
  *
  * attn_fwd_fp8_scaled — attn_fwd_fp8 on scaled codes: the score of row i and
@@ -149,7 +151,8 @@ int attn_fwd_fp8(const void* q8, const void* k8, const void* vt8, void* o, float
  * [B, Hq, sq_pitch], sk [B, Hkv, sk_pitch] as attn_fp8_quantize_tokens writes
  * them, sk_pitch a multiple of 4, sk 16-byte aligned), and column c of O is
  * multiplied by sv[b, hkv, c] ([B, Hkv, d], 16-byte aligned; NULL: V cast
- * without scales). P is rounded to e4m3 as in attn_fwd_fp8. d = 128.
+ * without scales). P is rounded to e4m3 as in attn_fwd_fp8. d <= 128 as
+ * attn_fwd_fp8.
  */
 int attn_fp8_quantize_tokens(const void* x, void* y, float* s, int B, int L, int H, int d, int s_pitch,
                              int dtype, void* stream);

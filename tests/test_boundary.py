@@ -192,9 +192,8 @@ def test_fp8_attention_argument_contract(kw):
     assert hasb.lib().attn_fwd_fp8(*_fp8_args(**kw)) == hasb.ATTN_ERR_INVALID_ARG
 
 
-@pytest.mark.parametrize("d", [64, 256])
-def test_fp8_attention_other_head_dims_are_unsupported(d):
-    assert hasb.lib().attn_fwd_fp8(*_fp8_args(d=d)) == hasb.ATTN_ERR_UNSUPPORTED
+def test_fp8_attention_head_dim_256_is_unsupported():
+    assert hasb.lib().attn_fwd_fp8(*_fp8_args(d=256)) == hasb.ATTN_ERR_UNSUPPORTED
 
 
 def test_fp8_cast_argument_contract():
@@ -208,7 +207,8 @@ def test_fp8_cast_argument_contract():
     vt = [A, A + 0x100000]
     assert L.attn_fp8_cast_vt(*vt, 1, 100, 1, 128, 96, 0, None) == hasb.ATTN_ERR_INVALID_ARG  # pitch < Lk
     assert L.attn_fp8_cast_vt(*vt, 1, 100, 1, 128, 120, 0, None) == hasb.ATTN_ERR_INVALID_ARG  # pitch % 16
-    assert L.attn_fp8_cast_vt(*vt, 1, 100, 1, 96, 112, 0, None) == hasb.ATTN_ERR_INVALID_ARG   # d % 64
+    assert L.attn_fp8_cast_vt(*vt, 1, 100, 1, 96, 112, 0, None) == hasb.ATTN_ERR_INVALID_ARG   # d not 2^k
+    assert L.attn_fp8_cast_vt(*vt, 1, 100, 1, 8, 112, 0, None) == hasb.ATTN_ERR_INVALID_ARG    # d < 16
     assert L.attn_fp8_cast_vt(A, A + 0x100, 1, 100, 1, 128, 112, 0, None) == hasb.ATTN_ERR_INVALID_ARG
 
 
@@ -237,8 +237,8 @@ def test_fp8_scaled_attention_argument_contract(kw):
     assert hasb.lib().attn_fwd_fp8_scaled(*_fp8s_args(**kw)) == hasb.ATTN_ERR_INVALID_ARG
 
 
-def test_fp8_scaled_attention_other_head_dims_are_unsupported():
-    assert hasb.lib().attn_fwd_fp8_scaled(*_fp8s_args(d=64)) == hasb.ATTN_ERR_UNSUPPORTED
+def test_fp8_scaled_attention_head_dim_256_is_unsupported():
+    assert hasb.lib().attn_fwd_fp8_scaled(*_fp8s_args(d=256)) == hasb.ATTN_ERR_UNSUPPORTED
 
 
 def test_fp8_quantize_argument_contract():
@@ -249,7 +249,7 @@ def test_fp8_quantize_argument_contract():
     assert L.attn_fp8_quantize_tokens(x, y, None, 1, 10, 2, 128, 10, 0, None) == hasb.ATTN_ERR_INVALID_ARG
     assert L.attn_fp8_quantize_tokens(x, x + 64, s, 1, 10, 2, 128, 10, 0, None) == hasb.ATTN_ERR_INVALID_ARG
     assert L.attn_fp8_quantize_tokens(x, y, s, 1, 10, 2, 128, 10, 5, None) == hasb.ATTN_ERR_INVALID_ARG  # dtype
-    assert L.attn_fp8_quantize_vt(x, y, s, 1, 100, 1, 32, 112, 0, None) == hasb.ATTN_ERR_INVALID_ARG     # d
+    assert L.attn_fp8_quantize_vt(x, y, s, 1, 100, 1, 48, 112, 0, None) == hasb.ATTN_ERR_INVALID_ARG     # d
     assert L.attn_fp8_quantize_vt(x, y, None, 1, 100, 1, 128, 112, 0, None) == hasb.ATTN_ERR_INVALID_ARG
     assert L.attn_fp8_quantize_vt(x, y, s, 1, 100, 1, 128, 104, 0, None) == hasb.ATTN_ERR_INVALID_ARG    # pitch
 

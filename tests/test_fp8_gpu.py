@@ -56,7 +56,8 @@ def test_cast_is_bit_exact(dtype):
 
 
 @pytest.mark.parametrize("B,Lk,Hkv,d,pitch", [(2, 700, 3, 128, None), (1, 64, 1, 64, 128),
-                                              (1, 1, 2, 128, None), (3, 129, 2, 192, 160)])
+                                              (1, 1, 2, 128, None), (3, 129, 2, 256, 160),
+                                              (2, 300, 2, 32, None), (1, 77, 3, 16, 96)])
 def test_transposed_cast_is_bit_exact_and_leaves_the_padding(B, Lk, Hkv, d, pitch):
     g = torch.Generator().manual_seed(Lk)
     v = (torch.randn(B, Lk, Hkv, d, generator=g) * 3.0).to(torch.bfloat16)
@@ -70,8 +71,7 @@ def test_transposed_cast_is_bit_exact_and_leaves_the_padding(B, Lk, Hkv, d, pitc
     assert bool((got[..., Lk:] == 0x55).all())
 
 
-def _fp8_case(B, Lq, Lk, Hq, Hkv, mask, off, seed, rows=None):
-    d = 128
+def _fp8_case(B, Lq, Lk, Hq, Hkv, mask, off, seed, rows=None, d=128):
     q, k, v = inputs.make_qkv(B, Lq, Lk, Hq, Hkv, d, torch.bfloat16, seed=seed)
     scale = 1.0 / math.sqrt(d)
     q8, k8, vt8 = hasb.fp8_cast(q.cuda()), hasb.fp8_cast(k.cuda()), hasb.fp8_cast_vt(v.cuda())
@@ -163,8 +163,7 @@ def test_quantize_vt_is_bit_exact(B, Lk, Hkv, d):
     np.testing.assert_array_equal(sv.cpu().numpy(), s_ref[:, 0])
 
 
-def _fp8_scaled_case(B, Lq, Lk, Hq, Hkv, mask, off, seed, rows=None, mag=1.0, v_scaled=True):
-    d = 128
+def _fp8_scaled_case(B, Lq, Lk, Hq, Hkv, mask, off, seed, rows=None, mag=1.0, v_scaled=True, d=128):
     q, k, v = inputs.make_qkv(B, Lq, Lk, Hq, Hkv, d, torch.float32, seed=seed)
     q, k, v = ((t * mag).to(torch.bfloat16) for t in (q, k, v))
     scale = 1.0 / math.sqrt(d) / mag ** 2
@@ -220,3 +219,24 @@ def test_fp8_scaled_attention_keeps_small_magnitudes():
 def test_fp8_scaled_attention_video_shape_sampled_rows():
     rows = inputs.sample_rows(20480, 48, seed=6).numpy()
     _fp8_scaled_case(1, 20480, 20480, 56, 56, 0, 0, seed=9, rows=rows)
+
+
+@pytest.mark.parametrize("d", [16, 32, 64])
+def test_fp8_small_head_dims(d):
+    """d < 128 through the 128-wide e4m3 kernel (zero-filled columns, O chunks
+    past d not stored), unscaled and per-token scaled, causal and plain."""
+    _fp8_case(2, 300, 700, 4, 2, 0, 0, seed=70 + d, d=d)
+    _fp8_case(1, 257, 900, 2, 1, 1, 643, seed=71 + d, d=d)
+    _fp8_scaled_case(1, 300, 700, 4, 2, 0, 0, seed=72 + d, d=d)
+
+
+@pytest.mark.parametrize("B,Lk,Hkv,d", [(2, 700, 3, 32), (1, 65, 2, 16)])
+def test_quantize_vt_small_head_dims_bit_exact(B, Lk, Hkv, d):
+    from oracle import quantize as qz
+    v = _scaled_inputs(B, Lk, Hkv, d, seed=Lk + d)
+    codes, sv = hasb.fp8_quantize_vt(v.cuda())
+    torch.cuda.synchronize()
+    c_ref, s_ref = qz.quantize(v.to(torch.float64).numpy(), "e4m3", qz.SLICE, axis=1)
+    want = torch.from_numpy(c_ref).to(torch.float8_e4m3fn).view(torch.uint8).permute(0, 2, 3, 1)
+    assert torch.equal(codes.cpu().view(torch.uint8)[..., :Lk], want)
+    np.testing.assert_array_equal(sv.cpu().numpy(), s_ref[:, 0])
