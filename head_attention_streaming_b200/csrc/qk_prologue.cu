@@ -98,26 +98,42 @@ __device__ __forceinline__ int item_feature(int o, int e, int d, bool split) {
   return split ? (e < 8 ? o + e : o + d / 2 + e - 8) : o + e;
 }
 
+// Which tensor, position and batch block-level token index `bid` names.
+struct TokenAt {
+  ProTensor T;
+  int pos, bat;
+};
+
+__device__ __forceinline__ TokenAt token_at(const ProParams& p, int bid) {
+  TokenAt a;
+  const int which = bid < p.tok_end[0] ? 0 : (bid < p.tok_end[1] ? 1 : 2);
+  a.T = which == 0 ? p.t[0] : (which == 1 ? p.t[1] : p.t[2]);
+  const int token = bid - (which == 0 ? 0 : p.tok_end[which - 1]);  // b * L + l
+  a.pos = token % a.T.L;                                            // sequence index l
+  a.bat = token / a.T.L;
+  return a;
+}
+
+__device__ __forceinline__ int angle_row(const ProTensor& T, int pos) {
+  const int r = T.rows != nullptr ? __ldg(T.rows + pos) : pos + T.row_off;
+  return r < 0 ? 0 : (r >= T.n_rows ? T.n_rows - 1 : r);
+}
+
+// One token (all its heads) of one tensor, by the whole block: `x` holds the
+// token's H d input values and `ang` its d-entry angle row (either in global
+// memory or staged in shared memory; `ang` unused without RoPE).
 template <bool BF16, int SCOPE, int STYLE>
-__global__ void __launch_bounds__(kThreads) qk_prologue_kernel(const ProParams p) {
-  __shared__ float red[kWarps];
-  __shared__ float cs_s[128], sn_s[128];  // cos / sin of the token's d/2 pair angles
+__device__ __forceinline__ void token_body(const ProParams& p, const ProTensor& T, int pos, int bat,
+                                           const uint16_t* x, const float* ang, float* red, float* cs_s,
+                                           float* sn_s) {
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  const int bid = blockIdx.x;
-  const int which = bid < p.tok_end[0] ? 0 : (bid < p.tok_end[1] ? 1 : 2);
-  const ProTensor T = which == 0 ? p.t[0] : (which == 1 ? p.t[1] : p.t[2]);
-  const int token = bid - (which == 0 ? 0 : p.tok_end[which - 1]);  // b * L + l
-  const int pos = token % T.L;                                      // sequence index l
-  const int bat = token / T.L;
   const bool raw = T.raw != 0;
   const int d = p.d;
   constexpr bool split = STYLE == ATTN_ROPE_SPLIT;
   const int per_head = d / 16;                  // items per head
   const int sh = __ffs(per_head) - 1;           // log2(per_head)
   const int items = T.H * per_head;             // items of the token
-  const uint16_t* x = static_cast<const uint16_t*>(T.x) +
-                      (static_cast<size_t>(bat) * T.xstride + pos) * T.H * d;
   uint16_t* y = static_cast<uint16_t*>(T.y) +
                 (static_cast<size_t>(bat) * T.ystride + T.yoff + pos) * T.H * d;
   // intra-head item index is the same for every item this thread handles
@@ -129,9 +145,7 @@ __global__ void __launch_bounds__(kThreads) qk_prologue_kernel(const ProParams p
     // pair r: first feature a_r = 2r (interleaved) or r (split-half)
     if (!raw && threadIdx.x < d / 2) {
       const int a = split ? threadIdx.x : 2 * threadIdx.x;
-      int arow = T.rows != nullptr ? __ldg(T.rows + pos) : pos + T.row_off;
-      arow = arow < 0 ? 0 : (arow >= T.n_rows ? T.n_rows - 1 : arow);
-      sincosf(T.angles[static_cast<size_t>(arow) * d + a], &sn_s[threadIdx.x], &cs_s[threadIdx.x]);
+      sincosf(ang[a], &sn_s[threadIdx.x], &cs_s[threadIdx.x]);
     }
   }
   float ghead[16];
@@ -243,38 +257,163 @@ __global__ void __launch_bounds__(kThreads) qk_prologue_kernel(const ProParams p
   }
 }
 
+
+
+// One block per token, operands read straight from global memory.
+template <bool BF16, int SCOPE, int STYLE>
+__global__ void __launch_bounds__(kThreads) qk_prologue_kernel(const ProParams p) {
+  __shared__ float red[kWarps];
+  __shared__ float cs_s[128], sn_s[128];  // cos / sin of the token's d/2 pair angles
+  const TokenAt a = token_at(p, blockIdx.x);
+  const uint16_t* x = static_cast<const uint16_t*>(a.T.x) +
+                      (static_cast<size_t>(a.bat) * a.T.xstride + a.pos) * a.T.H * p.d;
+  const float* ang = (STYLE != ATTN_ROPE_NONE && a.T.raw == 0)
+                         ? a.T.angles + static_cast<size_t>(angle_row(a.T, a.pos)) * p.d
+                         : nullptr;
+  token_body<BF16, SCOPE, STYLE>(p, a.T, a.pos, a.bat, x, ang, red, cs_s, sn_s);
+}
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+
+// Persistent blocks, one token at a time, with the next token's bytes (and
+// its angle row) copied into the other of two shared-memory buffers by
+// cp.async while the current one is processed: the HBM round trip of a token
+// hides behind the work on the previous one without holding registers.
+// `buf` bytes per buffer: the largest token (H d 16-bit values) and an angle row.
+#ifndef PRO_NBUF
+#define PRO_NBUF 2
+#endif
+#ifndef PRO_MINB
+#define PRO_MINB 1
+#endif
+constexpr int kStageBufs = PRO_NBUF;  // tokens in flight per block: the current one and the next ones
+
+template <bool BF16, int SCOPE, int STYLE>
+__global__ void __launch_bounds__(kThreads, PRO_MINB) qk_prologue_staged_kernel(const ProParams p, int buf) {
+  extern __shared__ __align__(16) uint8_t stage[];
+  __shared__ float red[kWarps];
+  __shared__ float cs_s[128], sn_s[128];
+  const int total = p.tok_end[2];
+  const int d = p.d;
+  auto issue = [&](int t, int b) {
+    const TokenAt a = token_at(p, t);
+    const uint8_t* src = static_cast<const uint8_t*>(a.T.x) +
+                         (static_cast<size_t>(a.bat) * a.T.xstride + a.pos) * a.T.H * d * 2;
+    uint8_t* dst = stage + b * buf;
+    const int chunks = a.T.H * d * 2 / 16;
+    for (int k = threadIdx.x; k < chunks; k += kThreads) cp_async16(dst + 16 * k, src + 16 * k);
+    if (STYLE != ATTN_ROPE_NONE && a.T.raw == 0) {
+      const float* arow = a.T.angles + static_cast<size_t>(angle_row(a.T, a.pos)) * d;
+      uint8_t* adst = dst + buf - d * 4;
+      for (int k = threadIdx.x; k < d / 4; k += kThreads) cp_async16(adst + 16 * k, arow + 4 * k);
+    }
+  };
+  int t = blockIdx.x;
+  if (t >= total) return;
+#pragma unroll
+  for (int q = 0; q < kStageBufs - 1; ++q) {  // the first tokens
+    const int tq = t + q * static_cast<int>(gridDim.x);
+    if (tq < total) issue(tq, q);
+    cp_async_commit();
+  }
+  for (int n = 0; t < total; ++n, t += gridDim.x) {
+    const int b = n % kStageBufs;
+    const int ahead = t + (kStageBufs - 1) * static_cast<int>(gridDim.x);
+    if (ahead < total) issue(ahead, (n + kStageBufs - 1) % kStageBufs);
+    cp_async_commit();  // one group per token (empty past the last)
+    // this thread's copies of token t have landed (only the newer groups may pend) ...
+    asm volatile("cp.async.wait_group %0;" ::"n"(kStageBufs - 1) : "memory");
+    __syncthreads();    // ... and so have everyone's
+    const TokenAt a = token_at(p, t);
+    const uint8_t* sb = stage + b * buf;
+    token_body<BF16, SCOPE, STYLE>(p, a.T, a.pos, a.bat, reinterpret_cast<const uint16_t*>(sb),
+                                   reinterpret_cast<const float*>(sb + buf - d * 4), red, cs_s, sn_s);
+    __syncthreads();  // buffer b is read out before the next round refills it
+  }
+}
+
 }  // namespace hasb_pro
 
 using namespace hasb_pro;
 
 namespace {
 
+int sm_count() {
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0, n = 0;
+    sms = (cudaGetDevice(&dev) == cudaSuccess &&
+           cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0)
+              ? n
+              : 148;
+  }
+  return sms;
+}
+
+// `buf` > 0: the staged persistent kernel (as many blocks as fit on every SM,
+// never more than tokens); 0: one block per token.
+template <bool BF16, int SCOPE, int STYLE>
+void launch_kernel(const ProParams& p, unsigned tokens, int buf, cudaStream_t s) {
+  if (buf == 0) {
+    qk_prologue_kernel<BF16, SCOPE, STYLE><<<tokens, kThreads, 0, s>>>(p);
+    return;
+  }
+  auto kern = qk_prologue_staged_kernel<BF16, SCOPE, STYLE>;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, kStageBufs * buf) != cudaSuccess ||
+      per_sm < 1)
+    per_sm = 1;
+  const unsigned g = static_cast<unsigned>(sm_count() * per_sm);
+  kern<<<tokens < g ? tokens : g, kThreads, kStageBufs * buf, s>>>(p, buf);
+}
+
 template <bool BF16, int SCOPE>
-void launch_style(const ProParams& p, int style, unsigned grid, cudaStream_t s) {
+void launch_style(const ProParams& p, int style, unsigned tokens, int buf, cudaStream_t s) {
   if (style == ATTN_ROPE_NONE)
-    qk_prologue_kernel<BF16, SCOPE, ATTN_ROPE_NONE><<<grid, kThreads, 0, s>>>(p);
+    launch_kernel<BF16, SCOPE, ATTN_ROPE_NONE>(p, tokens, buf, s);
   else if (style == ATTN_ROPE_INTERLEAVED)
-    qk_prologue_kernel<BF16, SCOPE, ATTN_ROPE_INTERLEAVED><<<grid, kThreads, 0, s>>>(p);
+    launch_kernel<BF16, SCOPE, ATTN_ROPE_INTERLEAVED>(p, tokens, buf, s);
   else
-    qk_prologue_kernel<BF16, SCOPE, ATTN_ROPE_SPLIT><<<grid, kThreads, 0, s>>>(p);
+    launch_kernel<BF16, SCOPE, ATTN_ROPE_SPLIT>(p, tokens, buf, s);
 }
 
 template <bool BF16>
-void launch_scope(const ProParams& p, int scope, int style, unsigned grid, cudaStream_t s) {
+void launch_scope(const ProParams& p, int scope, int style, unsigned tokens, int buf, cudaStream_t s) {
   if (scope == ATTN_NORM_NONE)
-    launch_style<BF16, ATTN_NORM_NONE>(p, style, grid, s);
+    launch_style<BF16, ATTN_NORM_NONE>(p, style, tokens, buf, s);
   else if (scope == ATTN_NORM_HEAD)
-    launch_style<BF16, ATTN_NORM_HEAD>(p, style, grid, s);
+    launch_style<BF16, ATTN_NORM_HEAD>(p, style, tokens, buf, s);
   else
-    launch_style<BF16, ATTN_NORM_INNER>(p, style, grid, s);
+    launch_style<BF16, ATTN_NORM_INNER>(p, style, tokens, buf, s);
 }
 
-void launch_prologue(const ProParams& p, bool bf16, int scope, int style, unsigned grid,
+// Staging buffer bytes for the tensors of `p` (the largest token plus an
+// angle row, 16-byte multiple), or 0 when a token is too large for two
+// buffers in 48 KB or an angle table is not 16-byte aligned.
+int staging_bytes(const ProParams& p, int style) {
+  int tok = 0;
+  for (int i = 0; i < 3; ++i) {
+    const int n = (i == 0 ? p.tok_end[0] : p.tok_end[i] - p.tok_end[i - 1]);
+    if (n <= 0) continue;
+    const ProTensor& T = p.t[i];
+    tok = T.H * p.d * 2 > tok ? T.H * p.d * 2 : tok;
+    if (style != ATTN_ROPE_NONE && !T.raw && (reinterpret_cast<uintptr_t>(T.angles) & 15u) != 0) return 0;
+  }
+  const int buf = (tok + p.d * 4 + 15) / 16 * 16;
+  return kStageBufs * buf <= 48 * 1024 ? buf : 0;
+}
+
+void launch_prologue(const ProParams& p, bool bf16, int scope, int style, unsigned tokens,
                      cudaStream_t s) {
+  const int buf = staging_bytes(p, style);
   if (bf16)
-    launch_scope<true>(p, scope, style, grid, s);
+    launch_scope<true>(p, scope, style, tokens, buf, s);
   else
-    launch_scope<false>(p, scope, style, grid, s);
+    launch_scope<false>(p, scope, style, tokens, buf, s);
 }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
