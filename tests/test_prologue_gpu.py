@@ -134,3 +134,26 @@ def test_invalid_call_raises():
                          angles_q=torch.zeros(3 * 64, device="cuda"))  # wrong table size
     with pytest.raises(hasb.AttnError):
         hasb.qk_prologue(q, rope_style=qp.ROPE_SPLIT)  # RoPE without angles
+
+
+def test_large_tokens_take_the_one_block_per_token_kernel():
+    """A token of 64 heads x 256 features (32 KB) is too large to stage in
+    shared memory: the one-block-per-token kernel serves it, same results."""
+    _run(1, 20, 12, 64, 8, 256, torch.bfloat16, qp.NORM_HEAD, qp.ROPE_SPLIT, seed=77)
+    _run(1, 20, 12, 64, 8, 256, torch.bfloat16, qp.NORM_INNER, qp.ROPE_INTERLEAVED, seed=78)
+
+
+def test_unaligned_angle_table_takes_the_one_block_per_token_kernel():
+    """An angle table that is 4- but not 16-byte aligned cannot be copied by
+    cp.async: the direct kernel serves the call."""
+    B, L, H, d = 1, 37, 4, 64
+    q = _draw((B, L, H, d), torch.bfloat16, 81)
+    ang = rope_angle_table(L, d, qp.ROPE_SPLIT, 100)
+    buf = torch.zeros(L * d + 1, dtype=torch.float32, device="cuda")
+    buf[1:] = ang.reshape(-1).cuda()
+    ang_off = buf[1:].view(L, d)                          # data_ptr 4 bytes past a 16-byte boundary
+    assert ang_off.data_ptr() % 16 != 0
+    oq, _ = hasb.qk_prologue(q.cuda(), None, norm_scope=hasb.NORM_NONE, rope_style=hasb.ROPE_SPLIT,
+                             angles_q=ang_off)
+    torch.cuda.synchronize()
+    _check(oq, q, None, 1e-6, qp.NORM_NONE, ang, qp.ROPE_SPLIT)
