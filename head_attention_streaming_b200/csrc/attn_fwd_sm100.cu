@@ -137,6 +137,27 @@ struct CfgE4m3 {
 };
 template <>
 struct Cfg<128, 1> : CfgE4m3<1> {};
+// e4m3 at d = 256: one query tile per unit as for 16-bit d = 256; a Q / K row
+// is two 128-byte chunks (32 KB per tile), a V^T tile 256 d-rows of 128 keys;
+// P for each of the two S buffers in shared memory (16 KB each).
+template <>
+struct Cfg<256, 1> {
+  static constexpr int kChunks = 2;
+  static constexpr int kChunkBytes = kTileRows * 128;
+  static constexpr int kTileBytes = 2 * kChunkBytes;
+  static constexpr int kStages = 4;
+  static constexpr int kOChunks = 4;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffKV = kTileBytes;
+  static constexpr int kOffP = kOffKV + kStages * kTileBytes;
+  static constexpr int kOffStg = 0;
+  static constexpr int kOffSk = 0;
+  static constexpr int kOffBar = kOffP + 2 * kChunkBytes;
+  static constexpr int kSmemBytes = kOffBar + 512 + 1024;
+  static __device__ __forceinline__ uint32_t col_s(int buf) { return buf ? 128u : 0u; }
+  static __device__ __forceinline__ uint32_t col_o(int) { return 256u; }
+  static constexpr uint32_t kTmemCols = 512;
+};
 template <>
 struct Cfg<128, 2> : CfgE4m3<2> {};
 
@@ -394,8 +415,11 @@ template <int D>
 __device__ __forceinline__ void issue_qk_f8(uint32_t d_tmem, uint32_t q_lo, uint32_t k_lo) {
   constexpr uint32_t idesc = mma_idesc_f16(false, 128, 128, false, false);
 #pragma unroll
-  for (int kk = 0; kk < D / 32; ++kk)
-    mma_f8_ss_lo_flag(d_tmem, q_lo + 2 * kk, k_lo + 2 * kk, idesc, kk > 0 ? 1u : 0u);
+  for (int kk = 0; kk < D / 32; ++kk) {
+    // 4 steps of 32 bytes per 128-byte chunk, chunks kTileRows * 128 bytes apart
+    const uint32_t off = static_cast<uint32_t>(((kk >> 2) * kTileRows * 128 + (kk & 3) * 32) >> 4);
+    mma_f8_ss_lo_flag(d_tmem, q_lo + off, k_lo + off, idesc, kk > 0 ? 1u : 0u);
+  }
 }
 
 // e4m3 O += P V for half HALF of the 128 keys: A = P (shared memory, K-major),
@@ -469,8 +493,8 @@ __device__ __forceinline__ void load_role(const CUtensorMap* tm_q, const CUtenso
       const uint32_t bf = bars + 8 * (kBarQFull + t);
       mbar_arrive_expect_tx(bf, C::kTileBytes);
 #pragma unroll
-      for (int c = 0; c < C::kChunks; ++c)
-        tma_load_4d(sQ + t * C::kTileBytes + c * C::kChunkBytes, tm_q, bf, c * 64, x.hq,
+      for (int c = 0; c < C::kChunks; ++c)  // 128 bytes a chunk: 64 16-bit or 128 e4m3 elements
+        tma_load_4d(sQ + t * C::kTileBytes + c * C::kChunkBytes, tm_q, bf, c * (F8 != 0 ? 128 : 64), x.hq,
                     x.r0 + t * kTileRows, x.b, pol_q);
     }
     for (int j = 0; j < x.nu && !aborted; ++j) {
@@ -486,12 +510,15 @@ __device__ __forceinline__ void load_role(const CUtensorMap* tm_q, const CUtenso
         mbar_arrive_expect_tx(bf, C::kTileBytes);
         if constexpr (F8 != 0) {
           // K: (d, head, key, batch); transposed V: (key, d, head, batch)
-          if (kv)
-            tma_load_4d(sKV + slot * C::kTileBytes, tm_v, bf, (x.j0 + j) * kTileRows, 0, x.hkv, x.b,
-                        pol_kv);
-          else
-            tma_load_4d(sKV + slot * C::kTileBytes, tm_k, bf, 0, x.hkv, (x.j0 + j) * kTileRows, x.b,
-                        pol_kv);
+#pragma unroll
+          for (int c = 0; c < C::kChunks; ++c) {  // V^T: 128 d-rows a chunk; K: 128 bytes a chunk
+            if (kv)
+              tma_load_4d(sKV + slot * C::kTileBytes + c * C::kChunkBytes, tm_v, bf, (x.j0 + j) * kTileRows,
+                          c * 128, x.hkv, x.b, pol_kv);
+            else
+              tma_load_4d(sKV + slot * C::kTileBytes + c * C::kChunkBytes, tm_k, bf, c * 128, x.hkv,
+                          (x.j0 + j) * kTileRows, x.b, pol_kv);
+          }
         } else {
 #pragma unroll
           for (int c = 0; c < C::kChunks; ++c)
@@ -1078,10 +1105,13 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
 // while the softmax works on tile j; O += P_j V_j follows once P_j is in. The
 // issuer commits kBarOFull after every P V, so the softmax knows when O may be
 // rescaled (and, after the last, read out).
-template <bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW>
+template <bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW, int F8>
 __device__ __forceinline__ void mma_role_single(const FwdParams& p, uint32_t tmem, uint32_t sQ,
-                                                uint32_t sKV, uint32_t bars, volatile int* abort_flag) {
-  using C = Cfg<256, 0>;
+                                                uint32_t sKV, uint32_t sP, uint32_t bars,
+                                                volatile int* abort_flag) {
+  using C = Cfg<256, F8>;
+  // e4m3: P of S buffer b in shared memory (K-major, 128-byte swizzle)
+  auto p_lo = [&](int b) { return smem_desc_lo(sP + b * kTileRows * 128, 16); };
   auto bar = [&](int i) { return bars + 8 * i; };
   const uint32_t q_lo = smem_desc_lo(sQ, 16);
   auto k_lo = [&](int idx) { return smem_desc_lo(sKV + (idx % C::kStages) * C::kTileBytes, 16); };
@@ -1109,7 +1139,8 @@ __device__ __forceinline__ void mma_role_single(const FwdParams& p, uint32_t tme
     ok = mbar_wait(bar(kBarQFull), uit & 1, abort_flag, kFaultMmaQFull, p.timeout_ns) && kv_full(kv_it);
     if (!ok) break;
     // S(0) = Q K_0^T
-    issue_qk<256, BF16>(tmem + C::col_s(sc & 1), q_lo, k_lo(kv_it));
+    if constexpr (F8 != 0) issue_qk_f8<256>(tmem + C::col_s(sc & 1), q_lo, k_lo(kv_it));
+    else issue_qk<256, BF16>(tmem + C::col_s(sc & 1), q_lo, k_lo(kv_it));
     mma_commit(bar(kBarSFull + (sc & 1)));
     mma_commit(bar(kBarKvEmpty + kv_it % C::kStages));
     if (n == 1) mma_commit(bar(kBarQEmpty));
@@ -1121,7 +1152,8 @@ __device__ __forceinline__ void mma_role_single(const FwdParams& p, uint32_t tme
         // S(j+1) into the other buffer: its last P was read by a P V issued earlier
         const int knext = vidx + 1;
         if (!kv_full(knext)) { ok = false; break; }
-        issue_qk<256, BF16>(tmem + C::col_s(sc & 1), q_lo, k_lo(knext));
+        if constexpr (F8 != 0) issue_qk_f8<256>(tmem + C::col_s(sc & 1), q_lo, k_lo(knext));
+        else issue_qk<256, BF16>(tmem + C::col_s(sc & 1), q_lo, k_lo(knext));
         mma_commit(bar(kBarSFull + (sc & 1)));
         mma_commit(bar(kBarKvEmpty + knext % C::kStages));
         if (j + 1 == n - 1) mma_commit(bar(kBarQEmpty));
@@ -1133,14 +1165,16 @@ __device__ __forceinline__ void mma_role_single(const FwdParams& p, uint32_t tme
         break;
       }
       tc_fence_after_sync();
-      issue_pv_half<256, BF16, 0>(o_t, s_j, v_lo(vidx), j > 0 ? 1u : 0u);
+      if constexpr (F8 != 0) issue_pv_half_f8<256, 0>(o_t, p_lo((sc - 1) & 1), k_lo(vidx), j > 0 ? 1u : 0u);
+      else issue_pv_half<256, BF16, 0>(o_t, s_j, v_lo(vidx), j > 0 ? 1u : 0u);
       if (!mbar_wait(bar(kBarPFull), pcnt & 1, abort_flag, kFaultMmaPFull, p.timeout_ns)) {
         ok = false;
         break;
       }
       ++pcnt;
       tc_fence_after_sync();
-      issue_pv_half<256, BF16, 1>(o_t, s_j, v_lo(vidx), 1u);
+      if constexpr (F8 != 0) issue_pv_half_f8<256, 1>(o_t, p_lo((sc - 1) & 1), k_lo(vidx), 1u);
+      else issue_pv_half<256, BF16, 1>(o_t, s_j, v_lo(vidx), 1u);
       mma_commit(bar(kBarKvEmpty + vidx % C::kStages));
       mma_commit(bar(kBarOFull));
       if (j + 1 < n) ++sc;
@@ -1157,10 +1191,10 @@ __device__ __forceinline__ void mma_role_single(const FwdParams& p, uint32_t tme
 // tile: wait for S_j; row max; wait until P_{j-1} V_{j-1} is done (O may then
 // be rescaled and S_j's buffer partner is free); exponentials into P_j. End of
 // a unit: wait for the last P V, O / l to 16 bits straight to global memory.
-template <bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW>
+template <bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW, int F8>
 __device__ __forceinline__ void softmax_role_single(const FwdParams& p, uint32_t tmem, uint32_t bars,
-                                                    volatile int* abort_flag) {
-  using C = Cfg<256, 0>;
+                                                    uint32_t sP, volatile int* abort_flag) {
+  using C = Cfg<256, F8>;
   constexpr int D = 256;
   const int warp = threadIdx.x / 32;
   const int r_in = threadIdx.x % kTileRows;
@@ -1252,10 +1286,17 @@ __device__ __forceinline__ void softmax_role_single(const FwdParams& p, uint32_t
         }
       }
       float sum[4] = {0.f, 0.f, 0.f, 0.f};
-      if (__any_sync(0xffffffffu, partial))
+      if constexpr (F8 != 0) {
+        const uint32_t prow = sP + buf * kTileRows * 128 + r_in * 128;  // e4m3 P row of this S buffer
+        if (__any_sync(0xffffffffu, partial))
+          exp_tile_f8<true>(r, sl2, -ref, lim, lim_lo, sum, prow, r_in, bar_ph, bar_p, 0u, false, lane);
+        else
+          exp_tile_f8<false>(r, sl2, -ref, lim, lim_lo, sum, prow, r_in, bar_ph, bar_p, 0u, false, lane);
+      } else if (__any_sync(0xffffffffu, partial)) {
         exp_tile<BF16, true>(r, sl2, -ref, lim, lim_lo, sum, tS, bar_ph, bar_p, 0u, false, lane);
-      else
+      } else {
         exp_tile<BF16, false>(r, sl2, -ref, lim, lim_lo, sum, tS, bar_ph, bar_p, 0u, false, lane);
+      }
       l += (sum[0] + sum[1]) + (sum[2] + sum[3]);
     }
     if constexpr (SPLIT) {
@@ -1394,13 +1435,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     // one query tile: warps 0-3 softmax, warp 8 loads, warp 9 issues the MMAs
     if (warp < 8) {
       regs_increase<kRegsSoftmax>();
-      if (warp < 4) softmax_role_single<BF16, CAUSAL, SPLIT, WINDOW>(p, tmem, bars, abort_flag);
+      if (warp < 4) softmax_role_single<BF16, CAUSAL, SPLIT, WINDOW, F8>(p, tmem, bars, sP, abort_flag);
     } else {
       regs_decrease<kRegsProducer>();
       if (warp == 8 && lane == 0)
         load_role<D, BF16, CAUSAL, SPLIT, WINDOW, F8>(&tm_q, &tm_k, &tm_v, p, sQ, sKV, bars, abort_flag);
       else if (warp == 9 && lane == 0)
-        mma_role_single<BF16, CAUSAL, SPLIT, WINDOW>(p, tmem, sQ, sKV, bars, abort_flag);
+        mma_role_single<BF16, CAUSAL, SPLIT, WINDOW, F8>(p, tmem, sQ, sKV, sP, bars, abort_flag);
     }
   } else if (warp < 8) {
     regs_increase<kRegsSoftmax>();
@@ -2086,7 +2127,8 @@ int fp8_fwd(const void* q8, const void* k8, const void* vt8, const float* sq, co
   const unsigned long long vt_bytes = 1ull * B * Hkv * d * vt_pitch;
   if (q_elems * 2 >= (1ull << 40) || k_elems >= (1ull << 40) || vt_bytes >= (1ull << 40))
     return ATTN_ERR_INVALID_ARG;
-  const long long n_pairs = (Lq + 2LL * kTileRows - 1) / (2LL * kTileRows);
+  const long long rows_per_unit = d == 256 ? kTileRows : 2LL * kTileRows;  // one tile per unit at 256
+  const long long n_pairs = (Lq + rows_per_unit - 1) / rows_per_unit;
   const long long n_units = n_pairs * B * Hq;
   if (n_units > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
   if (ranges_overlap(o, q_elems * 2, q8, q_elems) || ranges_overlap(o, q_elems * 2, k8, k_elems) ||
@@ -2103,7 +2145,8 @@ int fp8_fwd(const void* q8, const void* k8, const void* vt8, const float* sq, co
         (sv != nullptr && ranges_overlap(o, q_elems * 2, sv, 4ull * B * Hkv * d)))
       return ATTN_ERR_INVALID_ARG;
   }
-  if (d > 128) return ATTN_ERR_UNSUPPORTED;  // d < 128 runs the 128-wide kernel on zero-filled columns
+  // d < 128 runs the 128-wide kernel on zero-filled columns; 256 the one-tile kernel (unscaled only)
+  if (d == 256 && scaled) return ATTN_ERR_UNSUPPORTED;
   // ---- device
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
@@ -2134,6 +2177,9 @@ int fp8_fwd(const void* q8, const void* k8, const void* vt8, const float* sq, co
   const int grid = static_cast<int>(n_units < di.num_sms ? n_units : di.num_sms);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool c = causal == ATTN_MASK_CAUSAL;
+  if (d == 256)
+    return c ? launch_fwd<256, true, true, false, false, 1>(p, q8, k8, vt8, vt_pitch, grid, s)
+             : launch_fwd<256, true, false, false, false, 1>(p, q8, k8, vt8, vt_pitch, grid, s);
   if (scaled)
     return c ? launch_fwd<128, true, true, false, false, 2>(p, q8, k8, vt8, vt_pitch, grid, s)
              : launch_fwd<128, true, false, false, false, 2>(p, q8, k8, vt8, vt_pitch, grid, s);

@@ -118,9 +118,9 @@ int attn_fwd_window(const void* q, const void* k, const void* v, void* o, float*
  * vt_pitch); S = scale q8 k8^T and the softmax in float32; P rounded to e4m3
  * for the P V product (the row sum uses the unrounded P); o [B, Lq, Hq, d]
  * bfloat16 and lse as attn_fwd. Masks, GQA, kv_offset and errors as attn_fwd;
- * this build runs d = 16, 32, 64, 128 (below 128 through the 128-wide kernel,
- * whose 128-byte TMA boxes read the columns of Q, K and the rows of V^T past d
- * as zero; O chunks past d are not stored); d = 256: ATTN_ERR_UNSUPPORTED.
+ * d = 16, 32, 64, 128, 256 (below 128 through the 128-wide kernel, whose
+ * 128-byte TMA boxes read the columns of Q, K and the rows of V^T past d as
+ * zero, with the O chunks past d not stored; 256 through the one-tile kernel).
  */
 int attn_fp8_cast(const void* x, void* y, long long n, int dtype, void* stream);
 int attn_fp8_cast_vt(const void* v, void* vt, int B, int Lk, int Hkv, int d, int pitch, int dtype,
@@ -151,8 +151,8 @@ int attn_fwd_fp8(const void* q8, const void* k8, const void* vt8, void* o, float
  * [B, Hq, sq_pitch], sk [B, Hkv, sk_pitch] as attn_fp8_quantize_tokens writes
  * them, sk_pitch a multiple of 4, sk 16-byte aligned), and column c of O is
  * multiplied by sv[b, hkv, c] ([B, Hkv, d], 16-byte aligned; NULL: V cast
- * without scales). P is rounded to e4m3 as in attn_fwd_fp8. d <= 128 as
- * attn_fwd_fp8.
+ * without scales). P is rounded to e4m3 as in attn_fwd_fp8. d <= 128 (256:
+ * ATTN_ERR_UNSUPPORTED).
  */
 int attn_fp8_quantize_tokens(const void* x, void* y, float* s, int B, int L, int H, int d, int s_pitch,
                              int dtype, void* stream);

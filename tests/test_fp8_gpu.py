@@ -240,3 +240,24 @@ def test_quantize_vt_small_head_dims_bit_exact(B, Lk, Hkv, d):
     want = torch.from_numpy(c_ref).to(torch.float8_e4m3fn).view(torch.uint8).permute(0, 2, 3, 1)
     assert torch.equal(codes.cpu().view(torch.uint8)[..., :Lk], want)
     np.testing.assert_array_equal(sv.cpu().numpy(), s_ref[:, 0])
+
+
+@pytest.mark.parametrize("B,Lq,Lk,Hq,Hkv,mask,off", [
+    (1, 300, 700, 4, 2, 0, 0),
+    (2, 257, 900, 2, 1, 1, 643),
+    (1, 256, 1000, 2, 2, 2, 300),
+])
+def test_fp8_head_dim_256(B, Lq, Lk, Hq, Hkv, mask, off):
+    """d = 256 through the one-tile e4m3 kernel (two 128-byte chunks per row,
+    P of each S buffer in shared memory)."""
+    _fp8_case(B, Lq, Lk, Hq, Hkv, mask, off, seed=80 + Lq, d=256)
+
+
+def test_fp8_scaled_head_dim_256_is_unsupported():
+    q, k, v = inputs.make_qkv(1, 64, 64, 1, 1, 256, torch.bfloat16, seed=1)
+    q8, sq = hasb.fp8_quantize_tokens(q.cuda())
+    k8, sk = hasb.fp8_quantize_tokens(k.cuda())
+    vt8, sv = hasb.fp8_quantize_vt(v.cuda())
+    with pytest.raises(hasb.AttnError) as e:
+        hasb.attn_fwd_fp8_scaled(q8, sq, k8, sk, vt8, sv)
+    assert e.value.status == hasb.ATTN_ERR_UNSUPPORTED
