@@ -561,8 +561,8 @@ def run_fp8(args):
     ranks = Ranks("nccl")
     rank, world = ranks.rank, ranks.world
     w = select_workload(args)
-    if w.dtype != "bf16" or (args.scaled and w.d > 128):
-        raise SystemExit("--op fp8 runs bf16 workloads (per-token scales: head_dim <= 128)")
+    if w.dtype != "bf16":
+        raise SystemExit("--op fp8 runs bf16 workloads")
     q_cpu, k_cpu, v_cpu = inputs.make_qkv(w.B, w.Lq, w.Lk, w.Hq, w.Hkv, w.d, w.torch_dtype,
                                           seed=rank_seed(w.seed, rank), qk_rmsnorm=w.qk_rmsnorm)
     q, k, v = q_cpu.cuda(), k_cpu.cuda(), v_cpu.cuda()

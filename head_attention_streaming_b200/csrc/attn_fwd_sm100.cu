@@ -158,6 +158,14 @@ struct Cfg<256, 1> {
   static __device__ __forceinline__ uint32_t col_o(int) { return 256u; }
   static constexpr uint32_t kTmemCols = 512;
 };
+// per-token scales at d = 256: the key scales of the current tile, one
+// 512-byte copy per softmax warp
+template <>
+struct Cfg<256, 2> : Cfg<256, 1> {
+  static constexpr int kOffSk = Cfg<256, 1>::kOffBar;
+  static constexpr int kOffBar = kOffSk + 4 * 512;
+  static constexpr int kSmemBytes = kOffBar + 512 + 1024;
+};
 template <>
 struct Cfg<128, 2> : CfgE4m3<2> {};
 
@@ -1193,9 +1201,10 @@ __device__ __forceinline__ void mma_role_single(const FwdParams& p, uint32_t tme
 // a unit: wait for the last P V, O / l to 16 bits straight to global memory.
 template <bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW, int F8>
 __device__ __forceinline__ void softmax_role_single(const FwdParams& p, uint32_t tmem, uint32_t bars,
-                                                    uint32_t sP, volatile int* abort_flag) {
+                                                    uint32_t sP, uint32_t sSk, volatile int* abort_flag) {
   using C = Cfg<256, F8>;
   constexpr int D = 256;
+  const uint32_t skw = sSk + (threadIdx.x / 32) * 512;  // per-token scales: this warp's key scales
   const int warp = threadIdx.x / 32;
   const int r_in = threadIdx.x % kTileRows;
   const int lane = threadIdx.x % 32;
@@ -1219,7 +1228,22 @@ __device__ __forceinline__ void softmax_role_single(const FwdParams& p, uint32_t
     }
     float ref = -INFINITY;
     float l = 0.f;
+    float sl2r = sl2;  // per-token scales: times the row's Q scale
+    const float* skrow = nullptr;
+    float4 skv = make_float4(0.f, 0.f, 0.f, 0.f);
+    if constexpr (F8 == 2) {
+      const size_t qs = (static_cast<size_t>(x.b) * p.Hq + x.hq) * p.sq_pitch + row;
+      sl2r = sl2 * (row < p.Lq ? __ldg(p.sq + qs) : 1.f);
+      skrow = p.sk + (static_cast<size_t>(x.b) * p.Hkv + x.hkv) * p.sk_pitch;
+      skv = load_key_scales(skrow, x.j0 * kTileRows + 4 * lane, p.Lk);
+    }
     for (int j = 0; j < n; ++j) {
+      if constexpr (F8 == 2) {
+        __syncwarp();  // every lane is done with the previous tile's scales
+        st_shared_v4f(skw + 16 * lane, skv);
+        __syncwarp();
+        if (j + 1 < n) skv = load_key_scales(skrow, (x.j0 + j + 1) * kTileRows + 4 * lane, p.Lk);
+      }
       const int buf = sc & 1;
       const uint32_t tS = tmem + lane_bits + C::col_s(buf);
       bool ok = mbar_wait(bars + 8 * (kBarSFull + buf), (sc >> 1) & 1, abort_flag, kFaultSoftmaxSFull,
@@ -1231,6 +1255,19 @@ __device__ __forceinline__ void softmax_role_single(const FwdParams& p, uint32_t
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(tS + 32 * c, r + 32 * c);
       tmem_wait_ld_x128(r);
+      if constexpr (F8 == 2) {
+#pragma unroll
+        for (int c = 0; c < 128; c += 4) {
+          const float4 k4 = ld_shared_v4f(skw + 4 * c);
+          float a0, a1, a2, a3;
+          f2_unpack(f2_mul(f2_pack_bits(r[c], r[c + 1]), f2_pack(k4.x, k4.y)), a0, a1);
+          f2_unpack(f2_mul(f2_pack_bits(r[c + 2], r[c + 3]), f2_pack(k4.z, k4.w)), a2, a3);
+          r[c] = __float_as_uint(a0);
+          r[c + 1] = __float_as_uint(a1);
+          r[c + 2] = __float_as_uint(a2);
+          r[c + 3] = __float_as_uint(a3);
+        }
+      }
       const int key0 = (x.j0 + j) * kTileRows;
       const int lim = row_lim - key0;
       const int lim_lo = WINDOW ? row_lo - key0 : 0;
@@ -1256,7 +1293,7 @@ __device__ __forceinline__ void softmax_role_single(const FwdParams& p, uint32_t
         for (int i = 0; i < 5; ++i) c5[i] = fmax3(b[3 * i], b[3 * i + 1], b[3 * i + 2]);
         m_tile = fmaxf(fmax3(c5[0], c5[1], c5[2]), fmaxf(c5[3], c5[4]));
       }
-      const float m_scaled = (m_tile == -INFINITY) ? -INFINITY : m_tile * sl2;
+      const float m_scaled = (m_tile == -INFINITY) ? -INFINITY : m_tile * sl2r;
       if (j > 0) {
         // P_{j-1} V_{j-1} done: O may be rescaled
         ok = mbar_wait(bar_o, ocnt & 1, abort_flag, kFaultSoftmaxOFull, p.timeout_ns);
@@ -1289,9 +1326,9 @@ __device__ __forceinline__ void softmax_role_single(const FwdParams& p, uint32_t
       if constexpr (F8 != 0) {
         const uint32_t prow = sP + buf * kTileRows * 128 + r_in * 128;  // e4m3 P row of this S buffer
         if (__any_sync(0xffffffffu, partial))
-          exp_tile_f8<true>(r, sl2, -ref, lim, lim_lo, sum, prow, r_in, bar_ph, bar_p, 0u, false, lane);
+          exp_tile_f8<true>(r, sl2r, -ref, lim, lim_lo, sum, prow, r_in, bar_ph, bar_p, 0u, false, lane);
         else
-          exp_tile_f8<false>(r, sl2, -ref, lim, lim_lo, sum, prow, r_in, bar_ph, bar_p, 0u, false, lane);
+          exp_tile_f8<false>(r, sl2r, -ref, lim, lim_lo, sum, prow, r_in, bar_ph, bar_p, 0u, false, lane);
       } else if (__any_sync(0xffffffffu, partial)) {
         exp_tile<BF16, true>(r, sl2, -ref, lim, lim_lo, sum, tS, bar_ph, bar_p, 0u, false, lane);
       } else {
@@ -1349,6 +1386,20 @@ __device__ __forceinline__ void softmax_role_single(const FwdParams& p, uint32_t
       tmem_ld_32x32b_x32(tO + 32 * c, ov);
       tmem_wait_ld_x32(ov);
       if (in_range) {
+        if constexpr (F8 == 2) {
+          if (p.sv != nullptr) {  // V's per-channel scales
+            const float4* sv4 = reinterpret_cast<const float4*>(
+                p.sv + (static_cast<size_t>(x.b) * p.Hkv + x.hkv) * D + 32 * c);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float4 f = __ldg(sv4 + e);
+              ov[4 * e] = __float_as_uint(__uint_as_float(ov[4 * e]) * f.x);
+              ov[4 * e + 1] = __float_as_uint(__uint_as_float(ov[4 * e + 1]) * f.y);
+              ov[4 * e + 2] = __float_as_uint(__uint_as_float(ov[4 * e + 2]) * f.z);
+              ov[4 * e + 3] = __float_as_uint(__uint_as_float(ov[4 * e + 3]) * f.w);
+            }
+          }
+        }
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e)
@@ -1435,7 +1486,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // one query tile: warps 0-3 softmax, warp 8 loads, warp 9 issues the MMAs
     if (warp < 8) {
       regs_increase<kRegsSoftmax>();
-      if (warp < 4) softmax_role_single<BF16, CAUSAL, SPLIT, WINDOW, F8>(p, tmem, bars, sP, abort_flag);
+      if (warp < 4)
+        softmax_role_single<BF16, CAUSAL, SPLIT, WINDOW, F8>(p, tmem, bars, sP, sbase + C::kOffSk, abort_flag);
     } else {
       regs_decrease<kRegsProducer>();
       if (warp == 8 && lane == 0)
@@ -2146,7 +2198,6 @@ int fp8_fwd(const void* q8, const void* k8, const void* vt8, const float* sq, co
       return ATTN_ERR_INVALID_ARG;
   }
   // d < 128 runs the 128-wide kernel on zero-filled columns; 256 the one-tile kernel (unscaled only)
-  if (d == 256 && scaled) return ATTN_ERR_UNSUPPORTED;
   // ---- device
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
@@ -2177,6 +2228,9 @@ int fp8_fwd(const void* q8, const void* k8, const void* vt8, const float* sq, co
   const int grid = static_cast<int>(n_units < di.num_sms ? n_units : di.num_sms);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool c = causal == ATTN_MASK_CAUSAL;
+  if (d == 256 && scaled)
+    return c ? launch_fwd<256, true, true, false, false, 2>(p, q8, k8, vt8, vt_pitch, grid, s)
+             : launch_fwd<256, true, false, false, false, 2>(p, q8, k8, vt8, vt_pitch, grid, s);
   if (d == 256)
     return c ? launch_fwd<256, true, true, false, false, 1>(p, q8, k8, vt8, vt_pitch, grid, s)
              : launch_fwd<256, true, false, false, false, 1>(p, q8, k8, vt8, vt_pitch, grid, s);

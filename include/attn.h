@@ -151,8 +151,8 @@ int attn_fwd_fp8(const void* q8, const void* k8, const void* vt8, void* o, float
  * [B, Hq, sq_pitch], sk [B, Hkv, sk_pitch] as attn_fp8_quantize_tokens writes
  * them, sk_pitch a multiple of 4, sk 16-byte aligned), and column c of O is
  * multiplied by sv[b, hkv, c] ([B, Hkv, d], 16-byte aligned; NULL: V cast
- * without scales). P is rounded to e4m3 as in attn_fwd_fp8. d <= 128 (256:
- * ATTN_ERR_UNSUPPORTED).
+ * without scales). P is rounded to e4m3 as in attn_fwd_fp8. Head dims as
+ * attn_fwd_fp8.
  */
 int attn_fp8_quantize_tokens(const void* x, void* y, float* s, int B, int L, int H, int d, int s_pitch,
                              int dtype, void* stream);

@@ -253,11 +253,6 @@ def test_fp8_head_dim_256(B, Lq, Lk, Hq, Hkv, mask, off):
     _fp8_case(B, Lq, Lk, Hq, Hkv, mask, off, seed=80 + Lq, d=256)
 
 
-def test_fp8_scaled_head_dim_256_is_unsupported():
-    q, k, v = inputs.make_qkv(1, 64, 64, 1, 1, 256, torch.bfloat16, seed=1)
-    q8, sq = hasb.fp8_quantize_tokens(q.cuda())
-    k8, sk = hasb.fp8_quantize_tokens(k.cuda())
-    vt8, sv = hasb.fp8_quantize_vt(v.cuda())
-    with pytest.raises(hasb.AttnError) as e:
-        hasb.attn_fwd_fp8_scaled(q8, sq, k8, sk, vt8, sv)
-    assert e.value.status == hasb.ATTN_ERR_UNSUPPORTED
+@pytest.mark.parametrize("mask,off", [(0, 0), (1, 400)])
+def test_fp8_scaled_head_dim_256(mask, off):
+    _fp8_scaled_case(1, 300, 700, 4, 2, mask, off, seed=85 + mask, d=256)
