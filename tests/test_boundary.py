@@ -237,8 +237,8 @@ def test_fp8_scaled_attention_argument_contract(kw):
     assert hasb.lib().attn_fwd_fp8_scaled(*_fp8s_args(**kw)) == hasb.ATTN_ERR_INVALID_ARG
 
 
-def test_fp8_scaled_attention_head_dim_256_is_unsupported():
-    assert hasb.lib().attn_fwd_fp8_scaled(*_fp8s_args(d=256)) == hasb.ATTN_ERR_UNSUPPORTED
+def test_fp8_scaled_attention_head_dim_512_is_invalid():
+    assert hasb.lib().attn_fwd_fp8_scaled(*_fp8s_args(d=512)) == hasb.ATTN_ERR_INVALID_ARG
 
 
 def test_fp8_quantize_argument_contract():
