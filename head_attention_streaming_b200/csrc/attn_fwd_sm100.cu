@@ -20,7 +20,9 @@
 //   warp  11    O store: staged O tiles to global memory by TMA
 // A work unit is (batch, query head, 256-row pair of query tiles). Tensor
 // memory holds S_0, S_1 (128 fp32 columns each, P aliased as packed 16-bit in
-// the first 64 columns) and O_0, O_1 (d columns each).
+// the first 64 columns) and O_0, O_1 (d columns each). At d = 256 a unit is
+// one query tile: warps 0-3 run its softmax, warp 9 issues Q K^T into two
+// alternating S buffers, warp 10 issues P V, and the softmax stores O.
 
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -54,6 +56,7 @@ enum FaultBit : unsigned int {
   kFaultSoftmaxTurn = 1u << 7,
   kFaultStore = 1u << 9,
   kFaultSelftest = 1u << 8,
+  kFaultMmaSFree = 1u << 10,
 };
 
 constexpr int kThreads = 384;
@@ -183,6 +186,7 @@ enum Bar : int {
   kBarKvEmpty = 24, // [kStages] both MMA issuers -> TMA
   kBarStgFull = 32, //     softmax t -> store warp: O tile t staged (one arrival per warp)
   kBarStgFree = 34, // [2] store warp -> softmax t: staging buffer is t's to fill
+  kBarSFree = 36,   // [2] d = 256, P V issuer -> Q K^T issuer: the P V that read S buffer b is done
 };
 
 // Exponentials of the softmax: kPolyPairsPer8 of every 8 score pairs take
@@ -1108,14 +1112,21 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
 }
 
 // ----------------------------------------------------------------- d = 256
-// One query tile per unit and one MMA issuer: S alternates between two tensor
-// memory buffers over the KV tiles, so Q K_{j+1}^T runs on the tensor core
-// while the softmax works on tile j; O += P_j V_j follows once P_j is in. The
-// issuer commits kBarOFull after every P V, so the softmax knows when O may be
-// rescaled (and, after the last, read out).
+// The MMAs of the one query tile at d = 256, split over two issuing threads:
+// role 0 runs S_j = Q K_j^T into S buffer j % 2, role 1 runs O += P_j V_j. One
+// thread issuing both (Q K_{j+1}^T, then P_j V_j) measured 0.79x the speed
+// of the split on 8192 x 8192 x 16 heads: the issuing thread is held while its
+// MMAs are queued, so the next tile's Q K^T reached the tensor pipe late.
+// Hand-offs: S_full[b] (role 0 -> softmax), P_half / P_full (softmax -> role
+// 1), O_full after every P V (role 1 -> softmax: O may be rescaled or read
+// out), S_free[b] after every P V (role 1 -> role 0: P_j's buffer may take
+// S_{j+2}). S_free has one barrier per buffer, so the completion role 0 waits
+// for is the latest one that can have happened (P V_{j+2} needs S_{j+2}
+// first) and a parity wait cannot be a phase behind. Each K/V ring slot is
+// released by its one reader.
 template <bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW, int F8>
-__device__ __forceinline__ void mma_role_single(const FwdParams& p, uint32_t tmem, uint32_t sQ,
-                                                uint32_t sKV, uint32_t sP, uint32_t bars,
+__device__ __forceinline__ void mma_role_single(const int role, const FwdParams& p, uint32_t tmem,
+                                                uint32_t sQ, uint32_t sKV, uint32_t sP, uint32_t bars,
                                                 volatile int* abort_flag) {
   using C = Cfg<256, F8>;
   // e4m3: P of S buffer b in shared memory (K-major, 128-byte swizzle)
@@ -1131,67 +1142,72 @@ __device__ __forceinline__ void mma_role_single(const FwdParams& p, uint32_t tme
                      kFaultMmaKvFull, p.timeout_ns);
   };
   const uint32_t o_t = tmem + C::col_o(0);
-  int kv_it = 0, uit = 0, pcnt = 0, sc = 0;
+  int kv_it = 0, uit = 0, pcnt = 0;
+  int sc = 0;  // KV tiles issued so far by this thread, over all units: tile sc uses S buffer sc % 2
   bool ok = true;
   for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++uit) {
     const Unit x = decode_single<CAUSAL, SPLIT, WINDOW>(p, u);
     const int n = x.n0;
-    if (SPLIT && n == 0) {
-      // (causal key split) no key of this range is visible: release Q; O is
-      // neither written nor signalled, the softmax writes the empty partial
+    if (role == 0) {
       ok = mbar_wait(bar(kBarQFull), uit & 1, abort_flag, kFaultMmaQFull, p.timeout_ns);
       if (!ok) break;
-      mma_commit(bar(kBarQEmpty));
-      continue;
-    }
-    ok = mbar_wait(bar(kBarQFull), uit & 1, abort_flag, kFaultMmaQFull, p.timeout_ns) && kv_full(kv_it);
-    if (!ok) break;
-    // S(0) = Q K_0^T
-    if constexpr (F8 != 0) issue_qk_f8<256>(tmem + C::col_s(sc & 1), q_lo, k_lo(kv_it));
-    else issue_qk<256, BF16>(tmem + C::col_s(sc & 1), q_lo, k_lo(kv_it));
-    mma_commit(bar(kBarSFull + (sc & 1)));
-    mma_commit(bar(kBarKvEmpty + kv_it % C::kStages));
-    if (n == 1) mma_commit(bar(kBarQEmpty));
-    ++sc;
-    for (int j = 0; j < n; ++j) {
-      const int vidx = kv_it + 2 * j + 1;
-      const uint32_t s_j = tmem + C::col_s((sc - 1) & 1);  // tile j's S / P buffer
-      if (j + 1 < n) {
-        // S(j+1) into the other buffer: its last P was read by a P V issued earlier
-        const int knext = vidx + 1;
-        if (!kv_full(knext)) { ok = false; break; }
-        if constexpr (F8 != 0) issue_qk_f8<256>(tmem + C::col_s(sc & 1), q_lo, k_lo(knext));
-        else issue_qk<256, BF16>(tmem + C::col_s(sc & 1), q_lo, k_lo(knext));
-        mma_commit(bar(kBarSFull + (sc & 1)));
-        mma_commit(bar(kBarKvEmpty + knext % C::kStages));
-        if (j + 1 == n - 1) mma_commit(bar(kBarQEmpty));
+      if (SPLIT && n == 0) {
+        // (causal key split) no key of this range is visible: release Q; O is
+        // neither written nor signalled, the softmax writes the empty partial
+        mma_commit(bar(kBarQEmpty));
       }
-      // O += P_j V_j in two halves of 64 keys
-      if (!kv_full(vidx) ||
-          !mbar_wait(bar(kBarPHalf), pcnt & 1, abort_flag, kFaultMmaPFull, p.timeout_ns)) {
-        ok = false;
-        break;
+      for (int j = 0; j < n; ++j) {
+        const int b = sc & 1;
+        if (sc >= 2) {
+          // P V of the tile two back (this unit's or an earlier one's) is done with buffer b
+          ok = mbar_wait(bar(kBarSFree + b), ((sc >> 1) - 1) & 1, abort_flag, kFaultMmaSFree,
+                         p.timeout_ns);
+          if (!ok) break;
+          tc_fence_after_sync();
+        }
+        const int kidx = kv_it + 2 * j;  // K_j
+        if (!kv_full(kidx)) { ok = false; break; }
+        if constexpr (F8 != 0) issue_qk_f8<256>(tmem + C::col_s(b), q_lo, k_lo(kidx));
+        else issue_qk<256, BF16>(tmem + C::col_s(b), q_lo, k_lo(kidx));
+        mma_commit(bar(kBarSFull + b));
+        mma_commit(bar(kBarKvEmpty + kidx % C::kStages));
+        if (j == n - 1) mma_commit(bar(kBarQEmpty));
+        ++sc;
       }
-      tc_fence_after_sync();
-      if constexpr (F8 != 0) issue_pv_half_f8<256, 0>(o_t, p_lo((sc - 1) & 1), k_lo(vidx), j > 0 ? 1u : 0u);
-      else issue_pv_half<256, BF16, 0>(o_t, s_j, v_lo(vidx), j > 0 ? 1u : 0u);
-      if (!mbar_wait(bar(kBarPFull), pcnt & 1, abort_flag, kFaultMmaPFull, p.timeout_ns)) {
-        ok = false;
-        break;
+    } else {
+      for (int j = 0; j < n; ++j) {
+        const int b = sc & 1;
+        const int vidx = kv_it + 2 * j + 1;  // V_j
+        const uint32_t s_j = tmem + C::col_s(b);
+        // O += P_j V_j in two halves of 64 keys
+        if (!kv_full(vidx) ||
+            !mbar_wait(bar(kBarPHalf), pcnt & 1, abort_flag, kFaultMmaPFull, p.timeout_ns)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after_sync();
+        if constexpr (F8 != 0) issue_pv_half_f8<256, 0>(o_t, p_lo(b), k_lo(vidx), j > 0 ? 1u : 0u);
+        else issue_pv_half<256, BF16, 0>(o_t, s_j, v_lo(vidx), j > 0 ? 1u : 0u);
+        if (!mbar_wait(bar(kBarPFull), pcnt & 1, abort_flag, kFaultMmaPFull, p.timeout_ns)) {
+          ok = false;
+          break;
+        }
+        ++pcnt;
+        tc_fence_after_sync();
+        if constexpr (F8 != 0) issue_pv_half_f8<256, 1>(o_t, p_lo(b), k_lo(vidx), 1u);
+        else issue_pv_half<256, BF16, 1>(o_t, s_j, v_lo(vidx), 1u);
+        mma_commit(bar(kBarKvEmpty + vidx % C::kStages));
+        mma_commit(bar(kBarOFull));
+        mma_commit(bar(kBarSFree + b));
+        ++sc;
       }
-      ++pcnt;
-      tc_fence_after_sync();
-      if constexpr (F8 != 0) issue_pv_half_f8<256, 1>(o_t, p_lo((sc - 1) & 1), k_lo(vidx), 1u);
-      else issue_pv_half<256, BF16, 1>(o_t, s_j, v_lo(vidx), 1u);
-      mma_commit(bar(kBarKvEmpty + vidx % C::kStages));
-      mma_commit(bar(kBarOFull));
-      if (j + 1 < n) ++sc;
     }
     kv_it += 2 * x.nu;
   }
   if (!ok) {
-    mma_commit(bar(kBarDrain));
-    mbar_drain(bar(kBarDrain), 0);
+    // every MMA this thread issued must finish before tensor memory is freed
+    mma_commit(bar(kBarDrain + role));
+    mbar_drain(bar(kBarDrain + role), 0);
   }
 }
 
@@ -1453,9 +1469,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bars + 8 * (kBarStgFree + 0), 1);
     mbar_init(bars + 8 * (kBarStgFree + 1), 1);
     mbar_init(bars + 8 * (kBarDrain + 1), 1);
+    mbar_init(bars + 8 * (kBarSFree + 0), 1);
+    mbar_init(bars + 8 * (kBarSFree + 1), 1);
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(bars + 8 * (kBarKvFull + s), 1);
-      mbar_init(bars + 8 * (kBarKvEmpty + s), D == 256 ? 1 : 2);  // one MMA issuer at d = 256
+      // d = 256: a K tile is read by the Q K^T issuer only, a V tile by the P V issuer only
+      mbar_init(bars + 8 * (kBarKvEmpty + s), D == 256 ? 1 : 2);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -1483,7 +1502,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   griddep_launch_dependents();
 
   if constexpr (D == 256) {
-    // one query tile: warps 0-3 softmax, warp 8 loads, warp 9 issues the MMAs
+    // one query tile: warps 0-3 softmax, warp 8 loads, warp 9 issues Q K^T,
+    // warp 10 issues P V
     if (warp < 8) {
       regs_increase<kRegsSoftmax>();
       if (warp < 4)
@@ -1492,8 +1512,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       regs_decrease<kRegsProducer>();
       if (warp == 8 && lane == 0)
         load_role<D, BF16, CAUSAL, SPLIT, WINDOW, F8>(&tm_q, &tm_k, &tm_v, p, sQ, sKV, bars, abort_flag);
-      else if (warp == 9 && lane == 0)
-        mma_role_single<BF16, CAUSAL, SPLIT, WINDOW, F8>(p, tmem, sQ, sKV, sP, bars, abort_flag);
+      else if ((warp == 9 || warp == 10) && lane == 0)
+        mma_role_single<BF16, CAUSAL, SPLIT, WINDOW, F8>(warp - 9, p, tmem, sQ, sKV, sP, bars, abort_flag);
     }
   } else if (warp < 8) {
     regs_increase<kRegsSoftmax>();
