@@ -23,7 +23,7 @@ Also reported on the same JSON line:
                 of the same workload (rank 0, N = 1);
   clocks        SM clock samples taken by nvidia-smi during the timed region.
 
---impl reference times the FP64 CPU oracle (the only reference this build has)
+--impl reference times the FP64 CPU oracle (the method has no other reference code)
 on the same workload, metric and unit, each step a bounded sample of it.
 
 --op stream times one steady-state streaming self-attention step through the

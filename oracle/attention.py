@@ -25,7 +25,7 @@ developer guide's definition shapes them ([B, L, H, d] for Q, [B, S, H, d] for
 K and V) and as the FlashAttention-4 runtime page ("FLASH4.md", the H3 call
 layout) and the skill page ("Workflow 2", Step 2) use them.
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
 
 * Head mapping with fewer K/V heads (skill page, "Workflow 2", Step 3,
   multi-query attention; accelerated user guide, "Shared policy", separate

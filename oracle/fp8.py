@@ -19,7 +19,7 @@ pages' SageAttention remark): Q and K are quantized with one scale per token
 and head, V with one scale per channel and head (``quantize_attention_inputs``),
 and the oracle is the exact attention of the dequantized values.
 
-Readings (listed in DESIGN.md):
+Readings where the pages are silent:
 
 * The cast rounds to nearest even and saturates at +-448 (the largest finite
   e4m3 value; the type has no infinities).

@@ -21,7 +21,7 @@ flashdreams.accelerated developer guide, "Optimized Multi Head Attention" ->
   ``(r, r + d/2)``. The page applies normalisation first, then RoPE ("the
   reference below normalizes before applying RoPE").
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
 
 * The angles arrive "expanded" as ``rope_freqs`` shaped ``[L, 1, 1, d]``, one
   angle per feature; pair ``r`` uses the angle stored at its first feature

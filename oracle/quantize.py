@@ -23,7 +23,7 @@ scale floor eps:
 The pages compute the scales in float32; so does this oracle, including the
 division by the scale, because those roundings decide the integer or FP8 code.
 
-Readings (listed in DESIGN.md):
+Readings where the pages are silent:
 
 * eps is not given; it only matters for a slice whose max |X| / M_t falls
   below it (an all-zero row, say). It is taken as 2^-126, the smallest normal

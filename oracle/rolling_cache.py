@@ -15,7 +15,7 @@ caller runs ``before_update(chunk_idx)``, the attention call, then
 rolling cache before the chunk is queried; cached keys are evicted as the
 stream advances ("test both cache fill and post-eviction steady state").
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
 
 * Sizes are whole chunks: ``sink_size`` and ``window_size`` are multiples of
   the chunk length ``C``.
@@ -76,7 +76,7 @@ def stream_attention_after_rope(q_chunks, k_all, v_all, chunk: int, sink: int, w
     after-cache RoPE the angle table covers the query and every visible cache
     position; cached keys take cache-relative frequencies).
 
-    Reading (listed in the design doc): a visible key's current position is its
+    Reading where the pages are silent: a visible key's current position is its
     index in the visible set in stream order (sinks first, then the window
     oldest first, the current chunk last); the chunk's queries take the
     positions of the chunk's own keys, the last ``chunk`` of them.
