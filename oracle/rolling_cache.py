@@ -88,6 +88,19 @@ def stream_attention_after_rope(q_chunks, k_all, v_all, chunk: int, sink: int, w
     (a path that stores them in a 16-bit type rounds there; the default keeps
     them exact). Returns a list of (o, lse) as ``stream_attention``.
     """
+    out = []
+    for qr, k, v in after_rope_inputs(q_chunks, k_all, v_all, chunk, sink, window, angles, style,
+                                      round_rotated):
+        out.append(attention_fwd(qr, k, v, scale, MASK_NONE, 0))
+    return out
+
+
+def after_rope_inputs(q_chunks, k_all, v_all, chunk: int, sink: int, window: int, angles, style: int,
+                      round_rotated=None):
+    """Per chunk, the (queries, keys, values) that ``stream_attention_after_rope``
+    attends with: the chunk's queries and every visible key rotated at their
+    current (cache-relative) positions, optionally rounded, and the visible
+    values. Same readings and arguments as that function."""
     from .prologue import rope
     out = []
     ang = np.asarray(angles, dtype=np.float64)
@@ -98,5 +111,5 @@ def stream_attention_after_rope(q_chunks, k_all, v_all, chunk: int, sink: int, w
         qr = rope(np.asarray(q), ang[R - chunk:R], style)
         if round_rotated is not None:
             k, qr = round_rotated(k), round_rotated(qr)
-        out.append(attention_fwd(qr, k, np.asarray(v_all)[:, idx], scale, MASK_NONE, 0))
+        out.append((qr, k, np.asarray(v_all)[:, idx]))
     return out

@@ -21,7 +21,7 @@ import oracle
 from head_attention_streaming_b200.inputs import rope_angle_table
 from oracle import prologue as qp
 from oracle import rolling_cache as rc
-from test_parity_gpu import _check
+from test_parity_gpu import _check, _pbound
 
 pytestmark = pytest.mark.gpu
 
@@ -74,7 +74,8 @@ def _stream(B, C, sink, window, Hq, Hkv, d, n_chunks, dtype, norm, style, seed, 
         o_cpu, lse_cpu = o.cpu(), lse.cpu()
         if rows is not None:
             o_cpu, lse_cpu = o_cpu[:, rows], lse_cpu[:, :, rows]
-        _check(o_cpu, lse_cpu, o_ref, lse_ref, tag, what=f"chunk {c}", output_ulp=sample_rows is None)
+        pb = _pbound(qn, kn[:, idx], vn[:, idx], scale, tag) if sample_rows is None else None
+        _check(o_cpu, lse_cpu, o_ref, lse_ref, tag, what=f"chunk {c}", p_bound=pb)
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
@@ -124,9 +125,12 @@ def test_after_cache_rope_stream(style, sink, window, n_chunks, dtype):
     f64 = lambda t: t.to(torch.float64).numpy()
     qn = _round16(qp.rms_norm(f64(q), f64(gq), eps, qp.NORM_HEAD), dtype)
     kn = _round16(qp.rms_norm(f64(k), f64(gk), eps, qp.NORM_HEAD), dtype)
-    ref = rc.stream_attention_after_rope([qn[:, c * C:(c + 1) * C] for c in range(n_chunks)], kn, f64(v),
-                                         C, sink, window, scale, f64(ang), style,
-                                         round_rotated=lambda x: _round16(x, dtype))
+    q_chunks = [qn[:, c * C:(c + 1) * C] for c in range(n_chunks)]
+    r16 = lambda x: _round16(x, dtype)
+    ref = rc.stream_attention_after_rope(q_chunks, kn, f64(v), C, sink, window, scale, f64(ang), style,
+                                         round_rotated=r16)
+    rotated = rc.after_rope_inputs(q_chunks, kn, f64(v), C, sink, window, f64(ang), style,
+                                   round_rotated=r16)
     cache = hasb.BlockKVCache(B, Hkv, d, C, window, sink, dtype=dtype)
     tag = "bf16" if dtype == torch.bfloat16 else "fp16"
     for c in range(n_chunks):
@@ -138,7 +142,8 @@ def test_after_cache_rope_stream(style, sink, window, n_chunks, dtype):
                               rope_after_cache=True, angles_cache=ang.cuda())
         torch.cuda.synchronize()
         cache.after_update(c)
-        _check(o.cpu(), lse.cpu(), *ref[c], tag, what=f"after-cache chunk {c}", output_ulp=True)
+        _check(o.cpu(), lse.cpu(), *ref[c], tag, what=f"after-cache chunk {c}",
+               p_bound=_pbound(*rotated[c], scale, tag))
     # the cache itself keeps the normalised, unrotated keys of the visible chunks
     stored = cache.k.cpu().to(torch.float64).numpy()
     last = n_chunks - 1

@@ -13,7 +13,7 @@ import torch
 import head_attention_streaming_b200 as hasb
 import oracle
 from head_attention_streaming_b200 import inputs
-from test_parity_gpu import _check
+from test_parity_gpu import _check, _pbound
 
 pytestmark = pytest.mark.gpu
 
@@ -45,8 +45,9 @@ def test_small_head_dims(d, B, Lq, Lk, Hq, Hkv, dtype, mask, off):
     o, lse = hasb.attn_fwd(q.cuda(), k.cuda(), v.cuda(), scale=scale, causal=mask, kv_offset=off)
     torch.cuda.synchronize()
     o_ref, lse_ref = oracle.attention_fwd(f64(q), f64(k), f64(v), scale, mask, off)
-    _check(o.cpu(), lse.cpu(), o_ref, lse_ref, "bf16" if dtype == torch.bfloat16 else "fp16",
-           what=f"d={d}", output_ulp=True)
+    tag = "bf16" if dtype == torch.bfloat16 else "fp16"
+    _check(o.cpu(), lse.cpu(), o_ref, lse_ref, tag, what=f"d={d}",
+           p_bound=_pbound(q, k, v, scale, tag, mask, off))
 
 
 @pytest.mark.parametrize("d", [16, 32])
@@ -71,12 +72,13 @@ def test_small_head_dims_window_split_and_cache(d):
     o, lse = hasb.attn_fwd_window(qc, kc, vc, window=(100, 20), scale=scale, kv_offset=500)
     torch.cuda.synchronize()
     ref = oracle.attention_fwd(f64(q), f64(k), f64(v), scale, oracle.MASK_WINDOW, 500, window=(100, 20))
-    _check(o.cpu(), lse.cpu(), *ref, "bf16", what=f"window d={d}", output_ulp=True)
+    _check(o.cpu(), lse.cpu(), *ref, "bf16", what=f"window d={d}",
+           p_bound=_pbound(q, k, v, scale, "bf16", oracle.MASK_WINDOW, 500, window=(100, 20)))
     o, lse, used = hasb.attn_fwd_splitkv(qc, kc, vc, n_splits=3, scale=scale)
     torch.cuda.synchronize()
     assert used == 3
     ref = oracle.attention_fwd(f64(q), f64(k), f64(v), scale, 0, 0)
-    _check(o.cpu(), lse.cpu(), *ref, "bf16", what=f"split d={d}", output_ulp=True)
+    _check(o.cpu(), lse.cpu(), *ref, "bf16", what=f"split d={d}", p_bound=_pbound(q, k, v, scale, "bf16"))
     # a cache of 1200 slots of which the first 900 are valid
     S = 1200
     kcache = torch.zeros(1, S, 2, d, dtype=torch.bfloat16, device="cuda")
@@ -86,7 +88,7 @@ def test_small_head_dims_window_split_and_cache(d):
     o, lse = hasb.attn_fwd_cache(qc, kcache, vcache, 900, scale=scale, causal=hasb.MASK_CHUNK, kv_offset=600)
     torch.cuda.synchronize()
     ref = oracle.attention_fwd(f64(q), f64(k), f64(v), scale, 2, 600)
-    _check(o.cpu(), lse.cpu(), *ref, "bf16", what=f"cache d={d}", output_ulp=True)
+    _check(o.cpu(), lse.cpu(), *ref, "bf16", what=f"cache d={d}", p_bound=_pbound(q, k, v, scale, "bf16", 2, 600))
 
 
 # ---------------------------------------------------------------- d = 256
@@ -106,8 +108,8 @@ def test_d256(B, Lq, Lk, Hq, Hkv, dtype, mask, off):
     o, lse = hasb.attn_fwd(q.cuda(), k.cuda(), v.cuda(), scale=scale, causal=mask, kv_offset=off)
     torch.cuda.synchronize()
     o_ref, lse_ref = oracle.attention_fwd(f64(q), f64(k), f64(v), scale, mask, off)
-    _check(o.cpu(), lse.cpu(), o_ref, lse_ref, "bf16" if dtype == torch.bfloat16 else "fp16",
-           what="d=256", output_ulp=True)
+    tag = "bf16" if dtype == torch.bfloat16 else "fp16"
+    _check(o.cpu(), lse.cpu(), o_ref, lse_ref, tag, what="d=256", p_bound=_pbound(q, k, v, scale, tag, mask, off))
 
 
 def test_d256_large_scores_rescale_and_cache_prefix():
@@ -125,7 +127,8 @@ def test_d256_large_scores_rescale_and_cache_prefix():
     o, lse = hasb.attn_fwd_cache(q.cuda(), kc, vc, 900, scale=scale, causal=hasb.MASK_CHUNK, kv_offset=644)
     torch.cuda.synchronize()
     o_ref, lse_ref = oracle.attention_fwd(f64(q), f64(k), f64(v), scale, 2, 644)
-    _check(o.cpu(), lse.cpu(), o_ref, lse_ref, "bf16", what="d=256 cache", output_ulp=True)
+    _check(o.cpu(), lse.cpu(), o_ref, lse_ref, "bf16", what="d=256 cache",
+           p_bound=_pbound(q, k, v, scale, "bf16", 2, 644))
 
 
 def test_d256_deterministic():
@@ -143,7 +146,8 @@ def test_d256_window(window, off):
     o, lse = hasb.attn_fwd_window(q.cuda(), k.cuda(), v.cuda(), window=window, scale=scale, kv_offset=off)
     torch.cuda.synchronize()
     ref = oracle.attention_fwd(f64(q), f64(k), f64(v), scale, oracle.MASK_WINDOW, off, window=window)
-    _check(o.cpu(), lse.cpu(), *ref, "bf16", what=f"d=256 window {window}", output_ulp=True)
+    _check(o.cpu(), lse.cpu(), *ref, "bf16", what=f"d=256 window {window}",
+           p_bound=_pbound(q, k, v, scale, "bf16", oracle.MASK_WINDOW, off, window=window))
 
 
 @pytest.mark.parametrize("B,Lq,Lk,Hq,Hkv,dtype,mask,off,n", [
@@ -159,6 +163,7 @@ def test_d256_split(B, Lq, Lk, Hq, Hkv, dtype, mask, off, n):
                                          causal=mask, kv_offset=off)
     torch.cuda.synchronize()
     ref = oracle.attention_fwd(f64(q), f64(k), f64(v), scale, mask, off)
-    _check(o.cpu(), lse.cpu(), *ref, "bf16" if dtype == torch.bfloat16 else "fp16",
-           what=f"d=256 split {used}", output_ulp=True)
+    tag = "bf16" if dtype == torch.bfloat16 else "fp16"
+    _check(o.cpu(), lse.cpu(), *ref, tag, what=f"d=256 split {used}",
+           p_bound=_pbound(q, k, v, scale, tag, mask, off))
     assert hasb.device_fault(clear=True) == 0

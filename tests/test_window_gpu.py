@@ -12,7 +12,7 @@ import torch
 import head_attention_streaming_b200 as hasb
 import oracle
 from head_attention_streaming_b200 import inputs
-from test_parity_gpu import _check
+from test_parity_gpu import _check, _pbound
 
 pytestmark = pytest.mark.gpu
 
@@ -24,7 +24,7 @@ def _device(cuda_ok):
     assert hasb.device_fault(clear=True) == 0
 
 
-def _case(B, Lq, Lk, Hq, Hkv, d, dtype, window, off, seed, rows=None, output_ulp=True):
+def _case(B, Lq, Lk, Hq, Hkv, d, dtype, window, off, seed, rows=None, rounding_terms=True):
     q, k, v = inputs.make_qkv(B, Lq, Lk, Hq, Hkv, d, dtype, seed=seed)
     scale = 1.0 / math.sqrt(d)
     o, lse = hasb.attn_fwd_window(q.cuda(), k.cuda(), v.cuda(), window=window, scale=scale, kv_offset=off)
@@ -35,8 +35,9 @@ def _case(B, Lq, Lk, Hq, Hkv, d, dtype, window, off, seed, rows=None, output_ulp
     o_c, l_c = o.cpu(), lse.cpu()
     if rows is not None:
         o_c, l_c = o_c[:, rows], l_c[:, :, rows]
-    _check(o_c, l_c, o_ref, lse_ref, "bf16" if dtype == torch.bfloat16 else "fp16",
-           what=f"window {window}", output_ulp=output_ulp)
+    tag = "bf16" if dtype == torch.bfloat16 else "fp16"
+    pb = _pbound(q, k, v, scale, tag, oracle.MASK_WINDOW, off, rows=rows, window=window) if rounding_terms else None
+    _check(o_c, l_c, o_ref, lse_ref, tag, what=f"window {window}", p_bound=pb)
 
 
 @pytest.mark.parametrize("window", [(256, 256), (100, 0), (0, 100), (300, 37), (-1, 200), (128, -1),
@@ -59,7 +60,7 @@ def test_video_length_local_window_sampled_rows():
     """A 4096-key local window over the 20480-token video sequence (56 heads)."""
     rows = np.sort(np.random.default_rng(3).choice(20480, size=96, replace=False))
     _case(1, 20480, 20480, 56, 56, 128, torch.bfloat16, (2048, 2047), 0, seed=5, rows=rows,
-          output_ulp=False)
+          rounding_terms=False)
 
 
 def test_unbounded_and_causal_windows_match_the_other_masks():
