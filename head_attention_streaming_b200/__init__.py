@@ -5,7 +5,8 @@ The computation runs in ``libattn_sm100.so`` (C ABI in ``include/attn.h``);
 so importing ``head_attention_streaming_b200.inputs`` needs no GPU.
 """
 
-from .binding import (ATTN_ERR_CUDA, ATTN_ERR_INVALID_ARG, ATTN_ERR_TIMEOUT, ATTN_ERR_UNSUPPORTED,
+from .binding import (ATTN_ERR_CUDA, ATTN_ERR_INVALID_ARG, ATTN_ERR_SCRATCH_LIMIT, ATTN_ERR_TIMEOUT,
+                      ATTN_ERR_UNSUPPORTED,
                       ATTN_OK, MASK_CAUSAL, MASK_CHUNK, MASK_NONE, NORM_HEAD, NORM_INNER,
                       NORM_NONE, ROPE_INTERLEAVED, ROPE_NONE, ROPE_SPLIT, AttnError, attn_fwd,
                       attn_fwd_cache, attn_fwd_host, attn_fwd_splitkv, attn_fwd_splitkv_static,
@@ -19,6 +20,7 @@ from .binding import (ATTN_ERR_CUDA, ATTN_ERR_INVALID_ARG, ATTN_ERR_TIMEOUT, ATT
 __all__ = ["attn_fwd", "attn_fwd_host", "AttnError", "lib", "library_path", "status_string", "device_fault",
            "set_wait_timeout_ns", "selftest_mma", "selftest_exp2", "selftest_wait_timeout", "ATTN_OK",
            "ATTN_ERR_INVALID_ARG", "ATTN_ERR_UNSUPPORTED", "ATTN_ERR_CUDA", "ATTN_ERR_TIMEOUT",
+           "ATTN_ERR_SCRATCH_LIMIT",
            "MASK_NONE", "MASK_CAUSAL", "MASK_CHUNK", "qk_prologue", "NORM_NONE", "NORM_HEAD",
            "NORM_INNER", "ROPE_NONE", "ROPE_INTERLEAVED", "ROPE_SPLIT", "attn_fwd_cache", "stream_update",
            "attn_fwd_splitkv", "splitkv_workspace_bytes", "attn_fwd_splitkv_static", "attn_fwd_window",

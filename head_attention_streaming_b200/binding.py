@@ -22,6 +22,7 @@ ATTN_ERR_INVALID_ARG = 1
 ATTN_ERR_UNSUPPORTED = 2
 ATTN_ERR_CUDA = 3
 ATTN_ERR_TIMEOUT = 4
+ATTN_ERR_SCRATCH_LIMIT = 5
 
 MASK_NONE = 0
 MASK_CAUSAL = 1

@@ -1923,6 +1923,7 @@ const char* attn_status_string(int status) {
     case ATTN_ERR_UNSUPPORTED: return "unsupported configuration (head_dim or device)";
     case ATTN_ERR_CUDA: return "CUDA error";
     case ATTN_ERR_TIMEOUT: return "device-side wait timed out";
+    case ATTN_ERR_SCRATCH_LIMIT: return "request exceeds the library's fixed-size scratch";
     default: return "unknown status";
   }
 }
@@ -2072,11 +2073,31 @@ void choose_splits(int requested, int total_tiles, long long base_units, int num
 
 
 // Scratch of attn_fwd_splitkv_static: float32 partial outputs and LSEs of the
-// key ranges, in a file-scope device array (64 MB, reserved when the module is
-// loaded); that entry point allocates nothing. Calls that use it must not
-// overlap in time (one stream, or ordered by the caller).
+// key ranges, in a file-scope device array (64 MB, reserved on every device
+// that loads this library's module, until the process exits); that entry
+// point allocates nothing. Calls that use it must not overlap in time (one
+// stream, or ordered by the caller): they share the array.
 constexpr size_t kStaticScratchFloats = size_t(16) << 20;
 __device__ __align__(256) float g_split_scratch[kStaticScratchFloats];
+
+// Device address of g_split_scratch on the current device. In host code the
+// array's name is only a host-side stand-in, so the address is asked for once
+// per device (with that device current, on the first call there) and kept.
+int static_scratch(float** ptr) {
+  static std::once_flag flags[kMaxDevices];
+  static void* addr[kMaxDevices];
+  static int status[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
+  std::call_once(flags[dev], [dev]() {
+    void* a = nullptr;
+    status[dev] = cudaGetSymbolAddress(&a, g_split_scratch) == cudaSuccess && a != nullptr ? ATTN_OK
+                                                                                        : ATTN_ERR_CUDA;
+    addr[dev] = a;
+  });
+  *ptr = static_cast<float*>(addr[dev]);
+  return status[dev];
+}
 
 // Argument contract of the key-split entry points (no CUDA call).
 int splitkv_validate(const void* q, const void* k, const void* v, const void* o, const float* lse,
@@ -2089,9 +2110,10 @@ int splitkv_validate(const void* q, const void* k, const void* v, const void* o,
   return ATTN_OK;
 }
 
-// The key-split forward after validation. fit: lower the split count until the
-// partials fit the workspace (down to one range, i.e. plain attn_fwd) instead
-// of refusing a workspace that is too small.
+// The key-split forward after validation. fit (the library's fixed scratch):
+// an automatic split count (n_splits = 0) is lowered until the partials fit
+// (down to one range, i.e. plain attn_fwd); an explicit count that does not
+// fit is refused with ATTN_ERR_SCRATCH_LIMIT before anything is launched.
 int splitkv_run(const void* q, const void* k, const void* v, void* o, float* lse, float* workspace,
                 size_t workspace_bytes, bool fit, int n_splits, int B, int Lq, int Lk, int Hq,
                 int Hkv, int d, float scale, int causal, int kv_offset, int dtype, int* splits_used,
@@ -2111,6 +2133,8 @@ int splitkv_run(const void* q, const void* k, const void* v, void* o, float* lse
   int ns = 1, per = total_tiles;
   choose_splits(n_splits, total_tiles, base_units, di.num_sms, &ns, &per, causal == ATTN_MASK_CAUSAL);
   if (fit) {
+    if (n_splits > 0 && ns > 1 && attn_splitkv_workspace_bytes(B, Lq, Hq, d, ns) > workspace_bytes)
+      return ATTN_ERR_SCRATCH_LIMIT;
     while (ns > 1 && attn_splitkv_workspace_bytes(B, Lq, Hq, d, ns) > workspace_bytes) {
       per = (total_tiles + ns - 2) / (ns - 1);
       ns = (total_tiles + per - 1) / per;
@@ -2351,10 +2375,11 @@ int attn_fwd_splitkv_static(const void* q, const void* k, const void* v, void* o
   const int valid = splitkv_validate(q, k, v, o, lse, n_splits, B, Lq, Lk, Hq, Hkv, d, scale, causal,
                                      kv_offset, dtype);
   if (valid != ATTN_OK) return valid;
-  void* ws = nullptr;
-  if (cudaGetSymbolAddress(&ws, g_split_scratch) != cudaSuccess) return ATTN_ERR_CUDA;
-  return splitkv_run(q, k, v, o, lse, static_cast<float*>(ws), sizeof(g_split_scratch), true, n_splits,
-                     B, Lq, Lk, Hq, Hkv, d, scale, causal, kv_offset, dtype, splits_used, stream);
+  float* ws = nullptr;
+  const int st = static_scratch(&ws);
+  if (st != ATTN_OK) return st;
+  return splitkv_run(q, k, v, o, lse, ws, sizeof(g_split_scratch), true, n_splits, B, Lq, Lk, Hq, Hkv, d,
+                     scale, causal, kv_offset, dtype, splits_used, stream);
 }
 
 int attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, void* o_host,

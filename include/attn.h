@@ -31,7 +31,9 @@ typedef enum {
   ATTN_ERR_INVALID_ARG = 1,   /* an argument breaks the contract below; nothing was launched */
   ATTN_ERR_UNSUPPORTED = 2,   /* valid by the pages' contract but not built (head_dim, device) */
   ATTN_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed (launch, descriptor encode) */
-  ATTN_ERR_TIMEOUT = 4        /* a device-side wait ran past its limit (see attn_device_fault) */
+  ATTN_ERR_TIMEOUT = 4,       /* a device-side wait ran past its limit (see attn_device_fault) */
+  ATTN_ERR_SCRATCH_LIMIT = 5  /* the request needs more than the library's fixed-size scratch
+                                 (attn_fwd_splitkv_static); nothing was launched */
 } attn_status_t;
 
 typedef enum { ATTN_DTYPE_BF16 = 0, ATTN_DTYPE_FP16 = 1 } attn_dtype_t;
@@ -211,13 +213,30 @@ int attn_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float
                      int* splits_used, void* stream);
 
 /*
- * attn_fwd_splitkv_static — attn_fwd_splitkv without a workspace argument: the
- * partial outputs live in a 64 MB scratch array inside the library (device
- * memory reserved when the library is loaded), so the call allocates nothing.
- * If the chosen or requested split count needs more scratch, the count is
- * lowered until it fits (down to one range, i.e. attn_fwd); *splits_used
- * reports it. Calls must not overlap in time (one stream, or ordered by the
- * caller): they share the scratch. Arguments and errors as attn_fwd_splitkv.
+ * attn_fwd_splitkv_static — attn_fwd_splitkv for callers that cannot allocate
+ * device memory: no workspace argument, and the call allocates nothing (no
+ * cudaMalloc, no cudaFree, no allocating library routine). It exists for
+ * code that is handed only its input and output buffers, such as a plugin
+ * slot of a host framework with no workspace argument, or a step loop that
+ * must not call cudaMalloc because that call can synchronize the device. The
+ * pages describe no counterpart: it is a packaging of attn_fwd_splitkv.
+ *
+ * Scratch: the float32 partial outputs and LSEs live in one file-scope device
+ * array of 64 MB (16 Mi floats) inside this library. Every GPU that loads the
+ * library holds those 64 MB until the process exits. The first call on a
+ * device looks up the array's device address there (cudaGetSymbolAddress,
+ * with that device current) and keeps it; make that first call before any
+ * stream capture. Every call shares the one array and overwrites it: calls
+ * that overlap on the GPU (two streams, two host threads) race and must be
+ * ordered by the caller. Each call writes every partial it reads before
+ * reading it, so nothing is cleared between calls.
+ *
+ * Limit: with n_splits = 0 the split count is chosen as for attn_fwd_splitkv
+ * and then lowered until attn_splitkv_workspace_bytes(B, Lq, Hq, d, count)
+ * <= 64 MB (down to one range, which runs attn_fwd and needs no scratch). An
+ * explicit n_splits > 1 whose partials need more than 64 MB is refused with
+ * ATTN_ERR_SCRATCH_LIMIT before anything is launched. *splits_used reports
+ * the count used. Other arguments and errors as attn_fwd_splitkv.
  */
 int attn_fwd_splitkv_static(const void* q, const void* k, const void* v, void* o, float* lse,
                             int n_splits, int B, int Lq, int Lk, int Hq, int Hkv, int d, float scale,
