@@ -143,7 +143,7 @@ class ClockSampler:
                 pass
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100", "-i", ident],
+                 "-lms", "20", "-i", ident],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception as e:  # no nvidia-smi: report why
             self.err = str(e)
@@ -176,6 +176,53 @@ class ClockSampler:
                 "samples": len(sm), "power_w_max": max(power) if power else None}
 
 
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def blas_threads() -> int:
+    threads = os.cpu_count()
+    try:
+        from threadpoolctl import threadpool_info
+        info = [i for i in threadpool_info() if i.get("user_api") == "blas"]
+        if info:
+            threads = max(i.get("num_threads", 1) for i in info)
+    except Exception:
+        pass
+    return threads
+
+
+def oracle_full_tflops(w, q, k, v, seconds: float, threads: int | None = None):
+    """The FP64 oracle on the whole workload (every row of every head),
+    repeated until `seconds` have passed (at least once); `threads` limits the
+    BLAS thread pool (None: as configured)."""
+    import contextlib
+
+    import oracle
+    ctx = contextlib.nullcontext()
+    if threads is not None:
+        from threadpoolctl import threadpool_limits
+        ctx = threadpool_limits(limits=threads, user_api="blas")
+    qd, kd, vd = q.double().numpy(), k.double().numpy(), v.double().numpy()
+    with ctx:
+        used = blas_threads()
+        reps, t0 = 0, time.perf_counter()
+        while True:
+            oracle.attention_fwd(qd, kd, vd, w.scale, w.mask, w.kv_offset)
+            reps += 1
+            el = time.perf_counter() - t0
+            if el >= seconds:
+                break
+    return w.flops() * reps / el / 1e12, used, f"whole workload x {reps} (B={w.B}, Lq={w.Lq}, Lk={w.Lk}, Hq={w.Hq}, d={w.d}), numpy float64", el
+
+
 def oracle_sample_tflops(w, q, k, v, seconds: float):
     """FP64 oracle on the workload's seeded sample rows, repeated for >= `seconds`."""
     import numpy as np
@@ -199,14 +246,7 @@ def oracle_sample_tflops(w, q, k, v, seconds: float):
         el = time.perf_counter() - t0
         if el >= seconds:
             break
-    threads = os.cpu_count()
-    try:
-        from threadpoolctl import threadpool_info
-        info = [i for i in threadpool_info() if i.get("user_api") == "blas"]
-        if info:
-            threads = max(i.get("num_threads", 1) for i in info)
-    except Exception:
-        pass
+    threads = blas_threads()
     sample = (f"{len(rows)} seeded query rows of head 0 x {reps} repetitions "
               f"(B={w.B}, Lk={w.Lk}, d={w.d}), numpy float64")
     return f_once * reps / el / 1e12, threads, sample, el
@@ -824,7 +864,8 @@ def main():
         d2h = oh.numel() * oh.element_size() + lh.numel() * lh.element_size()
         e2e = {"value": job_rate(world, w.flops(), e_ms) / 1e12, "unit": "TFLOPS",
                "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "path": "attn_fwd_host (pinned host -> device, forward, device -> host), one stream"}
+               "path": "attn_fwd_host: pinned host K, V -> device first, then query-row chunks whose "
+                       "copies in and out overlap the other chunks' forwards (two copy streams)"}
 
     peaks, peak_src = load_peaks()
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
@@ -853,8 +894,18 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tf, threads, sample, _ = oracle_sample_tflops(w, q_cpu, k_cpu, v_cpu, args.cpu_seconds)
-        cpu = {"value": tf, "unit": "TFLOPS", "cores": threads, "kind": "oracle", "sample": sample}
+        host = {"cpu_model": cpu_model(), "nproc": os.cpu_count()}
+        if w.sample_rows == 0 and not args.shape:
+            # the whole workload; the smallest one also on a single BLAS thread
+            tf, threads, sample, _ = oracle_full_tflops(w, q_cpu, k_cpu, v_cpu, args.cpu_seconds)
+            cpu = {"value": tf, "unit": "TFLOPS", "cores": threads, "kind": "oracle", "sample": sample, **host}
+            if w.name == "bf16_257x8x128":
+                tf1, _, s1, _ = oracle_full_tflops(w, q_cpu, k_cpu, v_cpu, args.cpu_seconds / 2, threads=1)
+                cpu["single_thread"] = {"value": tf1, "unit": "TFLOPS", "cores": 1, "sample": s1}
+        else:
+            tf, threads, sample, _ = oracle_sample_tflops(w, q_cpu, k_cpu, v_cpu, args.cpu_seconds)
+            cpu = {"value": tf, "unit": "TFLOPS", "cores": threads, "kind": "oracle",
+                   "sample": sample + "; sampled rows, the rate stands for the whole workload", **host}
 
     if rank == 0:
         line = {

@@ -28,6 +28,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdint>
@@ -2216,6 +2217,116 @@ int splitkv_run(const void* q, const void* k, const void* v, void* o, float* lse
 
 
 
+// ------------------------------------------------------ host-buffer pipeline
+
+// attn_fwd_host's copies overlap the attention: K and V go first, then the
+// query rows in chunks (per batch, a multiple of 256 rows, the kernel's unit,
+// so each chunk computes exactly what the whole call computes for its rows),
+// each chunk's forward starting once its Q has landed and its O (and LSE)
+// going back while the next chunk computes. Host-to-device copies run on one
+// internal stream, device-to-host copies on another, the forwards on the
+// caller's stream; events order them, and the caller's stream waits for the
+// last copy, so synchronizing it covers the whole call. The streams and
+// events are created once per device and reused (calls on one device are
+// serialized by a mutex while they are queued).
+constexpr int kHostChunks = 16;
+
+struct HostPipe {
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t start = nullptr, kv_in = nullptr, done = nullptr;
+  cudaEvent_t q_in[kHostChunks] = {}, fwd_done[kHostChunks] = {};
+  std::mutex m;
+};
+
+HostPipe* host_pipe(int dev) {
+  static HostPipe pipes[kMaxDevices];
+  static std::once_flag flags[kMaxDevices];
+  static bool ok[kMaxDevices];
+  if (dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::call_once(flags[dev], [dev]() {
+    HostPipe& hp = pipes[dev];
+    bool good = cudaStreamCreateWithFlags(&hp.h2d, cudaStreamNonBlocking) == cudaSuccess &&
+                cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking) == cudaSuccess &&
+                cudaEventCreateWithFlags(&hp.start, cudaEventDisableTiming) == cudaSuccess &&
+                cudaEventCreateWithFlags(&hp.kv_in, cudaEventDisableTiming) == cudaSuccess &&
+                cudaEventCreateWithFlags(&hp.done, cudaEventDisableTiming) == cudaSuccess;
+    for (int c = 0; c < kHostChunks && good; ++c)
+      good = cudaEventCreateWithFlags(&hp.q_in[c], cudaEventDisableTiming) == cudaSuccess &&
+             cudaEventCreateWithFlags(&hp.fwd_done[c], cudaEventDisableTiming) == cudaSuccess;
+    ok[dev] = good;
+  });
+  return ok[dev] ? &pipes[dev] : nullptr;
+}
+
+int host_pipeline(HostPipe& hp, const void* q_host, const void* k_host, const void* v_host, void* o_host,
+                  float* lse_host, void* q_dev, void* k_dev, void* v_dev, void* o_dev, float* lse_dev, int B,
+                  int Lq, int Lk, int Hq, int Hkv, int d, float scale, int causal, int kv_offset, int dtype,
+                  cudaStream_t s) {
+  const size_t row_bytes = 2ull * Hq * d;      // one query row of Q or O, all heads
+  const size_t kv_bytes = 2ull * B * Lk * Hkv * d;
+  // chunks of whole 256-row pairs, at most kHostChunks in all
+  const long long per_b = (kHostChunks + B - 1) / B;
+  const long long want = (Lq + per_b - 1) / per_b;
+  const int rows = static_cast<int>(((want + 255) / 256) * 256);
+  const int n_per_b = (Lq + rows - 1) / rows;
+  const int n_chunks = B * n_per_b;
+  if (n_chunks > kHostChunks) return ATTN_ERR_INVALID_ARG;  // cannot happen for B <= kHostChunks
+  const auto bad = [](cudaError_t e) { return e != cudaSuccess; };
+  // streams: the copies wait for everything the caller queued before this call
+  if (bad(cudaEventRecord(hp.start, s)) || bad(cudaStreamWaitEvent(hp.h2d, hp.start, 0)) ||
+      bad(cudaStreamWaitEvent(hp.d2h, hp.start, 0)))
+    return ATTN_ERR_CUDA;
+  if (bad(cudaMemcpyAsync(k_dev, k_host, kv_bytes, cudaMemcpyHostToDevice, hp.h2d)) ||
+      bad(cudaMemcpyAsync(v_dev, v_host, kv_bytes, cudaMemcpyHostToDevice, hp.h2d)) ||
+      bad(cudaEventRecord(hp.kv_in, hp.h2d)))
+    return ATTN_ERR_CUDA;
+  for (int c = 0; c < n_chunks; ++c) {
+    const int b = c / n_per_b, r0 = (c % n_per_b) * rows;
+    const size_t off = (static_cast<size_t>(b) * Lq + r0) * row_bytes;
+    const size_t len = static_cast<size_t>(std::min(rows, Lq - r0)) * row_bytes;
+    if (bad(cudaMemcpyAsync(static_cast<char*>(q_dev) + off, static_cast<const char*>(q_host) + off, len,
+                            cudaMemcpyHostToDevice, hp.h2d)) ||
+        bad(cudaEventRecord(hp.q_in[c], hp.h2d)))
+      return ATTN_ERR_CUDA;
+  }
+  if (bad(cudaStreamWaitEvent(s, hp.kv_in, 0))) return ATTN_ERR_CUDA;
+  for (int c = 0; c < n_chunks; ++c) {
+    const int b = c / n_per_b, r0 = (c % n_per_b) * rows, n = std::min(rows, Lq - r0);
+    const size_t qo = (static_cast<size_t>(b) * Lq + r0) * Hq * d;          // elements
+    const size_t kvo = static_cast<size_t>(b) * Lk * Hkv * d;
+    // this chunk's LSE: [Hq, n] floats at the chunk's place in the batch's LSE area
+    float* lse_c = lse_dev == nullptr ? nullptr : lse_dev + static_cast<size_t>(b) * Hq * Lq +
+                                                      static_cast<size_t>(Hq) * r0;
+    // masks for a row range [r0, r0 + n): causal rows see j <= kv_offset + r (offset moves with r0);
+    // chunk rows see every key below kv_offset + Lq (no mask over that key prefix)
+    int mask = causal, off = kv_offset, lk = Lk;
+    if (causal == ATTN_MASK_CAUSAL) {
+      off = kv_offset + r0;
+    } else if (causal == ATTN_MASK_CHUNK) {
+      mask = ATTN_MASK_NONE;
+      off = 0;
+      lk = kv_offset + Lq;
+    }
+    if (bad(cudaStreamWaitEvent(s, hp.q_in[c], 0))) return ATTN_ERR_CUDA;
+    const int st = attn_fwd_impl(static_cast<const uint16_t*>(q_dev) + qo, static_cast<const uint16_t*>(k_dev) + kvo,
+                                 static_cast<const uint16_t*>(v_dev) + kvo, static_cast<uint16_t*>(o_dev) + qo, lse_c,
+                                 1, n, lk, Lk, Hq, Hkv, d, scale, mask, off, dtype, s);
+    if (st != ATTN_OK) return st;
+    if (bad(cudaEventRecord(hp.fwd_done[c], s)) || bad(cudaStreamWaitEvent(hp.d2h, hp.fwd_done[c], 0)) ||
+        bad(cudaMemcpyAsync(static_cast<char*>(o_host) + qo * 2, static_cast<const char*>(o_dev) + qo * 2,
+                            static_cast<size_t>(n) * row_bytes, cudaMemcpyDeviceToHost, hp.d2h)))
+      return ATTN_ERR_CUDA;
+    if (lse_host != nullptr &&
+        bad(cudaMemcpy2DAsync(lse_host + static_cast<size_t>(b) * Hq * Lq + r0, static_cast<size_t>(Lq) * 4,
+                              lse_c, static_cast<size_t>(n) * 4, static_cast<size_t>(n) * 4, Hq,
+                              cudaMemcpyDeviceToHost, hp.d2h)))
+      return ATTN_ERR_CUDA;
+  }
+  // the caller's stream covers the whole call
+  if (bad(cudaEventRecord(hp.done, hp.d2h)) || bad(cudaStreamWaitEvent(s, hp.done, 0))) return ATTN_ERR_CUDA;
+  return ATTN_OK;
+}
+
 }  // namespace hasb
 
 extern "C" {
@@ -2389,28 +2500,18 @@ int attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, vo
   if (!q_host || !k_host || !v_host || !o_host) return ATTN_ERR_INVALID_ARG;
   if ((lse_host == nullptr) != (lse_dev == nullptr)) return ATTN_ERR_INVALID_ARG;
   if (B < 1 || Lq < 1 || Lk < 1 || Hq < 1 || Hkv < 1 || d < 1) return ATTN_ERR_INVALID_ARG;
-  const size_t q_bytes = 2ull * B * Lq * Hq * d;
-  const size_t kv_bytes = 2ull * B * Lk * Hkv * d;
-  const size_t lse_bytes = 4ull * B * Hq * Lq;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // attn_fwd checks the device side; run its validation first by a dry call
-  // ordering: copies only once the arguments are known to be valid
+  // the device side's contract first: no copy is queued for a call attn_fwd would refuse
   const int pre = attn_fwd_validate(q_dev, k_dev, v_dev, o_dev, lse_dev, B, Lq, Lk, Hq, Hkv, d, scale,
                                     causal, kv_offset, dtype, Lk);
   if (pre != ATTN_OK) return pre;
-  if (cudaMemcpyAsync(q_dev, q_host, q_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      cudaMemcpyAsync(k_dev, k_host, kv_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      cudaMemcpyAsync(v_dev, v_host, kv_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
-    return ATTN_ERR_CUDA;
-  const int st = attn_fwd(q_dev, k_dev, v_dev, o_dev, lse_dev, B, Lq, Lk, Hq, Hkv, d, scale, causal,
-                          kv_offset, dtype, stream);
-  if (st != ATTN_OK) return st;
-  if (cudaMemcpyAsync(o_host, o_dev, q_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
-    return ATTN_ERR_CUDA;
-  if (lse_host != nullptr &&
-      cudaMemcpyAsync(lse_host, lse_dev, lse_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
-    return ATTN_ERR_CUDA;
-  return ATTN_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+  HostPipe* hp = host_pipe(dev);
+  if (hp == nullptr) return ATTN_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(hp->m);
+  return host_pipeline(*hp, q_host, k_host, v_host, o_host, lse_host, q_dev, k_dev, v_dev, o_dev, lse_dev, B,
+                       Lq, Lk, Hq, Hkv, d, scale, causal, kv_offset, dtype, s);
 }
 
 int attn_device_fault(unsigned int* bits, int clear) {

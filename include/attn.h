@@ -245,13 +245,23 @@ int attn_fwd_splitkv_static(const void* q, const void* k, const void* v, void* o
 /*
  * attn_fwd_host — the same forward for operands in host memory: copies q, k, v
  * from host to the caller's device buffers, runs attn_fwd, and copies o (and
- * lse when both lse pointers are given) back to host memory, all queued on
- * `stream` in that order (cudaMemcpyAsync; use pinned host memory for
- * asynchronous copies). The call returns once the work is queued; synchronize
- * `stream` before reading o_host. Shapes, dtype, mask and errors as attn_fwd;
- * additionally every host pointer but lse_host must be non-NULL, and lse_host
- * and lse_dev must be both NULL or both non-NULL. Device buffers are owned by
- * the caller and sized as attn_fwd's q, k, v, o, lse.
+ * lse when both lse pointers are given) back to host memory. The copies
+ * overlap the computation: k and v go first, then q in chunks of whole
+ * 256-row query pairs (per batch, at most 16 chunks in all); each chunk's
+ * forward starts once its rows have landed and its o (and lse) rows go back
+ * while the next chunk computes. Chunks hold whole work units of attn_fwd,
+ * so o and lse are bit-identical to one attn_fwd call. Host-to-device and
+ * device-to-host copies run on two streams the library creates once per
+ * device; the forwards run on `stream`, which waits for everything before the
+ * call returns control of it: synchronize `stream` before reading o_host (use
+ * pinned host memory: pageable memory serializes the copies). Calls on one
+ * device are queued one at a time (a per-device lock while queueing).
+ * Shapes, dtype, mask and errors as attn_fwd; additionally every host pointer
+ * but lse_host must be non-NULL, and lse_host and lse_dev must be both NULL
+ * or both non-NULL. Device buffers are owned by the caller and sized as
+ * attn_fwd's q, k, v, o, lse; lse_dev is used as scratch (after the call it
+ * holds each chunk's [Hq, rows] block in chunk order, not the [B, Hq, Lq]
+ * layout of lse_host).
  */
 int attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, void* o_host,
                   float* lse_host, void* q_dev, void* k_dev, void* v_dev, void* o_dev,
