@@ -14,7 +14,9 @@ import os
 
 import torch
 
-_SO_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libattn_sm100.so")
+# HASB_DEBUG=1 loads the index-checking debug build (-DATTN_DEBUG) instead
+_SO_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                        "libattn_sm100_debug.so" if os.environ.get("HASB_DEBUG") == "1" else "libattn_sm100.so")
 _LIB = None
 
 ATTN_OK = 0
@@ -71,6 +73,8 @@ _SIGNATURES = {
     "attn_rope_after_cache": (ctypes.c_int, [ctypes.c_void_p] * 5 + [ctypes.c_int] * 2 + [ctypes.c_void_p] +
                               [ctypes.c_int] * 9 + [ctypes.c_void_p]),
     "attn_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "attn_debug_fault_site": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint), ctypes.c_int]),
+    "attn_debug_build": (ctypes.c_int, []),
     "attn_device_fault": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint), ctypes.c_int]),
     "attn_set_wait_timeout_ns": (ctypes.c_int, [ctypes.c_ulonglong]),
     "attn_selftest_mma": (ctypes.c_int, [ctypes.c_void_p] * 5 + [ctypes.c_int, ctypes.c_void_p]),
@@ -636,6 +640,21 @@ def device_fault(clear: bool = True) -> int:
     if st not in (ATTN_OK, ATTN_ERR_TIMEOUT):
         raise AttnError(st, "attn_device_fault")
     return int(bits.value)
+
+
+def debug_fault_site(clear: bool = True) -> int:
+    """Synchronize the device and return (optionally clearing) the site number
+    of the first failed index check of the debug build (0: none; always 0 in
+    the release build)."""
+    site = ctypes.c_uint(0)
+    st = lib().attn_debug_fault_site(ctypes.byref(site), 1 if clear else 0)
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_debug_fault_site")
+    return int(site.value)
+
+
+def is_debug_build() -> bool:
+    return bool(lib().attn_debug_build())
 
 
 def set_wait_timeout_ns(ns: int) -> None:

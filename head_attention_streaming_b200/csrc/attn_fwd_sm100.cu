@@ -46,6 +46,9 @@ namespace hasb {
 
 // Device fault word: bit set by a kernel whose bounded wait ran out.
 __device__ unsigned int g_fault_bits = 0;
+// Debug build (-DATTN_DEBUG): the site number of the first index check that
+// failed in this file's kernels (0: none).
+__device__ unsigned int g_debug_site = 0;
 
 enum FaultBit : unsigned int {
   kFaultLoadQEmpty = 1u << 0,
@@ -59,7 +62,26 @@ enum FaultBit : unsigned int {
   kFaultStore = 1u << 9,
   kFaultSelftest = 1u << 8,
   kFaultMmaSFree = 1u << 10,
+  kFaultBounds = 1u << 11,  // debug build: an index check failed (site in attn_debug_fault_site)
 };
+
+// Index checks of the debug build (-DATTN_DEBUG): a check that fails sets
+// kFaultBounds, records its site number (the first failure wins) and makes
+// the caller skip the access; the kernel goes on, so no wait of another role
+// is left without its arrival. In the release build a check is `true` and
+// compiles away.
+__device__ __forceinline__ bool debug_check(bool ok, unsigned int site) {
+  if (!ok) {
+    atomicOr(&g_fault_bits, kFaultBounds);
+    atomicCAS(&g_debug_site, 0u, site);
+  }
+  return ok;
+}
+#ifdef ATTN_DEBUG
+#define ATTN_CHECK(cond, site) (::hasb::debug_check((cond), (site)))
+#else
+#define ATTN_CHECK(cond, site) true
+#endif
 
 constexpr int kThreads = 384;
 // Register split: 384 threads x 168 launch registers = 64512. The producer
@@ -82,11 +104,13 @@ struct Cfg {
   static constexpr int kOffKV = 2 * kTileBytes;
   static constexpr int kOffStg = kOffKV + kStages * kTileBytes;  // O staging for the TMA store
   static constexpr int kOffBar = kOffStg + kTileBytes;
-  static constexpr int kSmemBytes = kOffBar + 512 + 1024;  // barriers + 1 KB alignment slack
+  static constexpr int kOffMl = kOffBar + 512;  // pair-split merge: slot 1's (reference, row sum) per row
+  static constexpr int kSmemBytes = kOffMl + 1024 + 1024;  // + 1 KB alignment slack
   // tensor-memory columns of S_t (P_t aliased) and O_t
   static __device__ __forceinline__ uint32_t col_s(int t) { return t ? 128u : 0u; }
   static __device__ __forceinline__ uint32_t col_o(int t) { return t ? 256u + D : 256u; }
   static constexpr uint32_t kTmemCols = 512;
+  static_assert(256 + 2 * D <= 512, "S_0, S_1, O_0, O_1 must fit the 512 tensor-memory columns");
   static constexpr int kOChunks = D / 64;  // 64-column chunks of the 16-bit O staging tile
   static constexpr int kOffP = 0;          // P lives in tensor memory
   static constexpr int kOffSk = 0;         // no key scales
@@ -189,6 +213,8 @@ enum Bar : int {
   kBarStgFull = 32, //     softmax t -> store warp: O tile t staged (one arrival per warp)
   kBarStgFree = 34, // [2] store warp -> softmax t: staging buffer is t's to fill
   kBarSFree = 36,   // [2] d = 256, P V issuer -> Q K^T issuer: the P V that read S buffer b is done
+  kBarMerge1 = 38,  //     pair split, softmax 1 -> softmax 0: slot 1's (reference, row sum) written
+  kBarMerged = 39,  //     pair split, softmax 0 -> softmax 1: the merge has read slot 1's O and row state
 };
 
 // Exponentials of the softmax: kPolyPairsPer8 of every 8 score pairs take
@@ -274,6 +300,55 @@ struct Unit {
 };
 
 __device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+// The k-th work unit of this CTA, or -1 once none is left. Units are dealt in
+// rounds of gridDim.x, alternately forward and backward: with units ordered
+// longest first (causal), the CTA that takes one of the longest units of a
+// round takes one of the shortest of the next. Every role of a CTA walks the
+// same sequence. A partial round is always the last, so the walk stops at
+// the first unit past the end.
+__device__ __forceinline__ int cta_unit(int k, int n_units) {
+  const int g = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
+  const long long u = (k & 1) ? 1LL * (k + 1) * g - 1 - c : 1LL * k * g + c;
+  return u < n_units ? static_cast<int>(u) : -1;
+}
+
+// Pair-split work unit (causal problems with fewer row pairs than SMs): u ->
+// (b, hq, one 128-row query tile) whose n visible KV tiles are split between
+// the CTA's two slots, slot 0 taking KV tiles [0, n0), slot 1 [n0, n),
+// n0 = ceil(n / 2); the two partial results are merged by their row maxima
+// and sums (the regrouped softmax) before the store. Units run longest first
+// over all heads (the tile index varies slowest); p.n_pairs counts the tiles.
+__device__ __forceinline__ Unit decode_pair(const FwdParams& p, int u) {
+  Unit x;
+  x.split = 0;
+  const int bh = p.B * p.Hq;
+  const int rank = u / bh;
+  int t = u % bh;
+  const int g = t % p.group;
+  t /= p.group;
+  x.hkv = t % p.Hkv;
+  x.b = t / p.Hkv;
+  x.hq = x.hkv * p.group + g;
+  x.r0 = (p.n_pairs - 1 - rank) * kTileRows;
+  const int n = cdiv(min(p.Lk, p.kv_offset + x.r0 + kTileRows), kTileRows);
+  x.j0 = 0;
+  x.n0 = (n + 1) / 2;
+  x.n1 = n - x.n0;
+  x.s0 = 0;
+  x.s1 = x.n0;
+  x.nu = n;
+  return x;
+}
+// The two slots' KV tiles are streamed interleaved (0, n0, 1, n0 + 1, ...),
+// slot 0's extra tile (n0 = n1 + 1) last: stream position of slot t's k-th
+// tile, and the KV tile at a stream position.
+__device__ __forceinline__ int pair_pos(const Unit& x, int t, int k) {
+  return k < x.n1 ? 2 * k + t : x.n1 + k;
+}
+__device__ __forceinline__ int pair_tile(const Unit& x, int pos) {
+  return pos < 2 * x.n1 ? ((pos & 1) ? x.n0 + pos / 2 : pos / 2) : pos - x.n1;
+}
 
 // Work unit u -> (b, hq, row pair). Query heads of one GQA group are adjacent
 // and the row pairs of one head are adjacent, so CTAs running together read
@@ -484,7 +559,7 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint3
   issue_pv_half<D, BF16, 1>(d_tmem, p_tmem, v_lo, 1u);
 }
 
-template <int D, bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW, int F8>
+template <int D, bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW, int F8, bool PAIR = false>
 __device__ __forceinline__ void load_role(const CUtensorMap* tm_q, const CUtensorMap* tm_k,
                                           const CUtensorMap* tm_v, const FwdParams& p,
                                           uint32_t sQ, uint32_t sKV, uint32_t bars,
@@ -500,9 +575,10 @@ __device__ __forceinline__ void load_role(const CUtensorMap* tm_q, const CUtenso
   for (int i = 0; i < C::kStages; ++i) slot_last[i] = -1;
   int q_last[2] = {-1, -1};
   bool aborted = false;
-  for (int u = blockIdx.x; u < p.n_units && !aborted; u += gridDim.x, ++uit) {
+  for (int u = cta_unit(0, p.n_units); u >= 0 && !aborted; u = cta_unit(++uit, p.n_units)) {
     Unit x;
-    if constexpr (D == 256) x = decode_single<CAUSAL, SPLIT, WINDOW>(p, u);
+    if constexpr (PAIR) x = decode_pair(p, u);
+    else if constexpr (D == 256) x = decode_single<CAUSAL, SPLIT, WINDOW>(p, u);
     else x = decode_unit<CAUSAL, SPLIT, WINDOW>(p, u);
     for (int t = 0; t < (D == 256 ? 1 : 2); ++t) {
       const uint32_t bq = bars + 8 * (kBarQEmpty + t);
@@ -512,15 +588,23 @@ __device__ __forceinline__ void load_role(const CUtensorMap* tm_q, const CUtenso
       }
       const uint32_t bf = bars + 8 * (kBarQFull + t);
       mbar_arrive_expect_tx(bf, C::kTileBytes);
+      // site 1: the Q tile's head, batch and first row lie inside q
+      (void)ATTN_CHECK(x.hq >= 0 && x.hq < p.Hq && x.b >= 0 && x.b < p.B && x.r0 >= 0 &&
+                           x.r0 + (PAIR ? 0 : t * kTileRows) < p.Lq + kTileRows,
+                       1);
 #pragma unroll
       for (int c = 0; c < C::kChunks; ++c)  // 128 bytes a chunk: 64 16-bit or 128 e4m3 elements
         tma_load_4d(sQ + t * C::kTileBytes + c * C::kChunkBytes, tm_q, bf, c * (F8 != 0 ? 128 : 64), x.hq,
-                    x.r0 + t * kTileRows, x.b, pol_q);
+                    x.r0 + (PAIR ? 0 : t * kTileRows), x.b, pol_q);  // pair split: both slots, the same rows
       q_last[t] = uit & 1;
     }
-    // one K or V tile into its ring slot (ring index kv_it + 2 jj + kv)
+    // one K or V tile into its ring slot (ring index kv_it + 2 jj + kv); pair
+    // split: stream position jj holds KV tile pair_tile(jj)
     auto load_one = [&](int jj, int kv) -> bool {
       const int idx = kv_it + 2 * jj + kv;
+      const int tile = PAIR ? pair_tile(x, jj) : jj;
+      // site 2: the K / V tile starts inside the keys of its head and batch
+      (void)ATTN_CHECK(x.hkv >= 0 && x.hkv < p.Hkv && tile >= 0 && (x.j0 + tile) * kTileRows < p.Lk, 2);
       const int slot = idx % C::kStages;
       const uint32_t be = bars + 8 * (kBarKvEmpty + slot);
       if (!mbar_wait(be, ((idx / C::kStages) & 1) ^ 1, abort_flag, kFaultLoadKvEmpty, p.timeout_ns))
@@ -542,7 +626,7 @@ __device__ __forceinline__ void load_role(const CUtensorMap* tm_q, const CUtenso
 #pragma unroll
         for (int c = 0; c < C::kChunks; ++c)
           tma_load_4d(sKV + slot * C::kTileBytes + c * C::kChunkBytes, kv ? tm_v : tm_k, bf,
-                      c * 64, x.hkv, (x.j0 + jj) * kTileRows, x.b, pol_kv);
+                      c * 64, x.hkv, (x.j0 + tile) * kTileRows, x.b, pol_kv);
       }
       slot_last[slot] = idx;
       return true;
@@ -587,7 +671,7 @@ __device__ __forceinline__ void load_role(const CUtensorMap* tm_q, const CUtenso
 // issuing the other's GEMMs. With one thread per tile, the tensor core runs
 // whichever tile has work. Both threads read the same K/V ring slots; each slot
 // use is released by both (kv_empty takes two arrivals).
-template <int D, bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW, int F8>
+template <int D, bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW, int F8, bool PAIR = false>
 __device__ __forceinline__ void mma_role(const int t, const FwdParams& p, uint32_t tmem, uint32_t sQ,
                                          uint32_t sKV, uint32_t sP, uint32_t bars,
                                          volatile int* abort_flag) {
@@ -610,15 +694,18 @@ __device__ __forceinline__ void mma_role(const int t, const FwdParams& p, uint32
   const uint32_t s_t = tmem + C::col_s(t), o_t = tmem + C::col_o(t);
   int kv_it = 0, uit = 0, pcnt = 0;
   bool ok = true;
-  for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++uit) {
-    const Unit x = decode_unit<CAUSAL, SPLIT, WINDOW>(p, u);
+  for (int u = cta_unit(0, p.n_units); u >= 0 && ok; u = cta_unit(++uit, p.n_units)) {
+    Unit x;
+    if constexpr (PAIR) x = decode_pair(p, u);
+    else x = decode_unit<CAUSAL, SPLIT, WINDOW>(p, u);
     const int n = t ? x.n1 : x.n0;  // KV tiles this query tile uses
     const int s = WINDOW ? (t ? x.s1 : x.s0) : 0;  // ... starting this many tiles into the stream
     ok = mbar_wait(bar(kBarQFull + t), uit & 1, abort_flag, kFaultMmaQFull, p.timeout_ns);
-    if (CAUSAL && SPLIT && n == 0) {
-      // no key of this split is visible to the tile: release Q and pass the
-      // unit's tiles through. O is neither written nor signalled: the softmax
-      // decodes the same empty tile and writes the empty partial itself (an
+    if ((CAUSAL && SPLIT || PAIR) && n == 0) {
+      // no key of this split is visible to the tile (pair split: slot 1 of a
+      // one-tile range): release Q and pass the unit's tiles through. O is
+      // neither written nor signalled: the softmax decodes the same empty tile
+      // and writes the empty partial (pair split: an empty row state) itself (an
       // O-full commit here, with no hand-shake from the softmax, could complete
       // the barrier's phase twice before the softmax looked at it)
       if (!ok) break;
@@ -644,7 +731,18 @@ __device__ __forceinline__ void mma_role(const int t, const FwdParams& p, uint32
         }
       }
     }
-    const int kb = kv_it + 2 * s;  // ring index of this query tile's first K
+    // ring index of this query tile's j-th K (pair split: its stream position)
+    auto kring = [&](int j) { return kv_it + 2 * (PAIR ? pair_pos(x, t, j) : s + j); };
+    // pair split: release the other slot's stream positions [a, b) (K and V)
+    auto pass_positions = [&](int a, int b) {
+      for (int q = 2 * a; q < 2 * b && ok; ++q) {
+        const int idx = kv_it + q;
+        if (!kv_full(idx)) { ok = false; break; }
+        mbar_arrive(bar(kBarKvEmpty + idx % C::kStages));
+      }
+    };
+    if constexpr (PAIR) pass_positions(0, pair_pos(x, t, 0));
+    const int kb = kring(0);  // ring index of this query tile's first K
     ok = ok && kv_full(kb);
     if (!ok) break;
     // S_t(0) = Q_t K_0^T
@@ -654,8 +752,8 @@ __device__ __forceinline__ void mma_role(const int t, const FwdParams& p, uint32
     mma_commit(bar(kBarKvEmpty + kb % C::kStages));
     if (n == 1) mma_commit(bar(kBarQEmpty + t));
     for (int j = 0; j < n; ++j) {
-      const int vidx = kb + 2 * j + 1;  // V_j
-      const int knext = vidx + 1;          // K_{j+1}
+      const int vidx = kring(j) + 1;                  // V_j
+      const int knext = j + 1 < n ? kring(j + 1) : 0;  // K_{j+1}
       // O_t += P_t V_j: the first 64 keys as soon as their half of P is in
       // tensor memory, the rest once all of P is
       if (!kv_full(vidx) ||
@@ -678,6 +776,10 @@ __device__ __forceinline__ void mma_role(const int t, const FwdParams& p, uint32
       if (j == n - 1) {
         mma_commit(bar(kBarOFull + t));
       } else {
+        if constexpr (PAIR) {
+          pass_positions(pair_pos(x, t, j) + 1, pair_pos(x, t, j + 1));
+          if (!ok) break;
+        }
         if (!kv_full(knext)) { ok = false; break; }
         if constexpr (F8 != 0) issue_qk_f8<D>(s_t, q_lo, k_lo(knext));
         else issue_qk<D, BF16>(s_t, q_lo, k_lo(knext));
@@ -689,7 +791,8 @@ __device__ __forceinline__ void mma_role(const int t, const FwdParams& p, uint32
     // causal / window: tiles after this query tile's range still pass through
     // the ring; release this thread's share once each has landed (waiting for
     // the landing keeps the arrival in the slot's current phase)
-    for (int j = s + n; j < x.nu && ok; ++j) {
+    if constexpr (PAIR) pass_positions(pair_pos(x, t, n - 1) + 1, x.nu);
+    for (int j = PAIR ? x.nu : s + n; j < x.nu && ok; ++j) {
       for (int kv = 0; kv < 2 && ok; ++kv) {
         const int idx = kv_it + 2 * j + kv;
         if (!kv_full(idx)) { ok = false; break; }
@@ -833,34 +936,40 @@ __device__ __forceinline__ void exp_tile(const uint32_t (&r)[128], float sl2, fl
 // buffer to global memory with a TMA store (rows past Lq are clipped by the
 // tensor map), then hands the buffer to the other query tile. Order per unit:
 // tile 0, then tile 1, the same order the softmax warpgroups fill it in.
-template <int D, bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW, int F8>
+template <int D, bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW, int F8, bool PAIR = false>
 __device__ __forceinline__ void store_role(const CUtensorMap* tm_o, const FwdParams& p, uint32_t sStg,
                                            uint32_t bars, volatile int* abort_flag) {
   using C = Cfg<D, F8>;
   int scnt = 0;
   bool ok = true;
-  for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-    const Unit x = decode_unit<CAUSAL, SPLIT, WINDOW>(p, u);
-    for (int t = 0; t < 2 && ok; ++t) {
+  int k = 0;
+  for (int u = cta_unit(0, p.n_units); u >= 0 && ok; u = cta_unit(++k, p.n_units)) {
+    Unit x;
+    if constexpr (PAIR) x = decode_pair(p, u);
+    else x = decode_unit<CAUSAL, SPLIT, WINDOW>(p, u);
+    for (int t = 0; t < (PAIR ? 1 : 2) && ok; ++t) {  // pair split: one merged tile per unit
       ok = mbar_wait(bars + 8 * kBarStgFull, scnt & 1, abort_flag, kFaultStore, p.timeout_ns);
       if (!ok) break;
       ++scnt;
       const int dt = p.d > 0 ? p.d : D;  // a chunk wholly past the tensor's head dim is not stored
+      // site 3: a TMA store never starts at a negative coordinate
+      const bool st_ok = ATTN_CHECK(x.r0 >= 0 && x.hq >= 0 && x.hq < p.Hq && x.b >= 0 && x.b < p.B, 3);
 #pragma unroll
       for (int c = 0; c < C::kOChunks; ++c)
-        if (c * 64 < dt) tma_store_4d(tm_o, sStg + c * C::kChunkBytes, c * 64, x.hq, x.r0 + t * kTileRows, x.b);
+        if (c * 64 < dt && st_ok)
+          tma_store_4d(tm_o, sStg + c * C::kChunkBytes, c * 64, x.hq, x.r0 + t * kTileRows, x.b);
       bulk_commit_group();
       bulk_wait_group_read0();
-      mbar_arrive(bars + 8 * (kBarStgFree + (1 - t)));
+      mbar_arrive(bars + 8 * (kBarStgFree + (PAIR ? 0 : 1 - t)));
     }
   }
   bulk_wait_group0();  // every store complete before the CTA exits
 }
 
-template <int D, bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW, int F8>
+template <int D, bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW, int F8, bool PAIR = false>
 __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, uint32_t tmem,
                                              uint32_t bars, uint32_t sstg, uint32_t sP, uint32_t sSk,
-                                             volatile int* abort_flag) {
+                                             uint32_t sMl, volatile int* abort_flag) {
   using C = Cfg<D, F8>;
   const uint32_t prow = sP + t * C::kTileBytes + (threadIdx.x % kTileRows) * 128;  // e4m3 P row
   // per-token scales: this warp's copy of the current KV tile's 128 key scales
@@ -883,12 +992,26 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
   const uint32_t bar_o = bars + 8 * (kBarOFull + t);
   const float sl2 = p.sl2;
   int scnt = 0, ocnt = 0;
+  int o1cnt = 0;  // pair split: units whose slot 1 had KV tiles (phases of slot 1's O-full barrier)
+  // (WINDOW || PAIR): per-slot KV ranges, tile 0 may have more steps than tile 1
+  constexpr bool kRanges = WINDOW || PAIR;
 
-  for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
-    const Unit x = decode_unit<CAUSAL, SPLIT, WINDOW>(p, u);
+  int k = 0;
+  for (int u = cta_unit(0, p.n_units); u >= 0; u = cta_unit(++k, p.n_units)) {
+    Unit x;
+    if constexpr (PAIR) x = decode_pair(p, u);
+    else x = decode_unit<CAUSAL, SPLIT, WINDOW>(p, u);
     const int n = t ? x.n1 : x.n0;
-    const int s = WINDOW ? (t ? x.s1 : x.s0) : 0;  // first KV tile of this query tile, relative to x.j0
-    const int row = x.r0 + t * kTileRows + r_in;
+    const int s = kRanges ? (t ? x.s1 : x.s0) : 0;  // first KV tile of this query tile, relative to x.j0
+    const int row = x.r0 + (PAIR ? 0 : t * kTileRows) + r_in;  // pair split: both slots, the same rows
+    if constexpr (PAIR) {
+      // slot 1 reuses its O and row-state buffers only once slot 0 has merged the previous unit
+      if (t == 1 && k > 0) {
+        const bool okm = mbar_wait(bars + 8 * kBarMerged, (k - 1) & 1, abort_flag, kFaultSoftmaxOFull,
+                                   p.timeout_ns);
+        if (!__all_sync(0xffffffffu, okm)) return;
+      }
+    }
     // visible keys of this row: [row_lo, row_lim)
     int row_lim = CAUSAL ? min(p.Lk, p.kv_offset + row + 1) : p.kv_limit;
     int row_lo = 0;
@@ -906,7 +1029,11 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
     float4 skv = make_float4(0.f, 0.f, 0.f, 0.f);
     if constexpr (F8 == 2) {
       const size_t qs = (static_cast<size_t>(x.b) * p.Hq + x.hq) * p.sq_pitch + row;
-      sl2r = sl2 * (row < p.Lq ? __ldg(p.sq + qs) : 1.f);
+      // site 6: the row's and the head's scales lie inside [B, H, pitch]
+      const bool sok = ATTN_CHECK(x.b < p.B && x.hq < p.Hq && x.hkv < p.Hkv && p.Lq <= p.sq_pitch &&
+                                      p.Lk <= p.sk_pitch,
+                                  6);
+      sl2r = sl2 * (row < p.Lq && sok ? __ldg(p.sq + qs) : 1.f);
       skrow = p.sk + (static_cast<size_t>(x.b) * p.Hkv + x.hkv) * p.sk_pitch;
       skv = load_key_scales(skrow, (x.j0 + s) * kTileRows + 4 * lane, p.Lk);
     }
@@ -1017,8 +1144,8 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
       // step j + 1; each waits exactly for the hand-overs it is owed, so
       // arrivals and waits pair up per unit: min(n0, n1) on turn[1] and
       // min(n0 - 1, n1) on turn[0] (n0 > n1 can happen with a window).
-      const bool wait_turn = WINDOW ? (t == 0 ? (j >= 1 && j - 1 < x.n1) : j < x.n0)
-                                    : (t == 0 ? j >= 1 : j < x.n0);  // n0 <= n1 without a window
+      const bool wait_turn = kRanges ? (t == 0 ? (j >= 1 && j - 1 < x.n1) : j < x.n0)
+                                     : (t == 0 ? j >= 1 : j < x.n0);  // n0 <= n1 without ranges
       if (wait_turn) {
         bool ok_turn = mbar_wait(bar_turn_mine, tcnt & 1, abort_flag, kFaultSoftmaxTurn, p.timeout_ns);
         if (!__all_sync(0xffffffffu, ok_turn)) return;
@@ -1026,7 +1153,7 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
       }
 
       const float nref = -ref;
-      const bool hand_over = WINDOW ? (t == 0 ? j < x.n1 : j + 1 < x.n0) : (t == 0 || j + 1 < x.n0);
+      const bool hand_over = kRanges ? (t == 0 ? j < x.n1 : j + 1 < x.n0) : (t == 0 || j + 1 < x.n0);
       float sum[4] = {0.f, 0.f, 0.f, 0.f};
       // the masked variant is a separate instantiation so full tiles carry no
       // per-score compare/select. exp_tile holds warp-collective instructions
@@ -1057,7 +1184,8 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
       if (CAUSAL && n == 0) {
         // the tile sees no key of this split (the MMA issuer left O alone)
         const int row_e = x.r0 + t * kTileRows + r_in;
-        if (row_e < p.Lq) {
+        // site 5: the partial's row lies inside [n_splits, B, Hq, Lq]
+        if (row_e < p.Lq && ATTN_CHECK(x.split < p.n_splits && x.b < p.B && x.hq < p.Hq, 5)) {
           const size_t prow = ((static_cast<size_t>(x.split) * p.B + x.b) * p.Hq + x.hq) * p.Lq + row_e;
           float* dst = p.o_part + prow * D;
 #pragma unroll 1
@@ -1073,7 +1201,7 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
       // a row that sees no key of this split (causal) leaves O = 0, LSE = -inf
       const bool empty = !(l > 0.f);
       const float inv_l = empty ? 0.f : 1.f / l;
-      const bool in_range = row < p.Lq;
+      const bool in_range = row < p.Lq && ATTN_CHECK(x.split < p.n_splits && x.b < p.B && x.hq < p.Hq, 5);
       const size_t prow = ((static_cast<size_t>(x.split) * p.B + x.b) * p.Hq + x.hq) * p.Lq + row;
       float* dst = p.o_part + prow * D;
 #pragma unroll 1
@@ -1095,6 +1223,34 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
       continue;
     }
 
+    // pair split: slot 1 hands its row state to slot 0, which merges the two
+    // partial results (each relative to its own reference):
+    // O = (2^(ref0 - m) O_0 + 2^(ref1 - m) O_1) / (2^(ref0 - m) l_0 + 2^(ref1 - m) l_1),
+    // m = max(ref0, ref1); slot 1's O_1 is read from tensor memory (same lanes)
+    float a0 = 1.f, a1 = 0.f;  // the two slots' weights in the merge (pair split, slot 0)
+    if constexpr (PAIR) {
+      const uint32_t ml = sMl + r_in * 8;
+      if (t == 1) {
+        // a slot with no KV tile (one-tile range) leaves ref = -inf, l = 0: weight 0
+        asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(ml), "f"(ref), "f"(l) : "memory");
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bars + 8 * kBarMerge1);
+        continue;
+      }
+      bool okm = mbar_wait(bars + 8 * kBarMerge1, k & 1, abort_flag, kFaultSoftmaxOFull, p.timeout_ns);
+      if (x.n1 > 0)
+        okm = okm && mbar_wait(bars + 8 * (kBarOFull + 1), o1cnt & 1, abort_flag, kFaultSoftmaxOFull,
+                               p.timeout_ns);
+      if (!__all_sync(0xffffffffu, okm)) return;
+      float ref1, l1;
+      asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(ref1), "=f"(l1) : "r"(ml) : "memory");
+      const float m = fmaxf(ref, ref1);  // slot 0 always sees key 0: ref is finite
+      a0 = ex2_approx(ref - m);
+      a1 = x.n1 > 0 ? ex2_approx(ref1 - m) : 0.f;  // ex2(-inf) = 0 for rows slot 1 did not reach
+      l = a0 * l + a1 * l1;
+      ref = m;
+    }
+
     // epilogue: O / l to 16 bits into the shared staging tile (128-byte
     // swizzle, the layout of the TMA box), handed to the store warp; LSE.
     // The staging buffer alternates between the two query tiles: tile t fills
@@ -1107,13 +1263,15 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
     tc_fence_after_sync();
     const float inv_l = 1.f / l;
     const bool in_range = row < p.Lq;
+    const uint32_t tO1 = tmem + lane_bits + C::col_o(1);  // pair split: slot 1's O
 #pragma unroll 1
     for (int c = 0; c < D / 32; ++c) {
       uint32_t ov[32];
       tmem_ld_32x32b_x32(tO + 32 * c, ov);
       tmem_wait_ld_x32(ov);
       if constexpr (F8 == 2) {
-        if (p.sv != nullptr && 32 * c < p.d) {  // V's per-channel scales (columns past d stay 0)
+        // site 7: V's per-channel scales of this head lie inside [B, Hkv, d]
+        if (p.sv != nullptr && 32 * c < p.d && ATTN_CHECK(x.b < p.B && x.hkv < p.Hkv && 32 * c + 32 <= p.d, 7)) {
           const float4* sv4 =
               reinterpret_cast<const float4*>(p.sv + (static_cast<size_t>(x.b) * p.Hkv + x.hkv) * p.d + 32 * c);
 #pragma unroll
@@ -1126,6 +1284,16 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
           }
         }
       }
+      if constexpr (PAIR) {
+        if (x.n1 > 0) {  // add slot 1's partial, weighted
+          uint32_t o1[32];
+          tmem_ld_32x32b_x32(tO1 + 32 * c, o1);
+          tmem_wait_ld_x32(o1);
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            ov[e] = __float_as_uint(fmaf(__uint_as_float(o1[e]), a1, __uint_as_float(ov[e]) * a0));
+        }
+      }
       uint32_t pk[16];
 #pragma unroll
       for (int e = 0; e < 16; ++e)
@@ -1133,6 +1301,8 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
       // 32 columns = 4 units of 16 bytes in the 64-column box (c / 2); unit u of
       // row r sits at r * 128 + ((u ^ (r % 8)) * 16)
       const uint32_t box = stg + (c >> 1) * C::kChunkBytes + r_in * 128;
+      // site 8: the staged row lies inside the staging tile
+      if (!ATTN_CHECK((c >> 1) < C::kOChunks && r_in < kTileRows, 8)) continue;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const uint32_t unit = static_cast<uint32_t>(((c & 1) * 4 + e) ^ (r_in & 7));
@@ -1144,7 +1314,15 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) mbar_arrive(bar_stg_full);
-    if (p.lse != nullptr && in_range)
+    if constexpr (PAIR) {
+      // slot 1's O and row state have been read (tcgen05.wait::ld above): it may go on
+      if (x.n1 > 0) ++o1cnt;
+      tc_fence_before_sync();
+      if (lane == 0) mbar_arrive(bars + 8 * kBarMerged);
+    }
+    // site 4: the LSE index lies inside [B, Hq, Lq]
+    if (p.lse != nullptr && in_range &&
+        ATTN_CHECK(x.b < p.B && x.hq < p.Hq && row >= 0 && row < p.Lq, 4))
       p.lse[(static_cast<size_t>(x.b) * p.Hq + x.hq) * p.Lq + row] = (ref + log2f(l)) * kLn2;
   }
 }
@@ -1184,7 +1362,7 @@ __device__ __forceinline__ void mma_role_single(const int role, const FwdParams&
   int kv_it = 0, uit = 0, pcnt = 0;
   int sc = 0;  // KV tiles issued so far by this thread, over all units: tile sc uses S buffer sc % 2
   bool ok = true;
-  for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++uit) {
+  for (int u = cta_unit(0, p.n_units); u >= 0 && ok; u = cta_unit(++uit, p.n_units)) {
     const Unit x = decode_single<CAUSAL, SPLIT, WINDOW>(p, u);
     const int n = x.n0;
     if (role == 0) {
@@ -1270,7 +1448,8 @@ __device__ __forceinline__ void softmax_role_single(const FwdParams& p, uint32_t
   const uint32_t bar_o = bars + 8 * kBarOFull;
   const float sl2 = p.sl2;
   int sc = 0, ocnt = 0;
-  for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
+  int k = 0;
+  for (int u = cta_unit(0, p.n_units); u >= 0; u = cta_unit(++k, p.n_units)) {
     const Unit x = decode_single<CAUSAL, SPLIT, WINDOW>(p, u);
     const int n = x.n0;
     const int row = x.r0 + r_in;
@@ -1394,7 +1573,7 @@ __device__ __forceinline__ void softmax_role_single(const FwdParams& p, uint32_t
     if constexpr (SPLIT) {
       // float32 O / l and the LSE of this key range; a row (or the whole
       // tile) that sees no key of the range writes O = 0, LSE = -inf
-      const bool in_range = row < p.Lq;
+      const bool in_range = row < p.Lq && ATTN_CHECK(x.split < p.n_splits && x.b < p.B && x.hq < p.Hq, 5);
       const size_t prow = ((static_cast<size_t>(x.split) * p.B + x.b) * p.Hq + x.hq) * p.Lq + row;
       float* dst = p.o_part + prow * D;
       if (n == 0) {
@@ -1435,12 +1614,14 @@ __device__ __forceinline__ void softmax_role_single(const FwdParams& p, uint32_t
     const float inv_l = 1.f / l;
     const bool in_range = row < p.Lq;
     uint16_t* dst = static_cast<uint16_t*>(p.o) + ((static_cast<size_t>(x.b) * p.Lq + row) * p.Hq + x.hq) * D;
+    // site 9: the output row lies inside [B, Lq, Hq, D]
+    const bool dst_ok = ATTN_CHECK(x.b < p.B && x.hq < p.Hq && (row < p.Lq || !in_range), 9);
 #pragma unroll 1
     for (int c = 0; c < D / 32; ++c) {
       uint32_t ov[32];
       tmem_ld_32x32b_x32(tO + 32 * c, ov);
       tmem_wait_ld_x32(ov);
-      if (in_range) {
+      if (in_range && dst_ok) {
         if constexpr (F8 == 2) {
           if (p.sv != nullptr) {  // V's per-channel scales
             const float4* sv4 = reinterpret_cast<const float4*>(
@@ -1465,14 +1646,15 @@ __device__ __forceinline__ void softmax_role_single(const FwdParams& p, uint32_t
               make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
       }
     }
-    if (p.lse != nullptr && in_range)
+    if (p.lse != nullptr && in_range &&
+        ATTN_CHECK(x.b < p.B && x.hq < p.Hq && row >= 0 && row < p.Lq, 4))
       p.lse[(static_cast<size_t>(x.b) * p.Hq + x.hq) * p.Lq + row] = (ref + log2f(l)) * kLn2;
     // every TMEM read of O is complete (wait::ld) before the next unit's first
     // P V overwrites it: that MMA waits for this warpgroup's next P
   }
 }
 
-template <int D, bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW, int F8>
+template <int D, bool BF16, bool CAUSAL, bool SPLIT, bool WINDOW, int F8, bool PAIR = false>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
@@ -1510,6 +1692,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bars + 8 * (kBarDrain + 1), 1);
     mbar_init(bars + 8 * (kBarSFree + 0), 1);
     mbar_init(bars + 8 * (kBarSFree + 1), 1);
+    mbar_init(bars + 8 * kBarMerge1, kTileRows / 32);
+    mbar_init(bars + 8 * kBarMerged, kTileRows / 32);
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(bars + 8 * (kBarKvFull + s), 1);
       // d = 256: a K tile is read by the Q K^T issuer only, a V tile by the P V issuer only
@@ -1556,17 +1740,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp < 8) {
     regs_increase<kRegsSoftmax>();
-    softmax_role<D, BF16, CAUSAL, SPLIT, WINDOW, F8>(warp / 4, p, tmem, bars, sStg, sP, sbase + C::kOffSk,
-                                                     abort_flag);
+    uint32_t sMl = 0;  // pair split: slot 1's row state for the merge
+    if constexpr (PAIR) sMl = sbase + C::kOffMl;
+    softmax_role<D, BF16, CAUSAL, SPLIT, WINDOW, F8, PAIR>(warp / 4, p, tmem, bars, sStg, sP,
+                                                           sbase + C::kOffSk, sMl, abort_flag);
   } else {
     regs_decrease<kRegsProducer>();
     if (warp == 8) {
-      if (lane == 0) load_role<D, BF16, CAUSAL, SPLIT, WINDOW, F8>(&tm_q, &tm_k, &tm_v, p, sQ, sKV, bars, abort_flag);
+      if (lane == 0)
+        load_role<D, BF16, CAUSAL, SPLIT, WINDOW, F8, PAIR>(&tm_q, &tm_k, &tm_v, p, sQ, sKV, bars, abort_flag);
     } else if (warp == 9 || warp == 10) {
-      if (lane == 0) mma_role<D, BF16, CAUSAL, SPLIT, WINDOW, F8>(warp - 9, p, tmem, sQ, sKV, sP, bars,
-                                                                    abort_flag);
+      if (lane == 0)
+        mma_role<D, BF16, CAUSAL, SPLIT, WINDOW, F8, PAIR>(warp - 9, p, tmem, sQ, sKV, sP, bars, abort_flag);
     } else if (!SPLIT) {
-      if (lane == 0) store_role<D, BF16, CAUSAL, SPLIT, WINDOW, F8>(&tm_o, p, sStg, bars, abort_flag);
+      if (lane == 0) store_role<D, BF16, CAUSAL, SPLIT, WINDOW, F8, PAIR>(&tm_o, p, sStg, bars, abort_flag);
     }
   }
   __syncwarp();
@@ -1596,6 +1783,8 @@ __global__ void __launch_bounds__(256) split_merge_kernel(const float* __restric
   const int lane = threadIdx.x % 32;
   const long long rows = 1LL * B * Hq * Lq;
   if (w >= rows) return;
+  // site 10: this lane's columns lie inside the partial rows and the output row
+  if (!ATTN_CHECK(lane * kPer + kPer <= D && d_out <= D, 10)) return;
   // w = (b * Hq + hq) * Lq + i: the row index of the partial buffers
   const int i = static_cast<int>(w % Lq);
   const long long bh = w / Lq;
@@ -1846,7 +2035,7 @@ bool encode_e4m3_vt(CUtensorMap* map, const void* ptr, int B, int Lk, int pitch,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, bool BF16, bool CAUSAL, bool SPLIT = false, bool WINDOW = false, int F8 = 0>
+template <int D, bool BF16, bool CAUSAL, bool SPLIT = false, bool WINDOW = false, int F8 = 0, bool PAIR = false>
 int launch_fwd(const FwdParams& p, const void* q, const void* k, const void* v, int kv_rows, int grid,
                cudaStream_t stream) {
   using C = Cfg<D, F8>;
@@ -1871,7 +2060,7 @@ int launch_fwd(const FwdParams& p, const void* q, const void* k, const void* v, 
         !encode_bl_hd(&to, p.o, p.B, p.Lq, p.Hq, dt, BF16))
       return ATTN_ERR_CUDA;
   }
-  auto kern = attn_fwd_sm100_kernel<D, BF16, CAUSAL, SPLIT, WINDOW, F8>;
+  auto kern = attn_fwd_sm100_kernel<D, BF16, CAUSAL, SPLIT, WINDOW, F8, PAIR>;
   static std::once_flag attr_flags[kMaxDevices];
   static int attr_status[kMaxDevices];
   int dev = 0;
@@ -2027,6 +2216,19 @@ int attn_fwd_impl(const void* q, const void* k, const void* v, void* o, float* l
                 : launch_fwd<64, false, false, false, true>(p, q, k, v, kv_rows, grid, s);
   }
   const bool cz = causal == ATTN_MASK_CAUSAL;
+  if (cz && d <= 128 && n_units < di.num_sms) {
+    // pair split: one query tile per unit, its KV tiles shared by the CTA's
+    // two slots (causal units of unequal length that do not fill the SMs)
+    const long long n_tiles = (Lq + kTileRows - 1) / kTileRows;
+    p.n_pairs = static_cast<int>(n_tiles);
+    p.n_units = static_cast<int>(n_tiles * B * Hq);
+    const int pgrid = static_cast<int>(p.n_units < di.num_sms ? p.n_units : di.num_sms);
+    if (d == 128)
+      return bf16 ? launch_fwd<128, true, true, false, false, 0, true>(p, q, k, v, kv_rows, pgrid, s)
+                  : launch_fwd<128, false, true, false, false, 0, true>(p, q, k, v, kv_rows, pgrid, s);
+    return bf16 ? launch_fwd<64, true, true, false, false, 0, true>(p, q, k, v, kv_rows, pgrid, s)
+                : launch_fwd<64, false, true, false, false, 0, true>(p, q, k, v, kv_rows, pgrid, s);
+  }
   if (d == 256) {
     if (bf16) return cz ? launch_fwd<256, true, true>(p, q, k, v, kv_rows, grid, s) : launch_fwd<256, true, false>(p, q, k, v, kv_rows, grid, s);
     return cz ? launch_fwd<256, false, true>(p, q, k, v, kv_rows, grid, s) : launch_fwd<256, false, false>(p, q, k, v, kv_rows, grid, s);
@@ -2525,6 +2727,40 @@ int attn_device_fault(unsigned int* bits, int clear) {
   }
   *bits = b;
   return b ? ATTN_ERR_TIMEOUT : ATTN_OK;
+}
+
+}  // extern "C"
+
+// the debug site words of the other kernel files of the library
+namespace hasb_pro {
+unsigned int debug_site_read(bool clear);
+}
+namespace hasb_f8 {
+unsigned int debug_site_read(bool clear);
+}
+
+extern "C" {
+
+int attn_debug_fault_site(unsigned int* site, int clear) {
+  if (site == nullptr) return ATTN_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return ATTN_ERR_CUDA;
+  unsigned int a = 0;
+  if (cudaMemcpyFromSymbol(&a, g_debug_site, sizeof(a)) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (clear) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(g_debug_site, &zero, sizeof(zero)) != cudaSuccess) return ATTN_ERR_CUDA;
+  }
+  const unsigned int b = hasb_pro::debug_site_read(clear != 0), c = hasb_f8::debug_site_read(clear != 0);
+  *site = a != 0 ? a : (b != 0 ? b : c);
+  return ATTN_OK;
+}
+
+int attn_debug_build(void) {
+#ifdef ATTN_DEBUG
+  return 1;
+#else
+  return 0;
+#endif
 }
 
 int attn_selftest_mma(const void* q, const void* k, const void* v, float* s_out, float* o_out,

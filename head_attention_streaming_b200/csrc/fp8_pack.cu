@@ -18,6 +18,32 @@
 
 namespace hasb_f8 {
 
+// Debug build (-DATTN_DEBUG): the site number of the first index check that
+// failed in this file's kernels (0: none); a failed check skips the access.
+// In the release build a check is `true` and compiles away.
+__device__ unsigned int g_debug_site = 0;
+__device__ __forceinline__ bool debug_check(bool ok, unsigned int site) {
+  if (!ok) atomicCAS(&g_debug_site, 0u, site);
+  return ok;
+}
+#ifdef ATTN_DEBUG
+#define ATTN_CHECK(cond, site) (debug_check((cond), (site)))
+#else
+#define ATTN_CHECK(cond, site) true
+#endif
+
+// Reads (and with `clear` resets) this file's debug site word.
+unsigned int debug_site_read(bool clear) {
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_debug_site, sizeof(v)) != cudaSuccess) return 0;
+  if (clear) {
+    const unsigned int zero = 0;
+    (void)cudaMemcpyToSymbol(g_debug_site, &zero, sizeof(zero));
+  }
+  return v;
+}
+
+
 template <bool BF16>
 __device__ __forceinline__ float to_f32(uint16_t h) {
   if (BF16) return __uint_as_float(static_cast<uint32_t>(h) << 16);
@@ -72,6 +98,8 @@ __global__ void __launch_bounds__(256) cast_vt_kernel(const uint16_t* __restrict
     if (j >= Lk || c0 + cc >= d) continue;
     uint8_t* dst = vt + ((static_cast<size_t>(b) * H + h) * d + c0 + cc) * pitch + j;
     const uint32_t w = e4m3x2(tile[jj][cc], tile[jj + 1][cc]) | (e4m3x2(tile[jj + 2][cc], tile[jj + 3][cc]) << 16);
+    // site 31: the four keys stay inside the row's pitch, 4-byte aligned
+    if (!ATTN_CHECK(Lk <= pitch && (pitch & 3) == 0 && (j & 3) == 0, 31)) continue;
     if (j + 4 <= Lk) {
       *reinterpret_cast<uint32_t*>(dst) = w;  // pitch and j are multiples of 4
     } else {
@@ -127,7 +155,8 @@ __global__ void __launch_bounds__(256) quantize_tokens_kernel(const uint4* __res
                                   e4m3x2(g[4], g[5]) | (e4m3x2(g[6], g[7]) << 16));
     if (sub == 0) {
       const long long h = row % H, l = (row / H) % L, b = row / (static_cast<long long>(H) * L);
-      s[(b * H + h) * s_pitch + l] = sc;
+      // site 32: the token's scale lies inside its [pitch] row
+      if (ATTN_CHECK(l < s_pitch, 32)) s[(b * H + h) * s_pitch + l] = sc;
     }
   }
 }
@@ -188,6 +217,7 @@ __global__ void __launch_bounds__(256) quantize_vt_kernel(const uint16_t* __rest
     if (j >= Lk || c0 + cc >= d) continue;
     const float sc = slice_scale(__uint_as_float(amax_bits[static_cast<size_t>(bh) * d + c0 + cc]));
     uint8_t* dst = vt + ((static_cast<size_t>(b) * H + h) * d + c0 + cc) * pitch + j;
+    if (!ATTN_CHECK(Lk <= pitch && (pitch & 3) == 0 && (j & 3) == 0, 33)) continue;
     const uint32_t w = e4m3x2(__fdiv_rn(tile[jj][cc], sc), __fdiv_rn(tile[jj + 1][cc], sc)) |
                        (e4m3x2(__fdiv_rn(tile[jj + 2][cc], sc), __fdiv_rn(tile[jj + 3][cc], sc)) << 16);
     if (j + 4 <= Lk) {

@@ -32,6 +32,32 @@
 
 namespace hasb_pro {
 
+// Debug build (-DATTN_DEBUG): the site number of the first index check that
+// failed in this file's kernels (0: none); a failed check skips the access.
+// In the release build a check is `true` and compiles away.
+__device__ unsigned int g_debug_site = 0;
+__device__ __forceinline__ bool debug_check(bool ok, unsigned int site) {
+  if (!ok) atomicCAS(&g_debug_site, 0u, site);
+  return ok;
+}
+#ifdef ATTN_DEBUG
+#define ATTN_CHECK(cond, site) (debug_check((cond), (site)))
+#else
+#define ATTN_CHECK(cond, site) true
+#endif
+
+// Reads (and with `clear` resets) this file's debug site word.
+unsigned int debug_site_read(bool clear) {
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_debug_site, sizeof(v)) != cudaSuccess) return 0;
+  if (clear) {
+    const unsigned int zero = 0;
+    (void)cudaMemcpyToSymbol(g_debug_site, &zero, sizeof(zero));
+  }
+  return v;
+}
+
+
 constexpr int kWarps = 4;
 constexpr int kThreads = 32 * kWarps;
 
@@ -131,6 +157,10 @@ __device__ __forceinline__ void token_body(const ProParams& p, const ProTensor& 
   const bool raw = T.raw != 0;
   const int d = p.d;
   constexpr bool split = STYLE == ATTN_ROPE_SPLIT;
+  // site 21: the token and its output slot lie inside the tensor and the cache's rows
+  // (block-uniform: a failed check skips the whole token, barriers included)
+  if (!ATTN_CHECK(pos >= 0 && pos < T.L && pos < T.xstride && T.yoff >= 0 && T.yoff + pos < T.ystride, 21))
+    return;
   const int per_head = d / 16;                  // items per head
   const int sh = __ffs(per_head) - 1;           // log2(per_head)
   const int items = T.H * per_head;             // items of the token

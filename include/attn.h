@@ -253,8 +253,9 @@ int attn_fwd_splitkv_static(const void* q, const void* k, const void* v, void* o
  * so o and lse are bit-identical to one attn_fwd call. Host-to-device and
  * device-to-host copies run on two streams the library creates once per
  * device; the forwards run on `stream`, which waits for everything before the
- * call returns control of it: synchronize `stream` before reading o_host (use
- * pinned host memory: pageable memory serializes the copies). Calls on one
+ * call returns control of it: synchronize `stream` before reading o_host, and
+ * keep every host buffer allocated and unchanged until then (use pinned host
+ * memory: pageable memory serializes the copies). Calls on one
  * device are queued one at a time (a per-device lock while queueing).
  * Shapes, dtype, mask and errors as attn_fwd; additionally every host pointer
  * but lse_host must be non-NULL, and lse_host and lse_dev must be both NULL
@@ -392,6 +393,28 @@ const char* attn_status_string(int status);
  * when *bits != 0, else ATTN_OK (or ATTN_ERR_CUDA).
  */
 int attn_device_fault(unsigned int* bits, int clear);
+
+/*
+ * attn_debug_fault_site — synchronizes the current device, then returns in
+ * *site the site number of the first index check that failed in any kernel of
+ * this library since the last clear (0: none). Only the debug build
+ * (libattn_sm100_debug.so, compiled with -DATTN_DEBUG) checks: there every
+ * kernel tests the global-memory rows, shared-memory offsets and TMA
+ * coordinates it computes (tensor-memory columns are checked at compile time)
+ * against the shapes of the call before using them; a failed check sets
+ * bit 11 (0x800) of the fault word (attention kernels), records its site
+ * and skips that access, so the launch ends normally with a wrong result. In
+ * the release build *site is always 0. With clear != 0 the site words are
+ * reset. Returns ATTN_OK, ATTN_ERR_INVALID_ARG for a NULL site, or ATTN_ERR_CUDA.
+ * Sites: 1 Q tile coordinates, 2 K/V tile coordinates, 3 O store coordinates,
+ * 4 LSE index, 5 key-split partial row, 6 per-token scale rows, 7 V channel
+ * scales, 8 O staging row, 9 d = 256 output row, 10 key-split merge columns,
+ * 21 prologue token / cache slot, 31-33 FP8 cast and quantizer rows.
+ */
+int attn_debug_fault_site(unsigned int* site, int clear);
+
+/* 1 in the debug build (-DATTN_DEBUG), 0 in the release build. */
+int attn_debug_build(void);
 
 /*
  * attn_set_wait_timeout_ns — limit, in nanoseconds, of every device-side

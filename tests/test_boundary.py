@@ -43,7 +43,7 @@ def test_library_loads_and_exports_every_declared_symbol():
 
 
 def test_status_strings():
-    for st in range(5):
+    for st in range(6):
         assert hasb.status_string(st) != "unknown status"
     assert hasb.status_string(99) == "unknown status"
 

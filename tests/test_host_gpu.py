@@ -60,10 +60,14 @@ def test_host_path_without_lse_and_repeated_calls():
     q1, k1, v1 = inputs.make_qkv(1, 1500, 1500, 4, 4, 128, torch.bfloat16, seed=1)
     q2, k2, v2 = inputs.make_qkv(1, 1500, 1500, 4, 4, 128, torch.bfloat16, seed=2)
     bufs = [torch.empty_like(q1, device="cuda") for _ in range(4)]
-    outs = []
+    outs, keep = [], []
     for q, k, v in ((q1, k1, v1), (q2, k2, v2)):
         oh = torch.empty_like(q).pin_memory()
-        hasb.attn_fwd_host(q.pin_memory(), k.pin_memory(), v.pin_memory(), oh, None, *bufs, None)
+        # the host buffers must outlive the queued copies (a freed pinned block
+        # may be handed to the next pin_memory() before the copy has read it)
+        hin = [q.pin_memory(), k.pin_memory(), v.pin_memory()]
+        keep.append(hin)
+        hasb.attn_fwd_host(*hin, oh, None, *bufs, None)
         outs.append(oh)
     torch.cuda.current_stream().synchronize()
     for (q, k, v), oh in zip(((q1, k1, v1), (q2, k2, v2)), outs):
