@@ -57,6 +57,7 @@ sys.path.insert(0, ROOT)
 METRIC = "attention fwd TFLOPS on 1 B200 and % of dense BF16 tensor-core peak"
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "attn_fwd_video_20480x56x128.md")
+PROFILED_WORKLOAD = "video_20480x56x128"
 PROLOGUE_SUMMARY = os.path.join(ROOT, "profiles", "qk_prologue_dit_1785x40x128.md")
 FP8_SUMMARY = os.path.join(ROOT, "profiles", "attn_fwd_fp8_video_20480x56x128.md")
 KERNEL_SOURCES = [os.path.join(ROOT, "head_attention_streaming_b200", "csrc", f)
@@ -121,6 +122,15 @@ def profiled_traffic(summary=None, sources=None):
     if m_hash.group(1) != kernel_source_hash(sources):
         return None, "kernel changed since the ncu capture"
     return float(m_bytes.group(1)), "ncu"
+
+
+def attn_traffic(workload, split_used=None, window=None):
+    """DRAM bytes per launch for a 16-bit attention line: the committed capture
+    is of one video launch of the plain kernel, so it describes no other
+    workload and neither the key-split nor the windowed launch."""
+    if split_used is not None or window is not None or workload != PROFILED_WORKLOAD:
+        return None, "no ncu summary of this workload / variant"
+    return profiled_traffic()
 
 
 class ClockSampler:
@@ -872,7 +882,7 @@ def main():
     peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     launch_avg = statistics.mean(launch_ms)
     achieved = step_flops / (launch_avg * 1e-3) / 1e12
-    traffic, traffic_src = profiled_traffic()
+    traffic, traffic_src = attn_traffic(w.name, split_used, window)
     # The recipe's denominator: the burst GEMM peak for a kernel timed alone, the
     # sustained one (a seconds-long cuBLAS loop under the 1000 W cap) when the
     # timed region itself ran power-capped. Both fractions are reported.
@@ -880,8 +890,6 @@ def main():
     capped = ("sw_power_cap" in ci.get("reasons", []) and "sm_mhz" in ci
               and ci["sm_mhz"] < 0.97 * ci.get("sm_max_mhz", ci["sm_mhz"]))
     peak_used = peak_sus if capped else peak
-    if split_used is not None or window is not None:
-        traffic, traffic_src = None, "no ncu summary of this variant"
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak_used, "unit": "TFLOP/s",
                 "frac": achieved / peak_used, "traffic": traffic,
                 "peak_source": (f"bf16_tflops_sustained of {peak_src} (the timed region ran power-"
