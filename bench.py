@@ -435,6 +435,26 @@ def run_prologue(args):
     ms_step = ranks.max(statistics.mean(launch_ms), "cuda")
     value = job_rate(world, algo_bytes, ms_step) / 1e9
 
+    # the practical ceiling at this size: a device-to-device copy of the same
+    # Q and K (torch copy_, one cudaMemcpyAsync each), timed the same way
+    copy_ms = []
+    for _ in range(3):
+        oq.copy_(q)
+        ok.copy_(k)
+    for a, b in ev:
+        flush_buf.add_(1)
+        a.record(stream)
+        oq.copy_(q)
+        ok.copy_(k)
+        b.record(stream)
+        torch.cuda.synchronize()
+        copy_ms.append(a.elapsed_time(b))
+    copy_bytes = 2 * tensor_bytes  # read + write of Q and K
+    copy_ceiling = {"value": copy_bytes / (statistics.mean(copy_ms) * 1e-3) / 1e9, "unit": "GB/s",
+                    "ms": statistics.mean(copy_ms), "bytes": copy_bytes,
+                    "path": "device-to-device copy of Q and K (two cudaMemcpyAsync), L2 flushed before "
+                            "each step, CUDA events around the two copies (this rank)"}
+
     # end to end: pinned host Q, K in, prologue, Q, K out, every step
     qh, kh = q_cpu.pin_memory(), k_cpu.pin_memory()
     oqh, okh = torch.empty_like(qh).pin_memory(), torch.empty_like(kh).pin_memory()
@@ -468,7 +488,8 @@ def run_prologue(args):
                 "frac": achieved / peak, "traffic": traffic, "traffic_source": traffic_src,
                 "peak_source": f"hbm_gbs of {peak_src}", "kernel": "qk_prologue_kernel",
                 "algorithmic_bytes_per_launch": algo_bytes, "launch_ms_mean": statistics.mean(launch_ms),
-                "launch_ms_min": min(launch_ms), "launch_ms_max": max(launch_ms)}
+                "launch_ms_min": min(launch_ms), "launch_ms_max": max(launch_ms),
+                "copy_ceiling": copy_ceiling, "frac_of_copy": achieved / copy_ceiling["value"]}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
