@@ -906,8 +906,9 @@ def main():
         d2h = oh.numel() * oh.element_size() + lh.numel() * lh.element_size()
         e2e = {"value": job_rate(world, w.flops(), e_ms) / 1e12, "unit": "TFLOPS",
                "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "path": "attn_fwd_host: pinned host K, V -> device first, then query-row chunks whose "
-                       "copies in and out overlap the other chunks' forwards (two copy streams)"}
+               "path": "attn_fwd_host: pinned host buffers, chunks of at least 2 MB of Q (K, V and Q "
+                       "in, forward, O and LSE out) whose copies overlap the other chunks' forwards "
+                       "(two copy streams)"}
 
     peaks, peak_src = load_peaks()
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))

@@ -13,13 +13,13 @@ from .binding import (ATTN_ERR_CUDA, ATTN_ERR_INVALID_ARG, ATTN_ERR_SCRATCH_LIMI
                       attn_fwd_window, attn_fwd_fp8, attn_fwd_fp8_scaled, fp8_cast, fp8_cast_vt,
                       fp8_quantize_tokens, fp8_quantize_vt, qk_prologue, rope_after_cache,
                       splitkv_workspace_bytes, stream_update,
-                      debug_fault_site, device_fault, is_debug_build, lib, library_path, selftest_exp2,
+                      debug_fault_site, device_fault, host_chunks, is_debug_build, lib, library_path, selftest_exp2,
                       selftest_mma,
                       selftest_wait_timeout,
                       set_wait_timeout_ns, status_string)
 
 __all__ = ["attn_fwd", "attn_fwd_host", "AttnError", "lib", "library_path", "status_string", "device_fault",
-           "debug_fault_site", "is_debug_build",
+           "debug_fault_site", "host_chunks", "is_debug_build",
            "set_wait_timeout_ns", "selftest_mma", "selftest_exp2", "selftest_wait_timeout", "ATTN_OK",
            "ATTN_ERR_INVALID_ARG", "ATTN_ERR_UNSUPPORTED", "ATTN_ERR_CUDA", "ATTN_ERR_TIMEOUT",
            "ATTN_ERR_SCRATCH_LIMIT",

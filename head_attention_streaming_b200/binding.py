@@ -46,6 +46,7 @@ _SIGNATURES = {
                  [ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
     "attn_fwd_host": (ctypes.c_int, [ctypes.c_void_p] * 10 + [ctypes.c_int] * 6 +
                       [ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
+    "attn_host_chunks": (ctypes.c_int, [ctypes.c_int] * 4 + [ctypes.c_void_p]),
     "attn_qk_prologue": (ctypes.c_int, [ctypes.c_void_p] * 8 + [ctypes.c_int] * 7 +
                          [ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
     "attn_stream_update": (ctypes.c_int, [ctypes.c_void_p] * 10 + [ctypes.c_int] * 7 +
@@ -631,6 +632,16 @@ def attn_fwd_host(q_host, k_host, v_host, o_host, lse_host, q_dev, k_dev, v_dev,
                              DTYPE_CODES[q_host.dtype], _stream_handle(stream, q_dev.device))
     if st != ATTN_OK:
         raise AttnError(st, "attn_fwd_host")
+
+
+def host_chunks(B: int, Lq: int, Hq: int, d: int) -> list[tuple[int, int, int, int]]:
+    """The chunk plan of ``attn_fwd_host`` for these sizes: one (b0, nb, r0, n)
+    per chunk, rows [r0, r0 + n) of batches [b0, b0 + nb)."""
+    plan = (ctypes.c_int * 64)()
+    n = lib().attn_host_chunks(int(B), int(Lq), int(Hq), int(d), plan)
+    if n < 0:
+        raise AttnError(-n, "attn_host_chunks")
+    return [tuple(plan[4 * c:4 * c + 4]) for c in range(n)]
 
 
 def device_fault(clear: bool = True) -> int:

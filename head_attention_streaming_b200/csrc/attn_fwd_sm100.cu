@@ -2165,7 +2165,7 @@ int attn_fwd_validate(const void* q, const void* k, const void* v, const void* o
 int attn_fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Lq,
                   int Lk, int kv_rows, int Hq, int Hkv, int d, float scale, int causal, int kv_offset,
                   int dtype, void* stream, bool window = false, int win_left = -1,
-                  int win_right = -1) {
+                  int win_right = -1, int pair = -1) {
   // ---- argument contract (no CUDA call before it passes); a window uses the
   // offset rule of masks 1 and 2 (0 <= kv_offset, kv_offset + Lq <= Lk)
   const int valid = attn_fwd_validate(q, k, v, o, lse, B, Lq, Lk, Hq, Hkv, d, scale,
@@ -2216,7 +2216,10 @@ int attn_fwd_impl(const void* q, const void* k, const void* v, void* o, float* l
                 : launch_fwd<64, false, false, false, true>(p, q, k, v, kv_rows, grid, s);
   }
   const bool cz = causal == ATTN_MASK_CAUSAL;
-  if (cz && d <= 128 && n_units < di.num_sms) {
+  // pair < 0: decide from this launch's unit count; 0 / 1: the caller decided
+  // (a chunk of a larger call takes the whole call's choice, so its rows are
+  // computed exactly as the whole call computes them)
+  if (cz && d <= 128 && (pair < 0 ? n_units < di.num_sms : pair != 0)) {
     // pair split: one query tile per unit, its KV tiles shared by the CTA's
     // two slots (causal units of unequal length that do not fill the SMs)
     const long long n_tiles = (Lq + kTileRows - 1) / kTileRows;
@@ -2421,21 +2424,24 @@ int splitkv_run(const void* q, const void* k, const void* v, void* o, float* lse
 
 // ------------------------------------------------------ host-buffer pipeline
 
-// attn_fwd_host's copies overlap the attention: K and V go first, then the
-// query rows in chunks (per batch, a multiple of 256 rows, the kernel's unit,
-// so each chunk computes exactly what the whole call computes for its rows),
-// each chunk's forward starting once its Q has landed and its O (and LSE)
-// going back while the next chunk computes. Host-to-device copies run on one
-// internal stream, device-to-host copies on another, the forwards on the
-// caller's stream; events order them, and the caller's stream waits for the
-// last copy, so synchronizing it covers the whole call. The streams and
-// events are created once per device and reused (calls on one device are
-// serialized by a mutex while they are queued).
+// attn_fwd_host's copies overlap the attention. The call is cut into at most
+// kHostChunks chunks of at least kHostChunkMinBytes of Q each (a smaller one
+// would cost more in launches and copy calls than its overlap saves): whole
+// batches per chunk when there are at least as many batches as chunks, else
+// every batch cut into row ranges of whole 256-row pairs (the kernel's unit).
+// Per chunk the H2D stream copies the K and V of its batches (once per
+// batch) and its Q rows; its forward starts on the caller's stream once they
+// have landed, and its O (and LSE) go back on the D2H stream while the next
+// chunk computes. Events order the three streams, and the caller's stream
+// waits for the last copy, so synchronizing it covers the whole call. The
+// streams and events are created once per device and reused (calls on one
+// device are serialized by a mutex while they are queued).
 constexpr int kHostChunks = 16;
+constexpr size_t kHostChunkMinBytes = size_t(2) << 20;
 
 struct HostPipe {
   cudaStream_t h2d = nullptr, d2h = nullptr;
-  cudaEvent_t start = nullptr, kv_in = nullptr, done = nullptr;
+  cudaEvent_t start = nullptr, done = nullptr;
   cudaEvent_t q_in[kHostChunks] = {}, fwd_done[kHostChunks] = {};
   std::mutex m;
 };
@@ -2450,7 +2456,6 @@ HostPipe* host_pipe(int dev) {
     bool good = cudaStreamCreateWithFlags(&hp.h2d, cudaStreamNonBlocking) == cudaSuccess &&
                 cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking) == cudaSuccess &&
                 cudaEventCreateWithFlags(&hp.start, cudaEventDisableTiming) == cudaSuccess &&
-                cudaEventCreateWithFlags(&hp.kv_in, cudaEventDisableTiming) == cudaSuccess &&
                 cudaEventCreateWithFlags(&hp.done, cudaEventDisableTiming) == cudaSuccess;
     for (int c = 0; c < kHostChunks && good; ++c)
       good = cudaEventCreateWithFlags(&hp.q_in[c], cudaEventDisableTiming) == cudaSuccess &&
@@ -2460,50 +2465,77 @@ HostPipe* host_pipe(int dev) {
   return ok[dev] ? &pipes[dev] : nullptr;
 }
 
+// One chunk of attn_fwd_host: batches [b0, b0 + nb), query rows [r0, r0 + n)
+// of each (nb > 1 only with whole batches: r0 = 0, n = Lq).
+struct HostChunk {
+  int b0, nb, r0, n;
+};
+
+// The chunks of a call (host logic only; exported for tests through
+// attn_host_chunks). Returns their number, at most kHostChunks.
+int host_chunks(int B, int Lq, int Hq, int d, HostChunk* out) {
+  const size_t q_bytes = static_cast<size_t>(B) * Lq * Hq * d * 2;
+  const size_t by_size = q_bytes / kHostChunkMinBytes;
+  const int target = static_cast<int>(by_size < 1 ? 1 : (by_size > kHostChunks ? kHostChunks : by_size));
+  int n = 0;
+  if (target <= B) {
+    const int per = (B + target - 1) / target;  // whole batches per chunk
+    for (int b0 = 0; b0 < B; b0 += per) out[n++] = HostChunk{b0, std::min(per, B - b0), 0, Lq};
+  } else {
+    const long long per_b = target / B;        // >= 1 row ranges per batch
+    const long long want = (Lq + per_b - 1) / per_b;
+    const int rows = static_cast<int>(((want + 255) / 256) * 256);
+    for (int b = 0; b < B; ++b)
+      for (int r0 = 0; r0 < Lq; r0 += rows) out[n++] = HostChunk{b, 1, r0, std::min(rows, Lq - r0)};
+  }
+  return n;
+}
+
 int host_pipeline(HostPipe& hp, const void* q_host, const void* k_host, const void* v_host, void* o_host,
                   float* lse_host, void* q_dev, void* k_dev, void* v_dev, void* o_dev, float* lse_dev, int B,
                   int Lq, int Lk, int Hq, int Hkv, int d, float scale, int causal, int kv_offset, int dtype,
-                  cudaStream_t s) {
+                  cudaStream_t s, int num_sms) {
   const size_t row_bytes = 2ull * Hq * d;      // one query row of Q or O, all heads
-  const size_t kv_bytes = 2ull * B * Lk * Hkv * d;
-  // chunks of whole 256-row pairs, at most kHostChunks in all
-  const long long per_b = (kHostChunks + B - 1) / B;
-  const long long want = (Lq + per_b - 1) / per_b;
-  const int rows = static_cast<int>(((want + 255) / 256) * 256);
-  const int n_per_b = (Lq + rows - 1) / rows;
-  const int n_chunks = B * n_per_b;
-  if (n_chunks > kHostChunks) return ATTN_ERR_INVALID_ARG;  // cannot happen for B <= kHostChunks
+  const size_t kv_batch_bytes = 2ull * Lk * Hkv * d;
+  HostChunk ch[kHostChunks];
+  const int n_chunks = host_chunks(B, Lq, Hq, d, ch);
+  // the whole call's pair-split choice, taken by every chunk (bit-identical rows)
+  const long long units = static_cast<long long>(B) * Hq * ((Lq + 255) / 256);
+  const int pair = causal == ATTN_MASK_CAUSAL && d <= 128 && units < num_sms ? 1 : 0;
   const auto bad = [](cudaError_t e) { return e != cudaSuccess; };
   // streams: the copies wait for everything the caller queued before this call
   if (bad(cudaEventRecord(hp.start, s)) || bad(cudaStreamWaitEvent(hp.h2d, hp.start, 0)) ||
       bad(cudaStreamWaitEvent(hp.d2h, hp.start, 0)))
     return ATTN_ERR_CUDA;
-  if (bad(cudaMemcpyAsync(k_dev, k_host, kv_bytes, cudaMemcpyHostToDevice, hp.h2d)) ||
-      bad(cudaMemcpyAsync(v_dev, v_host, kv_bytes, cudaMemcpyHostToDevice, hp.h2d)) ||
-      bad(cudaEventRecord(hp.kv_in, hp.h2d)))
-    return ATTN_ERR_CUDA;
   for (int c = 0; c < n_chunks; ++c) {
-    const int b = c / n_per_b, r0 = (c % n_per_b) * rows;
-    const size_t off = (static_cast<size_t>(b) * Lq + r0) * row_bytes;
-    const size_t len = static_cast<size_t>(std::min(rows, Lq - r0)) * row_bytes;
+    const HostChunk& x = ch[c];
+    if (x.r0 == 0) {  // first chunk of its batches: their K and V
+      const size_t off = static_cast<size_t>(x.b0) * kv_batch_bytes, len = x.nb * kv_batch_bytes;
+      if (bad(cudaMemcpyAsync(static_cast<char*>(k_dev) + off, static_cast<const char*>(k_host) + off, len,
+                              cudaMemcpyHostToDevice, hp.h2d)) ||
+          bad(cudaMemcpyAsync(static_cast<char*>(v_dev) + off, static_cast<const char*>(v_host) + off, len,
+                              cudaMemcpyHostToDevice, hp.h2d)))
+        return ATTN_ERR_CUDA;
+    }
+    const size_t off = (static_cast<size_t>(x.b0) * Lq + x.r0) * row_bytes;
+    const size_t len = static_cast<size_t>(x.nb) * x.n * row_bytes;
     if (bad(cudaMemcpyAsync(static_cast<char*>(q_dev) + off, static_cast<const char*>(q_host) + off, len,
                             cudaMemcpyHostToDevice, hp.h2d)) ||
         bad(cudaEventRecord(hp.q_in[c], hp.h2d)))
       return ATTN_ERR_CUDA;
   }
-  if (bad(cudaStreamWaitEvent(s, hp.kv_in, 0))) return ATTN_ERR_CUDA;
   for (int c = 0; c < n_chunks; ++c) {
-    const int b = c / n_per_b, r0 = (c % n_per_b) * rows, n = std::min(rows, Lq - r0);
-    const size_t qo = (static_cast<size_t>(b) * Lq + r0) * Hq * d;          // elements
-    const size_t kvo = static_cast<size_t>(b) * Lk * Hkv * d;
-    // this chunk's LSE: [Hq, n] floats at the chunk's place in the batch's LSE area
-    float* lse_c = lse_dev == nullptr ? nullptr : lse_dev + static_cast<size_t>(b) * Hq * Lq +
-                                                      static_cast<size_t>(Hq) * r0;
+    const HostChunk& x = ch[c];
+    const size_t qo = (static_cast<size_t>(x.b0) * Lq + x.r0) * Hq * d;     // elements
+    const size_t kvo = static_cast<size_t>(x.b0) * Lk * Hkv * d;
+    // this chunk's LSE: [nb, Hq, n] floats at the chunk's place in its batches' LSE area
+    float* lse_c = lse_dev == nullptr ? nullptr : lse_dev + static_cast<size_t>(x.b0) * Hq * Lq +
+                                                      static_cast<size_t>(x.nb) * Hq * x.r0;
     // masks for a row range [r0, r0 + n): causal rows see j <= kv_offset + r (offset moves with r0);
     // chunk rows see every key below kv_offset + Lq (no mask over that key prefix)
     int mask = causal, off = kv_offset, lk = Lk;
     if (causal == ATTN_MASK_CAUSAL) {
-      off = kv_offset + r0;
+      off = kv_offset + x.r0;
     } else if (causal == ATTN_MASK_CHUNK) {
       mask = ATTN_MASK_NONE;
       off = 0;
@@ -2512,16 +2544,16 @@ int host_pipeline(HostPipe& hp, const void* q_host, const void* k_host, const vo
     if (bad(cudaStreamWaitEvent(s, hp.q_in[c], 0))) return ATTN_ERR_CUDA;
     const int st = attn_fwd_impl(static_cast<const uint16_t*>(q_dev) + qo, static_cast<const uint16_t*>(k_dev) + kvo,
                                  static_cast<const uint16_t*>(v_dev) + kvo, static_cast<uint16_t*>(o_dev) + qo, lse_c,
-                                 1, n, lk, Lk, Hq, Hkv, d, scale, mask, off, dtype, s);
+                                 x.nb, x.n, lk, Lk, Hq, Hkv, d, scale, mask, off, dtype, s, false, -1, -1, pair);
     if (st != ATTN_OK) return st;
     if (bad(cudaEventRecord(hp.fwd_done[c], s)) || bad(cudaStreamWaitEvent(hp.d2h, hp.fwd_done[c], 0)) ||
         bad(cudaMemcpyAsync(static_cast<char*>(o_host) + qo * 2, static_cast<const char*>(o_dev) + qo * 2,
-                            static_cast<size_t>(n) * row_bytes, cudaMemcpyDeviceToHost, hp.d2h)))
+                            static_cast<size_t>(x.nb) * x.n * row_bytes, cudaMemcpyDeviceToHost, hp.d2h)))
       return ATTN_ERR_CUDA;
     if (lse_host != nullptr &&
-        bad(cudaMemcpy2DAsync(lse_host + static_cast<size_t>(b) * Hq * Lq + r0, static_cast<size_t>(Lq) * 4,
-                              lse_c, static_cast<size_t>(n) * 4, static_cast<size_t>(n) * 4, Hq,
-                              cudaMemcpyDeviceToHost, hp.d2h)))
+        bad(cudaMemcpy2DAsync(lse_host + static_cast<size_t>(x.b0) * Hq * Lq + x.r0, static_cast<size_t>(Lq) * 4,
+                              lse_c, static_cast<size_t>(x.n) * 4, static_cast<size_t>(x.n) * 4,
+                              static_cast<size_t>(x.nb) * Hq, cudaMemcpyDeviceToHost, hp.d2h)))
       return ATTN_ERR_CUDA;
   }
   // the caller's stream covers the whole call
@@ -2709,11 +2741,26 @@ int attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, vo
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+  const DeviceInfo di = device_info(dev);
+  if (!di.ok) return ATTN_ERR_CUDA;
   HostPipe* hp = host_pipe(dev);
   if (hp == nullptr) return ATTN_ERR_CUDA;
   std::lock_guard<std::mutex> lock(hp->m);
   return host_pipeline(*hp, q_host, k_host, v_host, o_host, lse_host, q_dev, k_dev, v_dev, o_dev, lse_dev, B,
-                       Lq, Lk, Hq, Hkv, d, scale, causal, kv_offset, dtype, s);
+                       Lq, Lk, Hq, Hkv, d, scale, causal, kv_offset, dtype, s, di.num_sms);
+}
+
+int attn_host_chunks(int B, int Lq, int Hq, int d, int* plan) {
+  if (plan == nullptr || B < 1 || Lq < 1 || Hq < 1 || d < 1) return -ATTN_ERR_INVALID_ARG;
+  hasb::HostChunk ch[hasb::kHostChunks];
+  const int n = hasb::host_chunks(B, Lq, Hq, d, ch);
+  for (int c = 0; c < n; ++c) {
+    plan[4 * c] = ch[c].b0;
+    plan[4 * c + 1] = ch[c].nb;
+    plan[4 * c + 2] = ch[c].r0;
+    plan[4 * c + 3] = ch[c].n;
+  }
+  return n;
 }
 
 int attn_device_fault(unsigned int* bits, int clear) {

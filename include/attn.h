@@ -246,11 +246,15 @@ int attn_fwd_splitkv_static(const void* q, const void* k, const void* v, void* o
  * attn_fwd_host — the same forward for operands in host memory: copies q, k, v
  * from host to the caller's device buffers, runs attn_fwd, and copies o (and
  * lse when both lse pointers are given) back to host memory. The copies
- * overlap the computation: k and v go first, then q in chunks of whole
- * 256-row query pairs (per batch, at most 16 chunks in all); each chunk's
- * forward starts once its rows have landed and its o (and lse) rows go back
- * while the next chunk computes. Chunks hold whole work units of attn_fwd,
- * so o and lse are bit-identical to one attn_fwd call. Host-to-device and
+ * overlap the computation: the call is cut into at most 16 chunks with at
+ * least 2 MB of q each (attn_host_chunks gives the plan) — whole batches per
+ * chunk when there are at least as many batches as chunks, else each batch's
+ * query rows in ranges of whole 256-row pairs. Per chunk the k and v of its
+ * batches (first chunk of a batch only) and its q rows are copied in, its
+ * forward starts once they have landed, and its o (and lse) go back while the
+ * next chunk computes. Chunks hold whole work units of attn_fwd and every
+ * chunk takes the whole call's choice of schedule, so o and lse are
+ * bit-identical to one attn_fwd call. Host-to-device and
  * device-to-host copies run on two streams the library creates once per
  * device; the forwards run on `stream`, which waits for everything before the
  * call returns control of it: synchronize `stream` before reading o_host, and
@@ -261,13 +265,23 @@ int attn_fwd_splitkv_static(const void* q, const void* k, const void* v, void* o
  * but lse_host must be non-NULL, and lse_host and lse_dev must be both NULL
  * or both non-NULL. Device buffers are owned by the caller and sized as
  * attn_fwd's q, k, v, o, lse; lse_dev is used as scratch (after the call it
- * holds each chunk's [Hq, rows] block in chunk order, not the [B, Hq, Lq]
- * layout of lse_host).
+ * holds each chunk's [nb, Hq, rows] block at the chunk's place, which is the
+ * [B, Hq, Lq] layout of lse_host only when every chunk holds whole batches).
  */
 int attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, void* o_host,
                   float* lse_host, void* q_dev, void* k_dev, void* v_dev, void* o_dev,
                   float* lse_dev, int B, int Lq, int Lk, int Hq, int Hkv, int d, float scale,
                   int causal, int kv_offset, int dtype, void* stream);
+
+/*
+ * attn_host_chunks — the chunk plan attn_fwd_host uses for a call of these
+ * sizes (host logic only, no CUDA call). Writes 4 ints per chunk into plan
+ * (room for 16 chunks = 64 ints, caller-owned): first batch b0, batches nb,
+ * first query row r0, rows n; chunk c covers rows [r0, r0 + n) of batches
+ * [b0, b0 + nb). Returns the number of chunks (1..16), or
+ * -ATTN_ERR_INVALID_ARG for a NULL plan or a size below 1.
+ */
+int attn_host_chunks(int B, int Lq, int Hq, int d, int* plan);
 
 typedef enum {
   ATTN_NORM_NONE = 0,   /* Q and K unchanged */

@@ -1,9 +1,10 @@
 """attn_fwd_host on a B200: host operands in, the forward, host outputs back,
-with the copies overlapped with the computation in query-row chunks. Checked
-bit for bit against attn_fwd on device operands (the chunks are whole
-256-row work units, so nothing may differ) and against the FP64 oracle within
-the BF16 / FP16 bars, for several chunks per batch, ragged tails, B > 1, GQA
-and every mask mode."""
+with the copies overlapped with the computation in chunks (row ranges of one
+batch, or whole batches). Checked bit for bit against attn_fwd on device
+operands (chunks are whole 256-row work units and take the whole call's
+schedule, so nothing may differ) and against the FP64 oracle within the BF16 /
+FP16 bars, for several chunks per batch, ragged tails, whole-batch chunks,
+more than 16 batches, GQA and every mask mode."""
 
 from __future__ import annotations
 
@@ -28,13 +29,17 @@ def _device(cuda_ok):
 
 
 @pytest.mark.parametrize("B,Lq,Lk,Hq,Hkv,d,dtype,mask,off", [
-    (1, 3000, 3000, 2, 1, 128, torch.bfloat16, 0, 0),      # 12 chunks of 256 rows, ragged last
-    (2, 1100, 1500, 4, 2, 64, torch.float16, 1, 400),      # causal with an offset, two batches
-    (3, 513, 900, 2, 2, 128, torch.bfloat16, 2, 300),      # streaming chunk mask
+    (1, 5000, 5000, 16, 8, 128, torch.bfloat16, 0, 0),     # 7 row chunks of 768, ragged last
+    # causal, two batches of 2 row chunks: the whole call (192 units) runs
+    # unsplit, while a 1536-row chunk alone (48 units) would take the pair split
+    (2, 3000, 3400, 8, 4, 128, torch.float16, 1, 400),
+    (20, 512, 700, 8, 2, 128, torch.bfloat16, 2, 188),     # 10 chunks of 2 whole batches, chunk mask
+    (40, 200, 200, 8, 4, 64, torch.float16, 1, 0),         # more than 16 batches: chunks of 14, 14, 12
     (1, 100, 77, 1, 1, 128, torch.bfloat16, 0, 0),         # one chunk smaller than a tile
-    (1, 2048, 2048, 8, 8, 256, torch.bfloat16, 1, 0),      # head dim 256, causal
+    (1, 2048, 2048, 8, 8, 256, torch.bfloat16, 1, 0),      # head dim 256, causal, 4 row chunks
 ])
 def test_host_path_equals_device_call_and_oracle(B, Lq, Lk, Hq, Hkv, d, dtype, mask, off):
+    assert len(hasb.host_chunks(B, Lq, Hq, d)) == {5000: 7, 3000: 4, 512: 10, 200: 3, 100: 1, 2048: 4}[Lq]
     q, k, v = inputs.make_qkv(B, Lq, Lk, Hq, Hkv, d, dtype, seed=Lq + Lk + d)
     scale = 1.0 / math.sqrt(d)
     qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
