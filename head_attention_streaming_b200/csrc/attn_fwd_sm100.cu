@@ -580,11 +580,12 @@ __device__ __forceinline__ void load_role(const CUtensorMap* tm_q, const CUtenso
     if constexpr (PAIR) x = decode_pair(p, u);
     else if constexpr (D == 256) x = decode_single<CAUSAL, SPLIT, WINDOW>(p, u);
     else x = decode_unit<CAUSAL, SPLIT, WINDOW>(p, u);
-    // query tile t of the unit into its Q buffer, once the previous unit's
-    // last Q K^T of that tile is done
-    auto load_q = [&](int t) -> bool {
+    for (int t = 0; t < (D == 256 ? 1 : 2); ++t) {
       const uint32_t bq = bars + 8 * (kBarQEmpty + t);
-      if (!mbar_wait(bq, (uit & 1) ^ 1, abort_flag, kFaultLoadQEmpty, p.timeout_ns)) return false;
+      if (!mbar_wait(bq, (uit & 1) ^ 1, abort_flag, kFaultLoadQEmpty, p.timeout_ns)) {
+        aborted = true;
+        break;
+      }
       const uint32_t bf = bars + 8 * (kBarQFull + t);
       mbar_arrive_expect_tx(bf, C::kTileBytes);
       // site 1: the Q tile's head, batch and first row lie inside q
@@ -596,8 +597,7 @@ __device__ __forceinline__ void load_role(const CUtensorMap* tm_q, const CUtenso
         tma_load_4d(sQ + t * C::kTileBytes + c * C::kChunkBytes, tm_q, bf, c * (F8 != 0 ? 128 : 64), x.hq,
                     x.r0 + (PAIR ? 0 : t * kTileRows), x.b, pol_q);  // pair split: both slots, the same rows
       q_last[t] = uit & 1;
-      return true;
-    };
+    }
     // one K or V tile into its ring slot (ring index kv_it + 2 jj + kv); pair
     // split: stream position jj holds KV tile pair_tile(jj)
     auto load_one = [&](int jj, int kv) -> bool {
@@ -631,18 +631,7 @@ __device__ __forceinline__ void load_role(const CUtensorMap* tm_q, const CUtenso
       slot_last[slot] = idx;
       return true;
     };
-    // Q_0, then K_0, then Q_1: the first Q K^T needs only the first two, and
-    // at the start of a launch they come from HBM (1 % on the 1785-token DiT
-    // shape against loading both Q tiles first)
-    bool ok = load_q(0);
-    bool k0 = false;
-    if constexpr (D != 256) {
-      if (ok && x.nu > 0) {
-        ok = load_one(0, 0);
-        k0 = true;
-      }
-      ok = ok && load_q(1);
-    }
+    bool ok = !aborted;
     if constexpr (D == 256) {
       // K one tile ahead of V (K_0, K_1, V_0, K_2, V_1, ...): K and V have
       // slots of their own, so K_{j+1} (its slot free once Q K_j^T is done)
@@ -657,8 +646,7 @@ __device__ __forceinline__ void load_role(const CUtensorMap* tm_q, const CUtenso
       }
     } else {
       for (int j = 0; j < x.nu && ok; ++j)
-        for (int kv = 0; kv < 2 && ok; ++kv)
-          if (j != 0 || kv != 0 || !k0) ok = load_one(j, kv);
+        for (int kv = 0; kv < 2 && ok; ++kv) ok = load_one(j, kv);
     }
     if (!ok) aborted = true;
     else kv_it += 2 * x.nu;
