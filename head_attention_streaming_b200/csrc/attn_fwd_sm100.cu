@@ -580,6 +580,14 @@ __device__ __forceinline__ void load_role(const CUtensorMap* tm_q, const CUtenso
     if constexpr (PAIR) x = decode_pair(p, u);
     else if constexpr (D == 256) x = decode_single<CAUSAL, SPLIT, WINDOW>(p, u);
     else x = decode_unit<CAUSAL, SPLIT, WINDOW>(p, u);
+    // Both Q tiles before the unit's first K: the Q-empty wait of tile 1 (its
+    // last Q K^T of the previous unit issued) is what keeps tile 0 from
+    // starting the next unit while tile 1 still owes softmax turns in this
+    // one. Tile 0's first step of a unit hands the turn over without waiting
+    // for one, so with K_0 loaded ahead of Q_1 it can complete the turn
+    // barrier twice before tile 1 waits on it once, and tile 1's parity wait
+    // then misses a phase (measured: short key-split units stalled until the
+    // wait limit).
     for (int t = 0; t < (D == 256 ? 1 : 2); ++t) {
       const uint32_t bq = bars + 8 * (kBarQEmpty + t);
       if (!mbar_wait(bq, (uit & 1) ^ 1, abort_flag, kFaultLoadQEmpty, p.timeout_ns)) {

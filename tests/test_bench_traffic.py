@@ -31,3 +31,13 @@ def test_profiled_workload_uses_the_summary_only_while_the_sources_match():
         assert 1.0e9 < traffic < 1.4e9
     else:
         assert traffic is None and src == "kernel changed since the ncu capture"
+
+
+def test_digest_ignores_comments_but_not_code(tmp_path):
+    a, b, c = tmp_path / "a.cu", tmp_path / "b.cu", tmp_path / "c.cu"
+    a.write_text("int f(int x) {\n  return x + 1;\n}\n")
+    b.write_text("// the successor\nint f(int x) {  /* one more\n than x */\n\n  return x + 1;  // plus one\n}\n")
+    c.write_text("int f(int x) {\n  return x + 2;\n}\n")
+    h = lambda p: bench.kernel_source_hash([str(p)])
+    assert h(a) == h(b)
+    assert h(a) != h(c)
