@@ -580,20 +580,11 @@ __device__ __forceinline__ void load_role(const CUtensorMap* tm_q, const CUtenso
     if constexpr (PAIR) x = decode_pair(p, u);
     else if constexpr (D == 256) x = decode_single<CAUSAL, SPLIT, WINDOW>(p, u);
     else x = decode_unit<CAUSAL, SPLIT, WINDOW>(p, u);
-    // Both Q tiles before the unit's first K: the Q-empty wait of tile 1 (its
-    // last Q K^T of the previous unit issued) is what keeps tile 0 from
-    // starting the next unit while tile 1 still owes softmax turns in this
-    // one. Tile 0's first step of a unit hands the turn over without waiting
-    // for one, so with K_0 loaded ahead of Q_1 it can complete the turn
-    // barrier twice before tile 1 waits on it once, and tile 1's parity wait
-    // then misses a phase (measured: short key-split units stalled until the
-    // wait limit).
-    for (int t = 0; t < (D == 256 ? 1 : 2); ++t) {
+    // query tile t of the unit into its Q buffer, once the previous unit's
+    // last Q K^T of that tile is done
+    auto load_q = [&](int t) -> bool {
       const uint32_t bq = bars + 8 * (kBarQEmpty + t);
-      if (!mbar_wait(bq, (uit & 1) ^ 1, abort_flag, kFaultLoadQEmpty, p.timeout_ns)) {
-        aborted = true;
-        break;
-      }
+      if (!mbar_wait(bq, (uit & 1) ^ 1, abort_flag, kFaultLoadQEmpty, p.timeout_ns)) return false;
       const uint32_t bf = bars + 8 * (kBarQFull + t);
       mbar_arrive_expect_tx(bf, C::kTileBytes);
       // site 1: the Q tile's head, batch and first row lie inside q
@@ -605,7 +596,8 @@ __device__ __forceinline__ void load_role(const CUtensorMap* tm_q, const CUtenso
         tma_load_4d(sQ + t * C::kTileBytes + c * C::kChunkBytes, tm_q, bf, c * (F8 != 0 ? 128 : 64), x.hq,
                     x.r0 + (PAIR ? 0 : t * kTileRows), x.b, pol_q);  // pair split: both slots, the same rows
       q_last[t] = uit & 1;
-    }
+      return true;
+    };
     // one K or V tile into its ring slot (ring index kv_it + 2 jj + kv); pair
     // split: stream position jj holds KV tile pair_tile(jj)
     auto load_one = [&](int jj, int kv) -> bool {
@@ -639,7 +631,20 @@ __device__ __forceinline__ void load_role(const CUtensorMap* tm_q, const CUtenso
       slot_last[slot] = idx;
       return true;
     };
-    bool ok = !aborted;
+    // Q_0, then K_0, then Q_1: the first Q K^T needs only the first two, and
+    // at the start of a launch they come from HBM (1 % on the 1785-token DiT
+    // shape against loading both Q tiles first). Tile 0 may then enter a unit
+    // while tile 1 is still finishing the previous one; the softmax turn
+    // hand-back keeps their turns in order across units.
+    bool ok = load_q(0);
+    bool k0 = false;
+    if constexpr (D != 256) {
+      if (ok && x.nu > 0) {
+        ok = load_one(0, 0);
+        k0 = true;
+      }
+      ok = ok && load_q(1);
+    }
     if constexpr (D == 256) {
       // K one tile ahead of V (K_0, K_1, V_0, K_2, V_1, ...): K and V have
       // slots of their own, so K_{j+1} (its slot free once Q K_j^T is done)
@@ -654,7 +659,8 @@ __device__ __forceinline__ void load_role(const CUtensorMap* tm_q, const CUtenso
       }
     } else {
       for (int j = 0; j < x.nu && ok; ++j)
-        for (int kv = 0; kv < 2 && ok; ++kv) ok = load_one(j, kv);
+        for (int kv = 0; kv < 2 && ok; ++kv)
+          if (j != 0 || kv != 0 || !k0) ok = load_one(j, kv);
     }
     if (!ok) aborted = true;
     else kv_it += 2 * x.nu;
@@ -996,6 +1002,7 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
   const uint32_t bar_stg_free = bars + 8 * (kBarStgFree + t);
   const uint32_t stg = sstg;
   int tcnt = 0;
+  bool turn_back = false;  // tile 0: tile 1 owes the turn back from an earlier unit
   const int lane = threadIdx.x % 32;
   const uint32_t bar_o = bars + 8 * (kBarOFull + t);
   const float sl2 = p.sl2;
@@ -1028,6 +1035,10 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
       row_lo = p.win_left < 0 ? 0 : max(0, pos - p.win_left);
       row_lim = p.win_right < 0 ? p.Lk : min(p.Lk, pos + p.win_right + 1);
     }
+    // the unit ends with tile 0 handing the turn to tile 1 (tile 0 has steps and
+    // no more of them than tile 1): tile 1 then hands it back after its step
+    // n0 - 1, and tile 0 waits for that before its next unit's first step
+    const bool ret = x.n0 >= 1 && x.n0 <= x.n1;
     float ref = -INFINITY;  // scaled (log2) max the exponentials are taken against
     float l = 0.f;          // running row sum of exp2(s * sl2 - ref)
     // per-token scales: the row's Q scale joins the log2 factor; each lane
@@ -1149,19 +1160,26 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
       // the MUFU serves one of them at a time and each tile's GEMMs run on the
       // tensor core while the other tile computes. Step j of tile 0 hands over
       // if tile 1 has a step j; step j of tile 1 hands over if tile 0 has a
-      // step j + 1; each waits exactly for the hand-overs it is owed, so
-      // arrivals and waits pair up per unit: min(n0, n1) on turn[1] and
-      // min(n0 - 1, n1) on turn[0] (n0 > n1 can happen with a window).
-      const bool wait_turn = kRanges ? (t == 0 ? (j >= 1 && j - 1 < x.n1) : j < x.n0)
-                                     : (t == 0 ? j >= 1 : j < x.n0);  // n0 <= n1 without ranges
+      // step j + 1, and at the end of a unit that tile 0 ends by handing over
+      // (`ret`), tile 1's step n0 - 1 hands the turn back; each waits exactly
+      // for the hand-overs it is owed (tile 0's first step of a unit for the
+      // hand-back of an earlier one). So the hand-overs on each barrier
+      // alternate with its waits across units too, and no barrier can complete
+      // a phase twice before its waiter has seen the first (n0 > n1 can happen
+      // with a window: tile 0 then ends the unit by receiving the turn).
+      bool wait_turn = kRanges ? (t == 0 ? (j >= 1 && j - 1 < x.n1) : j < x.n0)
+                               : (t == 0 ? j >= 1 : j < x.n0);  // n0 <= n1 without ranges
+      if (t == 0 && j == 0) wait_turn = turn_back;
       if (wait_turn) {
         bool ok_turn = mbar_wait(bar_turn_mine, tcnt & 1, abort_flag, kFaultSoftmaxTurn, p.timeout_ns);
         if (!__all_sync(0xffffffffu, ok_turn)) return;
         ++tcnt;
       }
+      if (t == 0 && j == 0) turn_back = false;
 
       const float nref = -ref;
-      const bool hand_over = kRanges ? (t == 0 ? j < x.n1 : j + 1 < x.n0) : (t == 0 || j + 1 < x.n0);
+      const bool hand_over = (kRanges ? (t == 0 ? j < x.n1 : j + 1 < x.n0) : (t == 0 || j + 1 < x.n0)) ||
+                             (t == 1 && ret && j == x.n0 - 1);
       float sum[4] = {0.f, 0.f, 0.f, 0.f};
       // the masked variant is a separate instantiation so full tiles carry no
       // per-score compare/select. exp_tile holds warp-collective instructions
@@ -1185,6 +1203,7 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
       }
       l += (sum[0] + sum[1]) + (sum[2] + sum[3]);
     }
+    if (t == 0 && ret) turn_back = true;
 
     if constexpr (SPLIT) {
       // key split: float32 O / l of this split's keys, each thread its own
