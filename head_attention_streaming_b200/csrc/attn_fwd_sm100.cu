@@ -631,18 +631,25 @@ __device__ __forceinline__ void load_role(const CUtensorMap* tm_q, const CUtenso
       slot_last[slot] = idx;
       return true;
     };
-    // Q_0, then K_0, then Q_1: the first Q K^T needs only the first two, and
-    // at the start of a launch they come from HBM (1 % on the 1785-token DiT
-    // shape against loading both Q tiles first). Tile 0 may then enter a unit
-    // while tile 1 is still finishing the previous one; the softmax turn
-    // hand-back keeps their turns in order across units.
+    // 16-bit, two query tiles: Q_0, then K_0, then Q_1. The first Q K^T needs
+    // only the first two, and at the start of a launch they come from HBM
+    // (1 % on the 1785-token DiT shape against loading both Q tiles first).
+    // Tile 0 may then enter a unit while tile 1 is still finishing the
+    // previous one; the softmax turn hand-back keeps their turns in order.
+    // e4m3 loads both Q tiles first and has no hand-back (both measured
+    // slower there); then tile 0 cannot start a unit before tile 1 has issued
+    // its last Q K^T of the previous one, which leaves tile 1 far more time to
+    // take its last turn than tile 0 needs to offer the next.
+    constexpr bool kQ0K0Q1 = D != 256 && F8 == 0;
     bool ok = load_q(0);
     bool k0 = false;
-    if constexpr (D != 256) {
+    if constexpr (kQ0K0Q1) {
       if (ok && x.nu > 0) {
         ok = load_one(0, 0);
         k0 = true;
       }
+      ok = ok && load_q(1);
+    } else if constexpr (D != 256) {
       ok = ok && load_q(1);
     }
     if constexpr (D == 256) {
@@ -1010,6 +1017,9 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
   int o1cnt = 0;  // pair split: units whose slot 1 had KV tiles (phases of slot 1's O-full barrier)
   // (WINDOW || PAIR): per-slot KV ranges, tile 0 may have more steps than tile 1
   constexpr bool kRanges = WINDOW || PAIR;
+  // the turn hand-back at the end of a unit (16-bit; e4m3 relies on the
+  // loader's order, see load_role)
+  constexpr bool kHandBack = F8 == 0;
 
   int k = 0;
   for (int u = cta_unit(0, p.n_units); u >= 0; u = cta_unit(++k, p.n_units)) {
@@ -1038,7 +1048,7 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
     // the unit ends with tile 0 handing the turn to tile 1 (tile 0 has steps and
     // no more of them than tile 1): tile 1 then hands it back after its step
     // n0 - 1, and tile 0 waits for that before its next unit's first step
-    const bool ret = x.n0 >= 1 && x.n0 <= x.n1;
+    const bool ret = kHandBack && x.n0 >= 1 && x.n0 <= x.n1;
     float ref = -INFINITY;  // scaled (log2) max the exponentials are taken against
     float l = 0.f;          // running row sum of exp2(s * sl2 - ref)
     // per-token scales: the row's Q scale joins the log2 factor; each lane
@@ -1169,17 +1179,17 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
       // with a window: tile 0 then ends the unit by receiving the turn).
       bool wait_turn = kRanges ? (t == 0 ? (j >= 1 && j - 1 < x.n1) : j < x.n0)
                                : (t == 0 ? j >= 1 : j < x.n0);  // n0 <= n1 without ranges
-      if (t == 0 && j == 0) wait_turn = turn_back;
+      if (kHandBack && t == 0 && j == 0) wait_turn = turn_back;
       if (wait_turn) {
         bool ok_turn = mbar_wait(bar_turn_mine, tcnt & 1, abort_flag, kFaultSoftmaxTurn, p.timeout_ns);
         if (!__all_sync(0xffffffffu, ok_turn)) return;
         ++tcnt;
       }
-      if (t == 0 && j == 0) turn_back = false;
+      if (kHandBack && t == 0 && j == 0) turn_back = false;
 
       const float nref = -ref;
       const bool hand_over = (kRanges ? (t == 0 ? j < x.n1 : j + 1 < x.n0) : (t == 0 || j + 1 < x.n0)) ||
-                             (t == 1 && ret && j == x.n0 - 1);
+                             (kHandBack && t == 1 && ret && j == x.n0 - 1);
       float sum[4] = {0.f, 0.f, 0.f, 0.f};
       // the masked variant is a separate instantiation so full tiles carry no
       // per-score compare/select. exp_tile holds warp-collective instructions
@@ -1203,7 +1213,7 @@ __device__ __forceinline__ void softmax_role(const int t, const FwdParams& p, ui
       }
       l += (sum[0] + sum[1]) + (sum[2] + sum[3]);
     }
-    if (t == 0 && ret) turn_back = true;
+    if (kHandBack && t == 0 && ret) turn_back = true;
 
     if constexpr (SPLIT) {
       // key split: float32 O / l of this split's keys, each thread its own
